@@ -1,0 +1,391 @@
+"""Benchmark of the CSA2 FP4 sparse-decode step on B200.
+
+One step = one decode step of the workload's whole layer group: every Full
+layer appends its new tokens (K1) and indexes (K2 + K3), every Reindex layer
+indexes, every layer attends (K4 + K5). Default workload: batch 64, context
+131,072, one Full layer, top-k 2,048 (the 128K-context batch-64 decode).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle, timed on host cores
+
+Multi-GPU: one process per GPU (torchrun); every rank runs an independent
+replica with its own seed (weak scaling, no collective on the data path);
+time is the max over ranks. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from compressed_sparse_attention_quant_b200 import inputs  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+METRIC = "decode tokens/s and achieved HBM GB/s (% of 8 TB/s) for CSA2 FP4 sparse attn"
+KERNEL_SOURCES = ("csrc/common.cuh", "csrc/indexer.cuh", "csrc/topk.cuh")
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "compressed_sparse_attention_quant_b200", rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per indexer_topk call from a committed ncu summary, or None
+    when missing or taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", f"indexer_topk_{workload}.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        if d.get("kernel_source_hash") != kernel_source_hash():
+            return None
+        return float(d["dram_bytes_per_call"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=clocks.sm,clocks.max.sm,power.draw,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        try:
+            rows = [ln.split(",") for ln in open(self.path).read().strip().splitlines() if ln.strip()]
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = sorted(float(r[0]) for r in rows)
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[3:7]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": float(rows[0][1]), "samples": len(rows),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------- CPU oracle arm
+class OracleArm:
+    """The CPU oracle on sequences of the workload, generated on the CPU.
+
+    prepare() quantizes the owners' caches of the first n_seqs sequences
+    (set-up, untimed); step(b) times the oracle's per-step work for sequence
+    b: append quantization of the new tokens, indexer scores, top-k and
+    attention for every query token of every layer."""
+
+    def __init__(self, wl: inputs.Workload, n_seqs: int):
+        import oracle
+        self.oracle = oracle
+        self.wl = wl
+        self.own, self.src = oracle.plan(wl.modes)
+        self.seqs = list(range(min(n_seqs, wl.batch)))
+        self.caches = {}
+        self.layer_in = {}
+
+    def prepare(self):
+        o_, wl = self.oracle, self.wl
+        for b in self.seqs:
+            T = wl.lens()[b]
+            for o in set(self.own):
+                kv = torch.cat([r for _, r in inputs.kv_chunks(wl, o, b, "cpu")])
+                codes, scales = o_.quant_fp4(o_.bf16_bits(kv[:T - wl.q_tokens]))
+                self.caches[(o, b)] = (o_.bf16_bits(kv[T - wl.q_tokens:T]), codes, scales,
+                                       inputs.kidx_rows(wl, o, b, 0, T, "cpu").numpy(),
+                                       inputs.kidx_scale_rows(wl, o, b, 0, T, "cpu").numpy())
+        for li in range(len(wl.modes)):
+            self.layer_in[li] = (o_.bf16_bits(inputs.attn_query(wl, li, "cpu")),
+                                 o_.bf16_bits(inputs.swa_rows(wl, li, "cpu")),
+                                 inputs.idx_query(wl, li, "cpu").numpy(),
+                                 inputs.idx_weights(wl, li, "cpu").numpy())
+
+    def step(self, b: int) -> float:
+        import numpy as np
+        o_, wl = self.oracle, self.wl
+        T, Sq, W = wl.lens()[b], wl.q_tokens, inputs.WINDOW
+        scale = 1.0 / math.sqrt(576)
+        t0 = time.perf_counter()
+        cache = {}
+        results = {}
+        for li, mode in enumerate(wl.modes):
+            new_bits, codes, scales, kid, ks = self.caches[(self.own[li], b)]
+            if mode == "F":          # append: quantize the Sq new tokens into the cache
+                nc, ns = o_.quant_fp4(new_bits)
+                cache[li] = (np.concatenate([codes, nc]), np.concatenate([scales, ns]))
+            codes, scales = cache[self.own[li]]
+            q, swa, qi, w = (x[b] for x in self.layer_in[li])
+            for j in range(Sq):
+                pos = T - Sq + j
+                if mode in ("F", "R"):
+                    s = o_.indexer_scores(qi[j], w[j], kid[:pos + 1], ks[:pos + 1])
+                    idx = o_.topk(s, pos + 1, wl.top_k)
+                else:
+                    idx = results[(self.src[li], j)]
+                results[(li, j)] = idx
+                rows = [r for r in range(j, j + W) if T - (W + Sq - 1) + r >= 0]
+                o_.sparse_attn(q[j], codes, scales, idx, swa[rows], scale)
+        return time.perf_counter() - t0
+
+    def describe(self, n_timed: int) -> str:
+        wl = self.wl
+        return (f"{n_timed} sequence-steps over sequences {self.seqs} of {wl.batch}: "
+                f"{wl.q_tokens} query token(s) x {len(wl.modes)} layer(s), context {wl.lens()[0]}, "
+                f"top-k {wl.top_k}; single-threaded fp64 oracle; cache quantization untimed")
+
+
+def cpu_baseline(wl: inputs.Workload, n_seqs: int, budget_s: float) -> dict:
+    arm = OracleArm(wl, n_seqs)
+    arm.prepare()
+    spent, n = 0.0, 0
+    while spent < budget_s and n < 64:
+        spent += arm.step(arm.seqs[n % len(arm.seqs)])
+        n += 1
+    tok = n * wl.q_tokens
+    return {"value": tok / spent, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": arm.describe(n)}
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return                      # the oracle arm runs on rank 0 only
+    arm = OracleArm(wl, args.ref_seqs)
+    arm.prepare()
+    times = []
+    for i in range(args.warmup + args.steps):
+        t = arm.step(arm.seqs[i % len(arm.seqs)])
+        if i >= args.warmup:
+            times.append(t)
+    per_seq = sum(times) / len(times)
+    value = wl.q_tokens / per_seq
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": per_seq * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "q_tokens": wl.q_tokens,
+                       "context": wl.context, "top_k": wl.top_k, "modes": "".join(wl.modes),
+                       "step": "one sequence of the batch per step (bounded sample)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": arm.describe(len(times))},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- GPU arm
+def run_gpu(args, wl):
+    from compressed_sparse_attention_quant_b200 import lib, workload
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    # Each rank runs its own replica (different seed): weak scaling.
+    wl_r = inputs.Workload(**{**wl.__dict__, "seed": wl.seed + 1000 * rank}) if rank else wl
+    dw = workload.DeviceWorkload(wl_r, dev)
+    g = dw.group
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    acct = dw.algorithmic_bytes()
+    n_idx_calls = sum(1 for m in wl.modes if m in ("F", "R"))
+
+    # Timed step with events around the indexer_topk calls (the dominant op).
+    def step_instrumented(ev_pairs):
+        for li, mode in enumerate(g.modes):
+            cache = g.cache(li)
+            if mode == "F":
+                x_new, slots, kid, ks = dw.append[li]
+                lib.quant_kv_fp4(x_new, slots, cache, kid, ks)
+            if mode in ("F", "R"):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                lib.indexer_topk(dw.q_idx[li], dw.w[li], cache, dw.page_table, dw.seq_lens, g.k,
+                                 out=g._index[li], ws=g.ws_idx)
+                e1.record(stream)
+                ev_pairs.append((e0, e1))
+            lib.sparse_attn_decode(dw.q[li], cache, dw.page_table, dw.seq_lens, g.index(li), dw.swa[li],
+                                   g.scale, out=g.out[li], lse=g.lse[li], ws=g.ws_att)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step_instrumented([])
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+
+    launches0 = lib.launch_count()
+    step_events, idx_events = [], []
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            if not args.no_flush:
+                flush.zero_()                    # untimed: evict L2 between steps
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step_instrumented(idx_events)
+            e1.record(stream)
+            step_events.append((e0, e1))
+        torch.cuda.synchronize(dev)
+    launches = lib.launch_count() - launches0
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    step_ms = sum(a.elapsed_time(b) for a, b in step_events) / args.steps
+    idx_ms = sum(a.elapsed_time(b) for a, b in idx_events) / max(len(idx_events), 1)
+    status = lib.last_device_error()
+
+    # End to end: pinned host inputs -> device, step, device -> host outputs.
+    host_in = []
+    for li in range(len(g.modes)):
+        host_in.append((dw.q[li], dw.q[li].cpu().pin_memory()))
+        if li in dw.q_idx:
+            host_in.append((dw.q_idx[li], dw.q_idx[li].cpu().pin_memory()))
+            host_in.append((dw.w[li], dw.w[li].cpu().pin_memory()))
+        if li in dw.append:
+            for t in dw.append[li]:
+                host_in.append((t, t.cpu().pin_memory()))
+    host_out = [(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)) for t in g.out + g.lse]
+    h2d = sum(h.numel() * h.element_size() for _, h in host_in)
+    d2h = sum(h.numel() * h.element_size() for _, h in host_out)
+    e2e_events = []
+    for i in range(args.warmup + args.steps):
+        if not args.no_flush:
+            flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for d, h in host_in:
+            d.copy_(h, non_blocking=True)
+        dw.step()
+        for d, h in host_out:
+            h.copy_(d, non_blocking=True)
+        e1.record(stream)
+        if i >= args.warmup:
+            e2e_events.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_events) / args.steps
+
+    times = torch.tensor([step_ms, idx_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    step_ms, idx_ms, e2e_ms = times.tolist()
+
+    tokens_per_rank = wl.batch * wl.q_tokens
+    value = tokens_per_rank * world / (step_ms * 1e-3)
+    hbm, peak_kind = peaks()
+    idx_bytes = (acct["indexer"] + acct["topk_io"]) / max(n_idx_calls, 1)
+    achieved = idx_bytes / (idx_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(wl.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp4-e2m1/e4m3 cache, fp8 indexer, f16 mma, fp32 accum",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "q_tokens": wl.q_tokens, "context": wl.context,
+                   "top_k": wl.top_k, "modes": "".join(wl.modes), "parallelism": f"replicas x{world}",
+                   "l2": "inputs > L2; plus 256 MB L2 flush between steps (untimed)"
+                   if not args.no_flush else "inputs > L2, no flush"},
+        "step_hbm_gbs": acct["total"] / (step_ms * 1e-3) / 1e9,
+        "step_roofline_frac": acct["total"] / (step_ms * 1e-3) / 1e9 / hbm,
+        "roofline": {"bound": "hbm", "kernel": "csa2_indexer_topk (indexer score + exact top-k)",
+                     "achieved": achieved, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic, "ms_per_launch": idx_ms,
+                     "algorithmic_bytes_per_launch": idx_bytes},
+        "e2e": {"value": tokens_per_rank * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "device_status": lib.status_string(status),
+    }
+    clocks = clk.summary()
+    if clocks:
+        line["clocks"] = clocks
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.ref_seqs, args.cpu_budget)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
+    ap.add_argument("--workload", default="decode_b64_t128k", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--no-flush", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work (cpu_baseline)")
+    ap.add_argument("--ref-seqs", type=int, default=2, help="sequences the oracle arm prepares")
+    args = ap.parse_args()
+    wl = inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_gpu(args, wl)
+
+
+if __name__ == "__main__":
+    main()

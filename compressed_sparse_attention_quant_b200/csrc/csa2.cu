@@ -1,0 +1,330 @@
+// csa2.cu -- C-ABI entry points of the CSA2 FP4 sparse-decode library:
+// argument validation, workspace layout and kernel launches. The kernels are
+// in quant.cuh (K1), indexer.cuh (K2), topk.cuh (K3) and attn.cuh (K4/K5).
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "attn.cuh"
+#include "common.cuh"
+#include "indexer.cuh"
+#include "quant.cuh"
+#include "topk.cuh"
+
+namespace csa2 {
+
+std::atomic<uint64_t> g_launches{0};
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool ready = false;
+    int sm_count = 0;
+    int att_ctas_per_sm = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+cudaError_t device_info(DeviceInfo **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(indexer_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(sizeof(IdxSmem)));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(sizeof(AttSmem)));
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.att_ctas_per_sm, sparse_attn_kernel, kAttThreads,
+                                                          sizeof(AttSmem));
+        if (e != cudaSuccess) return e;
+        if (d.att_ctas_per_sm < 1) d.att_ctas_per_sm = 1;
+        d.ready = true;
+    }
+    *out = &d;
+    return cudaSuccess;
+}
+
+// ---------------------------------------------------------------- indexer / top-k workspace
+struct IdxLayout {
+    int64_t t_cap;
+    int n_chunks;
+    size_t scores, rows, hist, counters, chunk_cnt, chunk_off, total;
+};
+
+IdxLayout idx_layout(int B, int Sq, int max_pages) {
+    IdxLayout L{};
+    const int64_t R = static_cast<int64_t>(B) * Sq;
+    L.t_cap = static_cast<int64_t>(max_pages) * kPage;
+    L.n_chunks = static_cast<int>((L.t_cap + kTopkChunk - 1) / kTopkChunk);
+    size_t off = 0;
+    L.scores = off;    off = round_up(off + static_cast<size_t>(R * L.t_cap) * 4, 256);
+    L.rows = off;      off = round_up(off + static_cast<size_t>(R) * sizeof(TopkRow), 256);
+    L.hist = off;      off = round_up(off + static_cast<size_t>(R) * kTopkBins * 4, 256);
+    L.counters = off;  off = round_up(off + static_cast<size_t>(R) * 4, 256);
+    L.chunk_cnt = off; off = round_up(off + static_cast<size_t>(R) * L.n_chunks * 8, 256);
+    L.chunk_off = off; off = round_up(off + static_cast<size_t>(R) * L.n_chunks * 8, 256);
+    L.total = off;
+    return L;
+}
+
+// ---------------------------------------------------------------- attention splits
+struct AttSplit {
+    int n_splits;
+    int tiles_per_split;
+};
+
+// Split the (k + 128)-key list of each query row into S contiguous tile runs
+// so that R * S CTAs fill the machine: minimise waves x tiles per CTA, with a
+// small charge per split for writing and merging its partial.
+AttSplit att_split(int R, int k, int slots) {
+    const int n_tiles = (k + kWindow + kAttTile - 1) / kAttTile;
+    AttSplit best{1, n_tiles};
+    double best_cost = 1e30;
+    for (int s = 1; s <= n_tiles && s <= 64; ++s) {
+        const int tps = (n_tiles + s - 1) / s;
+        const int s_eff = (n_tiles + tps - 1) / tps;
+        const int64_t ctas = static_cast<int64_t>(R) * s_eff;
+        const int64_t waves = (ctas + slots - 1) / slots;
+        const double cost = static_cast<double>(waves) * tps + (s_eff > 1 ? 0.25 * s_eff : 0.0);
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = AttSplit{s_eff, tps};
+        }
+    }
+    return best;
+}
+
+size_t att_ws_bytes(int R, const AttSplit &sp) {
+    if (sp.n_splits <= 1) return 0;
+    const size_t po = round_up(static_cast<size_t>(R) * sp.n_splits * kHeads * kDim * 4, 256);
+    const size_t pm = round_up(static_cast<size_t>(R) * sp.n_splits * kHeads * 8, 256);
+    return po + pm;
+}
+
+csa2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
+
+bool cache_ok(const csa2_paged_cache *c) {
+    return c != nullptr && c->num_pages > 0 && c->num_pages <= (INT64_C(1) << 31) / kPage;
+}
+
+}  // namespace
+}  // namespace csa2
+
+using namespace csa2;
+
+extern "C" {
+
+csa2_status csa2_quant_kv_fp4(const void *x_bf16, int64_t n_tok, int dim, const int32_t *slot_mapping,
+                              const void *kidx_in, const float *kidx_scale_in,
+                              const csa2_paged_cache *cache, void *stream) {
+    if (n_tok < 0 || !cache_ok(cache)) return CSA2_ERR_INVALID_ARG;
+    if (dim != kDim) return CSA2_ERR_UNSUPPORTED;
+    if (n_tok == 0) return CSA2_OK;
+    if (!x_bf16 || !slot_mapping || !cache->kv_fp4 || !cache->kv_scale) return CSA2_ERR_INVALID_ARG;
+    if (kidx_in && (!kidx_scale_in || !cache->kidx || !cache->kidx_scale)) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(x_bf16, 16) || !aligned(cache->kv_fp4, 16) || !aligned(slot_mapping, 4) ||
+        (kidx_in && (!aligned(kidx_in, 16) || !aligned(cache->kidx, 16) || !aligned(cache->kidx_scale, 16) ||
+                     !aligned(kidx_scale_in, 4))))
+        return CSA2_ERR_ALIGNMENT;
+    if (n_tok > (INT64_C(1) << 31) * kQuantThreads / (kDim / kGroup)) return CSA2_ERR_INVALID_ARG;
+    return cuda_status(launch_quant_kv_fp4(x_bf16, n_tok, slot_mapping, kidx_in, kidx_scale_in, *cache,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+size_t csa2_indexer_topk_workspace_bytes(int B, int Sq, int max_pages, int k) {
+    (void)k;
+    if (B <= 0 || Sq <= 0 || max_pages <= 0) return 0;
+    return idx_layout(B, Sq, max_pages).total;
+}
+
+csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq, int idx_heads, int idx_dim,
+                              const csa2_paged_cache *cache, const int32_t *page_table, int max_pages,
+                              const int32_t *seq_lens, int k, int32_t *out_idx, void *ws, size_t ws_bytes,
+                              void *stream) {
+    if (idx_heads != kIdxHeads || idx_dim != kIdxDim) return CSA2_ERR_UNSUPPORTED;
+    if (B <= 0 || B > 65535 || Sq <= 0 || max_pages <= 0 || k <= 0 || k > 65536 || !cache_ok(cache))
+        return CSA2_ERR_INVALID_ARG;
+    if (Sq > 4) return CSA2_ERR_UNSUPPORTED;   // 4 query tokens x 4 heads = 16 MMA columns
+    if (static_cast<int64_t>(B) * Sq > 65535) return CSA2_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(max_pages) * kPage > (INT64_C(1) << 30)) return CSA2_ERR_UNSUPPORTED;
+    if (!q_idx || !w || !page_table || !seq_lens || !out_idx || !cache->kidx || !cache->kidx_scale)
+        return CSA2_ERR_INVALID_ARG;
+    if (!aligned(q_idx, 16) || !aligned(w, 16) || !aligned(cache->kidx, 16) || !aligned(cache->kidx_scale, 16) ||
+        !aligned(page_table, 4) || !aligned(seq_lens, 4) || !aligned(out_idx, 4))
+        return CSA2_ERR_ALIGNMENT;
+    const IdxLayout L = idx_layout(B, Sq, max_pages);
+    if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return CSA2_ERR_WORKSPACE;
+    DeviceInfo *dev = nullptr;
+    cudaError_t e = device_info(&dev);
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    float *scores = reinterpret_cast<float *>(base + L.scores);
+    TopkRow *rows = reinterpret_cast<TopkRow *>(base + L.rows);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(base + L.hist);
+    uint32_t *counters = reinterpret_cast<uint32_t *>(base + L.counters);
+    uint2 *chunk_cnt = reinterpret_cast<uint2 *>(base + L.chunk_cnt);
+    uint2 *chunk_off = reinterpret_cast<uint2 *>(base + L.chunk_off);
+    const int R = B * Sq;
+
+    dim3 g1((max_pages + kIdxPagesPerCta - 1) / kIdxPagesPerCta, B);
+    indexer_score_kernel<<<g1, kIdxThreads, sizeof(IdxSmem), st>>>(
+        static_cast<const uint8_t *>(q_idx), w, static_cast<const uint8_t *>(cache->kidx), cache->kidx_scale,
+        cache->num_pages, page_table, max_pages, seq_lens, Sq, k, scores, L.t_cap, rows, hist, counters);
+    count_launch();
+    dim3 g2(L.n_chunks, R);
+    for (int level = 0; level < 3; ++level) {
+        topk_radix_kernel<<<g2, kTopkThreads, 0, st>>>(scores, L.t_cap, rows, hist, counters, level);
+        count_launch();
+    }
+    topk_count_kernel<<<g2, kTopkThreads, 0, st>>>(scores, L.t_cap, rows, counters, chunk_cnt, chunk_off,
+                                                   L.n_chunks);
+    count_launch();
+    topk_write_kernel<<<g2, kTopkThreads, 0, st>>>(scores, L.t_cap, rows, chunk_off, L.n_chunks, k, out_idx);
+    count_launch();
+    return cuda_status(cudaGetLastError());
+}
+
+size_t csa2_sparse_attn_workspace_bytes(int B, int Sq, int k) {
+    if (B <= 0 || Sq <= 0 || k < 0) return 0;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return 0;
+    const int R = B * Sq;
+    return att_ws_bytes(R, att_split(R, k, dev->sm_count * dev->att_ctas_per_sm));
+}
+
+csa2_status csa2_sparse_attn_decode(const void *q_bf16, int B, int Sq, int H, int D,
+                                    const csa2_paged_cache *cache, const int32_t *page_table, int max_pages,
+                                    const int32_t *seq_lens, const int32_t *topk_idx, int k,
+                                    const void *swa_bf16, int W, float softmax_scale, float *out, float *lse,
+                                    void *ws, size_t ws_bytes, void *stream) {
+    if (H != kHeads || D != kDim || W != kWindow) return CSA2_ERR_UNSUPPORTED;
+    if (B <= 0 || Sq <= 0 || k < 0 || k > 65536 || max_pages <= 0 || !cache_ok(cache) ||
+        !std::isfinite(softmax_scale))
+        return CSA2_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(B) * Sq > 65535) return CSA2_ERR_UNSUPPORTED;
+    if (!q_bf16 || !page_table || !seq_lens || (k > 0 && !topk_idx) || !swa_bf16 || !out || !lse ||
+        !cache->kv_fp4 || !cache->kv_scale)
+        return CSA2_ERR_INVALID_ARG;
+    if (!aligned(q_bf16, 16) || !aligned(swa_bf16, 16) || !aligned(cache->kv_fp4, 16) ||
+        !aligned(cache->kv_scale, 4) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(page_table, 4) ||
+        !aligned(seq_lens, 4) || (topk_idx && !aligned(topk_idx, 4)))
+        return CSA2_ERR_ALIGNMENT;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return CSA2_ERR_CUDA;
+    const int R = B * Sq;
+    const AttSplit sp = att_split(R, k, dev->sm_count * dev->att_ctas_per_sm);
+    const size_t need = att_ws_bytes(R, sp);
+    if (need > 0 && (!ws || !aligned(ws, 256) || ws_bytes < need)) return CSA2_ERR_WORKSPACE;
+
+    AttParams P;
+    P.q = static_cast<const __nv_bfloat16 *>(q_bf16);
+    P.kv_fp4 = static_cast<const uint8_t *>(cache->kv_fp4);
+    P.kv_scale = static_cast<const uint8_t *>(cache->kv_scale);
+    P.num_pages = cache->num_pages;
+    P.page_table = page_table;
+    P.max_pages = max_pages;
+    P.seq_lens = seq_lens;
+    P.topk_idx = topk_idx;
+    P.k = k;
+    P.swa = static_cast<const __nv_bfloat16 *>(swa_bf16);
+    P.Sq = Sq;
+    P.scale_log2 = softmax_scale * 1.4426950408889634f;
+    P.out = out;
+    P.lse = lse;
+    P.n_splits = sp.n_splits;
+    P.tiles_per_split = sp.tiles_per_split;
+    P.part_o = nullptr;
+    P.part_ml = nullptr;
+    if (sp.n_splits > 1) {
+        uint8_t *base = static_cast<uint8_t *>(ws);
+        P.part_o = reinterpret_cast<float *>(base);
+        P.part_ml = reinterpret_cast<float2 *>(
+            base + round_up(static_cast<size_t>(R) * sp.n_splits * kHeads * kDim * 4, 256));
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    dim3 grid(sp.n_splits, R);
+    sparse_attn_kernel<<<grid, kAttThreads, sizeof(AttSmem), st>>>(P);
+    count_launch();
+    if (sp.n_splits > 1) {
+        attn_merge_kernel<<<R, kMergeThreads, sp.n_splits * kHeads * sizeof(float), st>>>(
+            P.part_o, P.part_ml, sp.n_splits, out, lse);
+        count_launch();
+    }
+    return cuda_status(cudaGetLastError());
+}
+
+csa2_status csa2_plan(const int *modes, int n_layers, int *kv_owner, int *index_src) {
+    if (!modes || !kv_owner || !index_src || n_layers <= 0) return CSA2_ERR_INVALID_ARG;
+    int owner = -1;
+    for (int i = 0; i < n_layers; ++i) {
+        switch (modes[i]) {
+            case CSA2_FULL:
+                owner = i;
+                kv_owner[i] = i;
+                index_src[i] = i;
+                break;
+            case CSA2_REINDEX:
+                if (owner < 0) return CSA2_ERR_BAD_PLAN;
+                kv_owner[i] = owner;
+                index_src[i] = i;
+                break;
+            case CSA2_REUSE:
+                if (owner < 0) return CSA2_ERR_BAD_PLAN;
+                kv_owner[i] = owner;
+                index_src[i] = owner;
+                break;
+            default:
+                return CSA2_ERR_BAD_PLAN;
+        }
+    }
+    return CSA2_OK;
+}
+
+csa2_status csa2_last_device_error(void *stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned int v = 0u;
+    if (cudaMemcpyFromSymbolAsync(&v, g_status, sizeof v, 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return CSA2_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return CSA2_ERR_CUDA;
+    if (v != 0u) {
+        const unsigned int zero = 0u;
+        if (cudaMemcpyToSymbolAsync(g_status, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+            return CSA2_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return CSA2_ERR_CUDA;
+    }
+    if (v & kStatusTimeout) return CSA2_ERR_TIMEOUT;
+    if (v & kStatusBounds) return CSA2_ERR_DEVICE_BOUNDS;
+    return CSA2_OK;
+}
+
+const char *csa2_status_string(csa2_status s) {
+    switch (s) {
+        case CSA2_OK: return "CSA2_OK";
+        case CSA2_ERR_INVALID_ARG: return "CSA2_ERR_INVALID_ARG";
+        case CSA2_ERR_UNSUPPORTED: return "CSA2_ERR_UNSUPPORTED";
+        case CSA2_ERR_CUDA: return "CSA2_ERR_CUDA";
+        case CSA2_ERR_BAD_PLAN: return "CSA2_ERR_BAD_PLAN";
+        case CSA2_ERR_TIMEOUT: return "CSA2_ERR_TIMEOUT";
+        case CSA2_ERR_DEVICE_BOUNDS: return "CSA2_ERR_DEVICE_BOUNDS";
+        case CSA2_ERR_WORKSPACE: return "CSA2_ERR_WORKSPACE";
+        case CSA2_ERR_ALIGNMENT: return "CSA2_ERR_ALIGNMENT";
+    }
+    return "CSA2_ERR_UNKNOWN";
+}
+
+uint64_t csa2_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

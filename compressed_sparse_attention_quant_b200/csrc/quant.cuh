@@ -1,0 +1,98 @@
+// quant.cuh -- K1: FP4 (E2M1 + E4M3 per 16 channels) quantize-and-append of
+// the global KV latent into the paged cache. Page "DeepSeek 首次公开
+// V4.1-Flash 技术报告…" (neodrop.ai), architecture part 3: the main KV cache
+// is E2M1 with one E4M3 scale for every 16 channels.
+//
+// One thread per (token, 16-channel group): two 16-byte loads of bf16, the
+// group max by compares, the scale by IEEE division and the hardware
+// round-to-nearest-even satfinite FP8 conversion, the codes by exact
+// compares against the scaled E2M1 midpoints, one 8-byte store of packed
+// codes and one scale byte. HBM-bound: 32 B read + 9 B written per group.
+#pragma once
+
+#include "common.cuh"
+
+namespace csa2 {
+
+constexpr int kQuantThreads = 256;
+
+__global__ void __launch_bounds__(kQuantThreads)
+quant_kv_fp4_kernel(const uint4 *__restrict__ x, int64_t n_tok, const int32_t *__restrict__ slots,
+                    const uint4 *__restrict__ kidx_in, const float *__restrict__ ksig_in,
+                    uint8_t *__restrict__ kv_fp4, uint8_t *__restrict__ kv_scale,
+                    uint8_t *__restrict__ kidx, float *__restrict__ kidx_scale, int64_t n_slots) {
+    constexpr int kGroups = kDim / kGroup;  // 36
+    const int64_t gid = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
+    const int64_t tok = gid / kGroups;
+    const int g = static_cast<int>(gid - tok * kGroups);
+    if (tok >= n_tok) return;
+    const int32_t slot = slots[tok];
+    if (slot < 0) return;                       // padding token: nothing to append
+    if (static_cast<int64_t>(slot) >= n_slots) {
+        if (g == 0) flag_status(kStatusBounds);
+        return;
+    }
+
+    // 16 bf16 channels = two 16-byte vectors.
+    const uint4 v0 = x[(tok * kGroups + g) * 2 + 0];
+    const uint4 v1 = x[(tok * kGroups + g) * 2 + 1];
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float f[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+
+    // Scale: E4M3FN nearest to amax/6. The fp32 quotient is correctly rounded
+    // and cannot cross an E4M3 midpoint (amax has 8 significant bits, 6 x a
+    // midpoint at most 7), so RNE of the fp32 quotient is RNE of the exact one.
+    const float t = __fdiv_rn(amax, 6.0f);
+    const __nv_fp8_storage_t sb = __nv_cvt_float_to_fp8(t, __NV_SATFINITE, __NV_E4M3);
+    const float s = __half2float(__half(__nv_cvt_fp8_to_halfraw(sb, __NV_E4M3)));
+
+    // Codes: count the E2M1 midpoints below |x|/s, comparing |x| with s * mu
+    // (exact in fp32). Ties go to the even code: strict '>' at midpoints that
+    // sit above an even code, '>=' at those above an odd code.
+    const float m0 = s * 0.25f, m1 = s * 0.75f, m2 = s * 1.25f, m3 = s * 1.75f;
+    const float m4 = s * 2.5f, m5 = s * 3.5f, m6 = s * 5.0f;
+    uint32_t packed[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float a = fabsf(f[i]);
+        uint32_t c = (a > m0) + (a >= m1) + (a > m2) + (a >= m3) + (a > m4) + (a >= m5) + (a > m6);
+        if (s == 0.0f) c = 0u;
+        if (c != 0u && f[i] < 0.0f) c |= 8u;
+        packed[i >> 3] |= c << (4 * (i & 7));
+    }
+    const int64_t sl = slot;
+    *reinterpret_cast<uint2 *>(kv_fp4 + sl * kFp4Bytes + g * 8) = make_uint2(packed[0], packed[1]);
+    kv_scale[sl * kScaleBytes + g] = sb;
+
+    // Indexer key and scale of the token, in the page's core-matrix order.
+    if (kidx_in != nullptr && g < 4) {
+        const int64_t page = sl / kPage;
+        const int r = static_cast<int>(sl % kPage);
+        uint8_t *dst = kidx + page * kKidxPageBytes + (r >> 3) * 512 + g * 128 + (r & 7) * 16;
+        *reinterpret_cast<uint4 *>(dst) = kidx_in[tok * 4 + g];
+        if (g == 0) kidx_scale[sl] = ksig_in[tok];
+    }
+}
+
+inline cudaError_t launch_quant_kv_fp4(const void *x, int64_t n_tok, const int32_t *slots,
+                                       const void *kidx_in, const float *ksig_in,
+                                       const csa2_paged_cache &c, cudaStream_t stream) {
+    const int64_t threads = n_tok * (kDim / kGroup);
+    const int64_t blocks = (threads + kQuantThreads - 1) / kQuantThreads;
+    quant_kv_fp4_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
+        static_cast<const uint4 *>(x), n_tok, slots, static_cast<const uint4 *>(kidx_in), ksig_in,
+        static_cast<uint8_t *>(c.kv_fp4), static_cast<uint8_t *>(c.kv_scale),
+        static_cast<uint8_t *>(c.kidx), c.kidx_scale, c.num_pages * kPage);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -1,0 +1,237 @@
+/*
+ * csa2.h -- C ABI of the B200 (sm_100a) library for the decode step of
+ * Compressed Sparse Attention 2 (CSA2) over an FP4 main KV cache.
+ *
+ * Sources of the operations (page title and section):
+ *   [NEO] "DeepSeek 首次公开 V4.1-Flash 技术报告：552B 骨干参数与 CED 架构亮相，
+ *         KV 缓存压至 890 字节" (neodrop.ai), architecture part 2 (CSA2: three
+ *         static modes, shared main KV and indexer keys, top-K indices reused
+ *         across layers) and part 3 (FP4 main KV: E2M1 with one E4M3 scale per
+ *         16 channels).
+ *   [ZUL] "DeepSeek V4 1-Flash 架构拆解：CED、CSA2、Engram、mHC 与 DSp"
+ *         (blog.zulogic.cn), section 3 (mode table; KV owner -> compressed
+ *         global KV, indexer K / scale, top-K metadata -> consumer layers) and
+ *         section 4 (a 128-token sliding window kept per layer beside the
+ *         global KV).
+ *   [INF] "DeepSeek V4.1 Flash 模型架構與推論優化技術規格剖析" (infernews.com),
+ *         section 2 (the window is the last 128 tokens) and the section-4 table
+ *         (row "CSA 2": modes Full / Index / Reuse).
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers marked "device" point to device memory owned by the caller. The
+ *     library allocates nothing and never synchronises on the compute calls.
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream. Compute calls only enqueue work on it.
+ *   - Argument errors (null pointers, unsupported shapes, misaligned buffers,
+ *     too small workspace) are detected on the host before anything is
+ *     enqueued and returned as a status; nothing runs in that case.
+ *   - Out-of-range values found in device data (page-table entries, slot ids,
+ *     top-k indices, sequence lengths) never fault: the kernel skips the
+ *     access, treats the entry as empty and sets a sticky device status word
+ *     that csa2_last_device_error() reads and clears.
+ *   - The shapes are fixed by the model: 16 query heads, 576 latent channels
+ *     (keys = values), 4 indexer heads of 64 channels, a 128-token window and
+ *     64-token KV pages. Other values return CSA2_ERR_UNSUPPORTED.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Static per-layer mode ([NEO part 2], [ZUL section 3]). */
+typedef enum csa2_mode {
+    CSA2_FULL = 0,     /* builds KV + indexer state, selects top-k, attends   */
+    CSA2_REINDEX = 1,  /* reuses the owner's KV; recomputes its own top-k      */
+    CSA2_REUSE = 2     /* reuses the owner's KV and an earlier layer's top-k   */
+} csa2_mode;
+
+typedef enum csa2_status {
+    CSA2_OK = 0,
+    CSA2_ERR_INVALID_ARG = 1,   /* null / negative / inconsistent argument      */
+    CSA2_ERR_UNSUPPORTED = 2,   /* shape other than the fixed model shape       */
+    CSA2_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed         */
+    CSA2_ERR_BAD_PLAN = 4,      /* a layer has no Full layer before it          */
+    CSA2_ERR_TIMEOUT = 5,       /* a bounded device wait gave up                */
+    CSA2_ERR_DEVICE_BOUNDS = 6, /* device data held an out-of-range entry       */
+    CSA2_ERR_WORKSPACE = 7,     /* workspace missing, misaligned or too small   */
+    CSA2_ERR_ALIGNMENT = 8      /* a device buffer is not 16-byte aligned       */
+} csa2_status;
+
+enum {
+    CSA2_HEADS = 16,            /* attention heads per query token              */
+    CSA2_DIM = 576,             /* latent channels (keys = values)              */
+    CSA2_IDX_HEADS = 4,         /* indexer heads                                */
+    CSA2_IDX_DIM = 64,          /* indexer channels                             */
+    CSA2_WINDOW = 128,          /* sliding window ([ZUL section 4], [INF 2])    */
+    CSA2_PAGE_TOKENS = 64,      /* tokens per KV page                           */
+    CSA2_GROUP = 16,            /* channels per E4M3 scale ([NEO part 3])       */
+    CSA2_FP4_BYTES = 288,       /* packed E2M1 bytes per token (576 / 2)        */
+    CSA2_SCALE_BYTES = 36,      /* E4M3 scale bytes per token (576 / 16)        */
+    CSA2_KIDX_PAGE_BYTES = 4096 /* indexer-key bytes per page (64 x 64)         */
+};
+
+/*
+ * The paged global cache of one KV owner (a Full layer), shared by the layers
+ * that alias it ([ZUL section 3]: KV owner -> compressed global KV, indexer
+ * K / scale). A host-side struct of caller-owned device arrays, all indexed
+ * by physical page p in [0, num_pages), each 16-byte aligned:
+ *
+ *   kv_fp4     uint8 [num_pages][64][288]  token-major; byte j of a token
+ *              holds channel 2j in its low nibble and channel 2j+1 in its high
+ *              nibble, each an E2M1 code (bit 3 sign, bits 2..0 magnitude code
+ *              of {0, .5, 1, 1.5, 2, 3, 4, 6}).
+ *   kv_scale   uint8 [num_pages][64][36]   E4M3FN scale of channels 16g..16g+15.
+ *   kidx       uint8 [num_pages][4096]     indexer keys, E4M3FN, 64 tokens x 64
+ *              channels; byte of (token t, channel c) at
+ *              (t/8)*512 + (c/16)*128 + (t%8)*16 + c%16
+ *              (8x16-byte core matrices, the no-swizzle K-major operand layout
+ *              of the tensor cores).
+ *   kidx_scale float [num_pages][64]       per-token indexer scale sigma.
+ *
+ * Token t of sequence b lives in physical page page_table[b][t / 64], row
+ * t % 64. A slot id is page * 64 + row.
+ */
+typedef struct csa2_paged_cache {
+    void *kv_fp4;
+    void *kv_scale;
+    void *kidx;
+    float *kidx_scale;
+    int64_t num_pages;
+} csa2_paged_cache;
+
+/*
+ * csa2_quant_kv_fp4 -- Full mode: quantize and append KV ([NEO part 3]).
+ *
+ * For each of n_tok tokens, quantizes the bf16 latent x[t][0..dim) to FP4:
+ * per 16-channel group, s = the E4M3FN value nearest to max|x|/6 (ties to
+ * even, saturated at 448; 0 when max|x|/6 is at most 2^-10), and each channel
+ * gets the E2M1 code nearest to |x|/s (ties to even code, saturated at 6,
+ * canonical +0 for a zero magnitude; all codes 0 when s = 0). Inputs must be
+ * finite. The packed bytes and scales go to slot slot_mapping[t] of `cache`.
+ * When kidx_in is not NULL the token's indexer key kidx_in[t][0..64) (E4M3FN)
+ * and its scale kidx_scale_in[t] are written to the same slot too.
+ *
+ *   x_bf16        device bf16 [n_tok][dim], dim must be 576
+ *   slot_mapping  device int32 [n_tok]; a negative slot skips the token; a
+ *                 slot >= 64 * num_pages sets CSA2_ERR_DEVICE_BOUNDS
+ *   kidx_in       device uint8 [n_tok][64] or NULL
+ *   kidx_scale_in device float [n_tok] (required iff kidx_in != NULL)
+ *   cache         host pointer to the destination cache descriptor
+ * Bulk cache builds (n_tok = B*T) and per-step appends (n_tok = B*Sq) use the
+ * same call.
+ */
+csa2_status csa2_quant_kv_fp4(const void *x_bf16, int64_t n_tok, int dim,
+                              const int32_t *slot_mapping,
+                              const void *kidx_in, const float *kidx_scale_in,
+                              const csa2_paged_cache *cache, void *stream);
+
+/*
+ * csa2_indexer_topk -- Full / Reindex: score every cached token with the
+ * lightweight indexer and select the top-k ([NEO part 2] "Top-K sparse
+ * addressing index"; [ZUL section 3]: Full and Reindex compute the index).
+ *
+ * Query token j of sequence b sits at position pos = seq_lens[b] - Sq + j and
+ * scores every cached token t <= pos:
+ *     s_t = sum_h w[b][j][h] * max(0, sigma_t * <q[b][j][h], k_t>)
+ * (the pages print no formula; this is the DSA-style reading). The dot
+ * product of E4M3 operands runs on the FP8 tensor cores with fp32
+ * accumulation. out_idx[b][j] receives the k tokens with the largest s_t, ties
+ * to the lower token index, in ascending token order; when pos + 1 < k the
+ * remaining entries are -1. The selection is exact and deterministic for the
+ * scores as computed; scores equal the mathematical value whenever every
+ * partial sum is exact in fp32 (e.g. small-integer E4M3 inputs, sigma = 1 and
+ * power-of-two weights).
+ *
+ *   q_idx       device uint8 [B][Sq][4][64] (E4M3FN)
+ *   w           device float [B][Sq][4]
+ *   cache       host pointer; reads kidx and kidx_scale of the owner's cache
+ *   page_table  device int32 [B][max_pages]
+ *   seq_lens    device int32 [B]; Sq <= seq_lens[b] <= 64 * max_pages
+ *   k           1 <= k <= 65536
+ *   out_idx     device int32 [B][Sq][k]
+ *   ws          device workspace of at least csa2_indexer_topk_workspace_bytes()
+ *               bytes, 256-byte aligned; contents need no initialisation and
+ *               are clobbered.
+ */
+size_t csa2_indexer_topk_workspace_bytes(int B, int Sq, int max_pages, int k);
+csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq,
+                              int idx_heads, int idx_dim,
+                              const csa2_paged_cache *cache,
+                              const int32_t *page_table, int max_pages,
+                              const int32_t *seq_lens, int k, int32_t *out_idx,
+                              void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * csa2_sparse_attn_decode -- all modes: attention over the selected FP4
+ * entries plus the sliding window ([NEO part 2]; [ZUL section 4]).
+ *
+ * For query token j of sequence b (position pos = seq_lens[b] - Sq + j) and
+ * head h, the keys are the dequantized cache entries topk_idx[b][j][i] >= 0
+ * together with the window rows j .. j+W-1 of swa[b] (row r holds position
+ * seq_lens[b] - (W + Sq - 1) + r; rows at negative positions are skipped).
+ * The same vectors are the values. One softmax over their union:
+ *     out[b][j][h] = sum_i softmax_i(scale * <q, key_i>) * key_i
+ *     lse[b][j][h] = log sum_i exp(scale * <q, key_i>)
+ * With no key at all out = 0 and lse = -inf. Dequantized FP4 entries are
+ * exact in f16; q and the window rows are rounded to f16 (exact for
+ * magnitudes in [2^-14, 65504]); probabilities are rounded to f16; all sums
+ * accumulate in fp32.
+ *
+ *   q_bf16      device bf16 [B][Sq][16][576]
+ *   cache       host pointer; reads kv_fp4 and kv_scale of the owner's cache
+ *   page_table  device int32 [B][max_pages];   seq_lens device int32 [B]
+ *   topk_idx    device int32 [B][Sq][k] (k may be 0: window only)
+ *   swa_bf16    device bf16 [B][W + Sq - 1][576], W must be 128
+ *   out         device float [B][Sq][16][576];  lse device float [B][Sq][16]
+ *   ws          device workspace of csa2_sparse_attn_workspace_bytes() bytes,
+ *               256-byte aligned (split-k partials); clobbered.
+ */
+size_t csa2_sparse_attn_workspace_bytes(int B, int Sq, int k);
+csa2_status csa2_sparse_attn_decode(const void *q_bf16, int B, int Sq, int H,
+                                    int D, const csa2_paged_cache *cache,
+                                    const int32_t *page_table, int max_pages,
+                                    const int32_t *seq_lens,
+                                    const int32_t *topk_idx, int k,
+                                    const void *swa_bf16, int W,
+                                    float softmax_scale, float *out, float *lse,
+                                    void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * csa2_plan -- ownership bookkeeping for a group of layers ([ZUL section 3]:
+ * KV owner layer -> consumer layers; [NEO part 2]: KV, indexer keys and top-K
+ * indices shared across layers). Host-only, no device work.
+ *
+ * Fills, for each layer i, kv_owner[i] = the Full layer whose cache it reads
+ * (itself for a Full layer, else the nearest Full layer before it) and
+ * index_src[i] = the layer whose top-k indices it attends with (itself for
+ * Full and Reindex; the nearest Full layer before it for Reuse). Returns
+ * CSA2_ERR_BAD_PLAN when a Reindex or Reuse layer has no Full layer before
+ * it or a mode is unknown, CSA2_ERR_INVALID_ARG for null pointers.
+ */
+csa2_status csa2_plan(const int *modes, int n_layers, int *kv_owner,
+                      int *index_src);
+
+/*
+ * csa2_last_device_error -- synchronises `stream`, then reads and clears the
+ * sticky device status word of the current device. Returns CSA2_OK,
+ * CSA2_ERR_DEVICE_BOUNDS or CSA2_ERR_TIMEOUT (the first set, in that order of
+ * precedence: timeout first), or CSA2_ERR_CUDA if the synchronisation failed.
+ * A diagnostic call: it blocks the host.
+ */
+csa2_status csa2_last_device_error(void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *csa2_status_string(csa2_status s);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t csa2_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA2_H */
