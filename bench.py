@@ -70,52 +70,63 @@ def recorded_traffic(workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    """SM clocks and clock-event reasons sampled by NVML from a thread while
+    the timed region runs (a few ms between samples)."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+    # NVML clocks-event-reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, gpu_index: int, period_s: float = 0.002):
+        self.gpu, self.period = gpu_index, period_s
+        self.samples = []
+        self.max_mhz = None
+        self.ok = False
 
     def __enter__(self):
+        import threading
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=clocks.sm,clocks.max.sm,power.draw,"
-                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
-                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[self.gpu]) if vis and vis.split(",")[0].isdigit() else self.gpu
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
         except Exception:
-            self.proc = None
+            return self
+        self.stop = threading.Event()
+
+        def run():
+            while not self.stop.is_set():
+                try:
+                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                    rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((mhz, rs))
+                except Exception:
+                    pass
+                time.sleep(self.period)
+
+        self.th = threading.Thread(target=run, daemon=True)
+        self.th.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            self.f.close()
+        if self.ok:
+            self.stop.set()
+            self.th.join(timeout=5)
 
     def summary(self):
-        if self.proc is None:
+        if not self.ok or not self.samples:
             return None
-        try:
-            rows = [ln.split(",") for ln in open(self.path).read().strip().splitlines() if ln.strip()]
-        except Exception:
-            return None
-        if not rows:
-            return None
-        sm = sorted(float(r[0]) for r in rows)
+        sm = sorted(m for m, _ in self.samples)
         reasons = set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            for name, v in zip(names, r[3:7]):
-                if v.strip().lower() == "active":
+        for _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
                     reasons.add(name)
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": float(rows[0][1]), "samples": len(rows),
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
                 "reasons": sorted(reasons)}
 
 
@@ -276,6 +287,8 @@ def run_gpu(args, wl):
     launches0 = lib.launch_count()
     step_events, idx_events = [], []
     with ClockSampler(local) as clk:
+        time.sleep(0.01)                          # first clock sample before the region
+        torch.cuda.nvtx.range_push("timed")
         for _ in range(args.steps):
             if not args.no_flush:
                 flush.zero_()                    # untimed: evict L2 between steps
@@ -285,6 +298,7 @@ def run_gpu(args, wl):
             step_instrumented(idx_events)
             e1.record(stream)
             step_events.append((e0, e1))
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize(dev)
     launches = lib.launch_count() - launches0
     if dist:
@@ -374,13 +388,14 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
-    ap.add_argument("--workload", default="decode_b64_t128k", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--workload", default="decode_b64_t128k",
+                    choices=sorted(inputs.WORKLOADS) + sorted(inputs.PROFILE_WORKLOADS))
     ap.add_argument("--no-flush", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work (cpu_baseline)")
     ap.add_argument("--ref-seqs", type=int, default=2, help="sequences the oracle arm prepares")
     args = ap.parse_args()
-    wl = inputs.WORKLOADS[args.workload]
+    wl = {**inputs.WORKLOADS, **inputs.PROFILE_WORKLOADS}[args.workload]
     if args.impl == "reference":
         run_reference(args, wl)
     else:

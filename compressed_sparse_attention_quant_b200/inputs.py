@@ -92,6 +92,12 @@ WORKLOADS = {
     "long_b4_t1m": Workload("long_b4_t1m", 4, 1, 1048576, 2048, ("F",), True, True, 4),
 }
 
+# A quarter-batch copy of the 128K decode workload (same per-sequence shape,
+# indexer keys still > L2) for profiler captures that must stay small.
+PROFILE_WORKLOADS = {
+    "decode_b16_t128k": Workload("decode_b16_t128k", 16, 1, 131072, 2048, ("F",), True, False, 2),
+}
+
 
 def _seed(*parts) -> int:
     h = hashlib.sha256(repr(parts).encode()).digest()
