@@ -266,6 +266,44 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int B, int Sq, int H, in
     return cuda_status(cudaGetLastError());
 }
 
+}  // extern "C"
+
+namespace csa2 {
+namespace {
+
+// Library-owned scratch of csa2_sparse_attn_decode_noalloc: one copy per GPU
+// that loads the library, alive until process exit.
+__device__ __align__(256) uint8_t g_noalloc_scratch[CSA2_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch per device, looked up on the first call
+// with that device current (the host-side symbol is not a device address).
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+}  // namespace
+}  // namespace csa2
+
+extern "C" {
+
+csa2_status csa2_sparse_attn_decode_noalloc(const void *q_bf16, int B, int Sq, int H, int D,
+                                            const csa2_paged_cache *cache, const int32_t *page_table,
+                                            int max_pages, const int32_t *seq_lens, const int32_t *topk_idx,
+                                            int k, const void *swa_bf16, int W, float softmax_scale, float *out,
+                                            float *lse, void *stream) {
+    if (B <= 0 || Sq <= 0 || k < 0) return CSA2_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CSA2_ERR_CUDA;
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return CSA2_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    const size_t need = csa2_sparse_attn_workspace_bytes(B, Sq, k);
+    if (need > CSA2_NOALLOC_SCRATCH_BYTES) return CSA2_ERR_WORKSPACE;
+    return csa2_sparse_attn_decode(q_bf16, B, Sq, H, D, cache, page_table, max_pages, seq_lens, topk_idx, k,
+                                   swa_bf16, W, softmax_scale, out, lse, g_noalloc_ptr[dev],
+                                   CSA2_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 csa2_status csa2_plan(const int *modes, int n_layers, int *kv_owner, int *index_src) {
     if (!modes || !kv_owner || !index_src || n_layers <= 0) return CSA2_ERR_INVALID_ARG;
     int owner = -1;

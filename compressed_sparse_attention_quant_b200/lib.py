@@ -25,7 +25,8 @@ STATUS = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_UNSUPPORTED", 3:
 
 # Every function include/csa2.h declares (checked by the CPU test suite).
 EXPORTS = ("csa2_quant_kv_fp4", "csa2_indexer_topk_workspace_bytes", "csa2_indexer_topk",
-           "csa2_sparse_attn_workspace_bytes", "csa2_sparse_attn_decode", "csa2_plan",
+           "csa2_sparse_attn_workspace_bytes", "csa2_sparse_attn_decode",
+           "csa2_sparse_attn_decode_noalloc", "csa2_plan",
            "csa2_last_device_error", "csa2_status_string", "csa2_launch_count")
 
 
@@ -58,6 +59,8 @@ def _load():
         "csa2_sparse_attn_workspace_bytes": (_sz, [_i32, _i32, _i32]),
         "csa2_sparse_attn_decode": (_i32, [_vp, _i32, _i32, _i32, _i32, _cp, _vp, _i32, _vp, _vp, _i32,
                                            _vp, _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
+        "csa2_sparse_attn_decode_noalloc": (_i32, [_vp, _i32, _i32, _i32, _i32, _cp, _vp, _i32, _vp, _vp,
+                                                   _i32, _vp, _i32, _f32, _vp, _vp, _vp]),
         "csa2_plan": (_i32, [_ip, _i32, _ip, _ip]),
         "csa2_last_device_error": (_i32, [_vp]),
         "csa2_status_string": (ctypes.c_char_p, [_i32]),
@@ -202,6 +205,33 @@ def sparse_attn_decode(q: torch.Tensor, cache: PagedCache, page_table: torch.Ten
                                     ws.numel() * ws.element_size(), _stream())
     _check("csa2_sparse_attn_decode", rc)
     return out, lse
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def sparse_attn_decode_noalloc(q: torch.Tensor, cache: PagedCache, page_table: torch.Tensor,
+                               seq_lens: torch.Tensor, topk_idx: Optional[torch.Tensor], swa: torch.Tensor,
+                               softmax_scale: float, out: torch.Tensor, lse: torch.Tensor) -> None:
+    """sparse_attn_decode without a workspace: the library's own device
+    scratch holds the split partials (see csa2_sparse_attn_decode_noalloc in
+    csa2.h). The caller passes the output buffers; nothing is allocated."""
+    B, Sq = q.shape[0], q.shape[1]
+    max_pages = page_table.shape[1]
+    _req(q, torch.bfloat16, "q", (B, Sq, HEADS, DIM))
+    _req(page_table, torch.int32, "page_table", (B, max_pages))
+    _req(seq_lens, torch.int32, "seq_lens", (B,))
+    k = 0 if topk_idx is None else topk_idx.shape[2]
+    if topk_idx is not None:
+        _req(topk_idx, torch.int32, "topk_idx", (B, Sq, k))
+    _req(swa, torch.bfloat16, "swa", (B, WINDOW + Sq - 1, DIM))
+    _req(out, torch.float32, "out", (B, Sq, HEADS, DIM))
+    _req(lse, torch.float32, "lse", (B, Sq, HEADS))
+    rc = _L.csa2_sparse_attn_decode_noalloc(_ptr(q), B, Sq, HEADS, DIM, ctypes.byref(cache.desc),
+                                            _ptr(page_table), max_pages, _ptr(seq_lens), _ptr(topk_idx), k,
+                                            _ptr(swa), WINDOW, float(softmax_scale), _ptr(out), _ptr(lse),
+                                            _stream())
+    _check("csa2_sparse_attn_decode_noalloc", rc)
 
 
 def plan(modes: Sequence[str]) -> Tuple[list, list]:

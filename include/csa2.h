@@ -202,6 +202,42 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int B, int Sq, int H,
                                     void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * csa2_sparse_attn_decode_noalloc -- csa2_sparse_attn_decode for callers that
+ * cannot allocate device memory. The pages describe no such variant; it is a
+ * convenience of this library.
+ *
+ * Who needs it: code that is handed only its input and output buffers by a
+ * host framework and has no allocator to call (for example a plugin whose
+ * enqueue hook receives no workspace), and decode loops that must not call
+ * cudaMalloc because it can synchronise the device and stall the stream.
+ *
+ * Same arguments and results as csa2_sparse_attn_decode, minus the workspace:
+ * the split-k partials live in one library-owned device array of
+ * CSA2_NOALLOC_SCRATCH_BYTES (32 MiB), which every GPU that loads the library
+ * keeps until process exit. The call allocates nothing and never calls
+ * cudaMalloc / cudaFree. Its first call on a device looks up the device
+ * address of that array with the device current; make that first call before
+ * any stream capture. When the partials of a call would need more than
+ * CSA2_NOALLOC_SCRATCH_BYTES (csa2_sparse_attn_workspace_bytes() larger than
+ * the limit) it returns CSA2_ERR_WORKSPACE and enqueues nothing. Every call on
+ * a device shares the one array: two calls whose kernels can overlap on the
+ * GPU (different streams without ordering between them) race on it and give
+ * wrong results; calls ordered on one stream are safe. Nothing in the array
+ * needs to start at zero (each call writes every partial it reads).
+ */
+#define CSA2_NOALLOC_SCRATCH_BYTES (32u << 20)
+csa2_status csa2_sparse_attn_decode_noalloc(const void *q_bf16, int B, int Sq,
+                                            int H, int D,
+                                            const csa2_paged_cache *cache,
+                                            const int32_t *page_table,
+                                            int max_pages,
+                                            const int32_t *seq_lens,
+                                            const int32_t *topk_idx, int k,
+                                            const void *swa_bf16, int W,
+                                            float softmax_scale, float *out,
+                                            float *lse, void *stream);
+
+/*
  * csa2_plan -- ownership bookkeeping for a group of layers ([ZUL section 3]:
  * KV owner layer -> consumer layers; [NEO part 2]: KV, indexer keys and top-K
  * indices shared across layers). Host-only, no device work.
