@@ -6,21 +6,28 @@
 // 架构拆解…" (blog.zulogic.cn), section 4 (a 128-token window kept per layer
 // beside the global compressed state).
 //
-// One CTA (8 warps) per (query token, split of its key list). The key list
-// is the k selected positions followed by the 128 window rows. Per tile of 64
-// keys:
-//   gather   4 threads per key: 16-byte loads of the 288 packed bytes and
-//            2-byte loads of the group scales (or of the bf16 window row),
-//            hardware E2M1x2 -> f16x2 and E4M3x2 -> f16x2 conversion, one
-//            exact f16 multiply, 16-byte stores into a [64][584] f16 tile;
-//   QK       warp (key group kg, channel quarter cq): 4 n-tiles x 9 k-steps of
-//            m16n8k16 f16 MMA, query fragments resident in registers; the four
-//            channel quarters are summed through shared memory;
+// One CTA (8 warps, two CTAs per SM) per (query token, split of its key
+// list). The key list is the k selected positions followed by the 128 window
+// rows; a split owns a run of at most 6 tiles of 64 keys.
+//   set-up   the split's selected positions are resolved once to physical
+//            cache slots (top-k index -> page table) in a shared table;
+//   prefetch right after a tile is dequantized, cp.async (16-byte and 4-byte
+//            LDGSTS, zero-filled for empty slots) fetches the next tile's
+//            packed FP4 records and scales, overlapping the tile's math;
+//   dequant  4 threads per key: hardware E2M1x2 -> f16x2 and E4M3x2 -> f16x2
+//            conversion and one exact f16 multiply into a [64][576] f16 tile
+//            whose 16-byte chunks are XOR-swizzled by key (conflict-free
+//            ldmatrix); window rows: bf16 loads rounded to f16;
+//   QK       warp (32-key group, 144-channel quarter): 4 n-tiles x 9 k-steps of
+//            m16n8k16 f16 MMA with the query fragments resident in registers;
+//            the quarters are summed through shared memory;
 //   softmax  two heads per warp, warp-shuffle max / sum in the exp2 domain,
 //            probabilities rounded to f16 (the same values feed the sum);
-//   PV       warp w owns 72 output channels (9 n-tiles), ldmatrix.trans of the
-//            same f16 tile serves as the value operand.
-// Splits write unnormalised partials (m, l, O) that K5 merges.
+//   PV       warp w owns 72 output channels; ldmatrix.trans of the same tile
+//            is the value operand.
+// Warp-level mma.sync is used deliberately: with 16 heads the MMA N extent is
+// 16, and at that width the warp MMAs issue faster than tcgen05 single-thread
+// MMAs. Splits write unnormalised partials (m, l, O) that K5 merges.
 #pragma once
 
 #include "common.cuh"
@@ -29,19 +36,22 @@ namespace csa2 {
 
 constexpr int kAttThreads = 256;
 constexpr int kAttTile = 64;
-constexpr int kKhPitch = kDim + 8;          // halfs per tile row (1168 B: conflict-free ldmatrix)
+constexpr int kKhRow = kDim * 2;            // 1152 bytes per f16 key row (no padding: swizzled chunks)
 constexpr int kPPitch = kAttTile + 8;       // halfs per probability row
-constexpr int kRedPitch = 36;               // floats per partial-score row
+constexpr int kMaxTilesPerSplit = 6;
 
 struct AttSmem {
-    alignas(128) __half kh[kAttTile][kKhPitch];
-    alignas(16) float red[8][16][kRedPitch];
-    alignas(16) __half p[16][kPPitch];
+    alignas(128) uint8_t kh[kAttTile * kKhRow];            // 73,728: f16 keys / values
+    alignas(16) float red[8][16][32];                      // 16,384: QK partials; P reuses the start
+    alignas(16) uint8_t raw[kAttTile][kFp4Bytes];          // 18,432: staged packed FP4 of the next tile
+    alignas(16) uint8_t rsc[kAttTile][kScaleBytes];        // 2,304: staged scales of the next tile
+    int slot[kMaxTilesPerSplit * kAttTile];                // 1,536: physical slot of each selected key
     float m_run[16];
     float l_run[16];
     float alpha[16];
     int valid[kAttTile];
 };
+constexpr size_t kAttSmemBytes = sizeof(AttSmem);
 
 struct AttParams {
     const __nv_bfloat16 *q;        // [R][16][576]
@@ -64,30 +74,80 @@ struct AttParams {
     int tiles_per_split;
 };
 
+// Byte offset of 8-channel chunk `chunk` (0..71) of key row `key`: chunks are
+// XOR-swizzled by the key's low 3 bits so that the 8 rows an ldmatrix reads
+// fall in 8 different bank groups.
+__device__ __forceinline__ uint32_t kh_off(int key, int chunk) {
+    return static_cast<uint32_t>(key * kKhRow + ((chunk ^ (key & 7)) << 4));
+}
+
+// Float index of (head, key-in-group) in a warp's QK partial block: columns
+// XOR-swizzled by the head (in 8-float blocks) so that the four heads a
+// half-warp's float2 fragment stores touch land in four different bank groups.
+__device__ __forceinline__ int red_col(int head, int col) { return col ^ ((head & 3) << 3); }
+
 __global__ void __launch_bounds__(kAttThreads, 2)
 sparse_attn_kernel(const AttParams P) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     AttSmem &sm = *reinterpret_cast<AttSmem *>(smem_raw);
+    __half (*pmat)[kPPitch] = reinterpret_cast<__half (*)[kPPitch]>(&sm.red[0][0][0]);   // P overlays red
     const int row = blockIdx.y;
     const int split = blockIdx.x;
     const int b = row / P.Sq, j = row % P.Sq;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, tig = lane & 3;
     const int n_rows_swa = kWindow + P.Sq - 1;
+    pdl_wait();                                         // the selection's indices are ready
+    pdl_trigger();
 
     int T = P.seq_lens[b];
     if (T < P.Sq || T > P.max_pages * kPage) {
         if (tid == 0 && split == 0) flag_status(kStatusBounds);
-        T = -1;                                   // no valid key at all
+        T = -1;                                          // no valid key at all
     }
     const int n_slots = P.k + kWindow;
     const int n_tiles = (n_slots + kAttTile - 1) / kAttTile;
     const int tile0 = split * P.tiles_per_split;
-    const int tile1 = min(tile0 + P.tiles_per_split, n_tiles);
+    const int tile1 = min(min(tile0 + P.tiles_per_split, n_tiles), tile0 + kMaxTilesPerSplit);
+    const int n_it = max(tile1 - tile0, 0);
 
     if (tid < 16) {
         sm.m_run[tid] = -INFINITY;
         sm.l_run[tid] = 0.0f;
+    }
+    // Physical slots of this split's selected keys: all index loads first,
+    // then all page-table loads, so only two load latencies are exposed.
+    {
+        constexpr int kPer = (kMaxTilesPerSplit * kAttTile + kAttThreads - 1) / kAttThreads;   // 2
+        int ti[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int i = tid + u * kAttThreads;
+            const int slot = tile0 * kAttTile + i;
+            ti[u] = (i < n_it * kAttTile && slot < P.k && T > 0)
+                        ? P.topk_idx[static_cast<int64_t>(row) * P.k + slot] : -1;
+        }
+        int64_t ph[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            ph[u] = -1;
+            if (ti[u] >= 0) {
+                if (ti[u] < T) ph[u] = P.page_table[static_cast<int64_t>(b) * P.max_pages + (ti[u] >> 6)];
+                else flag_status(kStatusBounds);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int i = tid + u * kAttThreads;
+            if (i < n_it * kAttTile) {
+                int phys_slot = -1;
+                if (ti[u] >= 0 && ti[u] < T) {
+                    if (ph[u] >= 0 && ph[u] < P.num_pages) phys_slot = static_cast<int>(ph[u] * kPage + (ti[u] & 63));
+                    else flag_status(kStatusBounds);
+                }
+                sm.slot[i] = phys_slot;
+            }
+        }
     }
 
     // Query fragments for QK: warp (kg, cq) covers channels cq*144 .. +143.
@@ -104,97 +164,103 @@ sparse_attn_kernel(const AttParams P) {
             qa[ks][3] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + (g + 8) * kDim + cb + 8));
         }
     }
-
     float o[9][4];
 #pragma unroll
     for (int nt = 0; nt < 9; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.0f;
+    __syncthreads();                                     // slot table ready
+
+    const int gkey = tid >> 2, gpart = tid & 3;          // gather role: 4 threads per key
+    auto prefetch = [&](int tile) {
+        const int slot = tile * kAttTile + gkey;
+        if (slot >= P.k) return;                         // window / padding keys are not staged
+        const int ps = sm.slot[(tile - tile0) * kAttTile + gkey];
+        const uint32_t nb16 = ps >= 0 ? 16u : 0u, nb4 = ps >= 0 ? 4u : 0u;
+        const uint8_t *src = P.kv_fp4 + (ps >= 0 ? static_cast<int64_t>(ps) * kFp4Bytes : 0);
+        const uint8_t *ssrc = P.kv_scale + (ps >= 0 ? static_cast<int64_t>(ps) * kScaleBytes : 0);
+        for (int c = gpart; c < kFp4Bytes / 16; c += 4) cp_async16(&sm.raw[gkey][c * 16], src + c * 16, nb16);
+        for (int wd = gpart; wd < kScaleBytes / 4; wd += 4) cp_async4(&sm.rsc[gkey][wd * 4], ssrc + wd * 4, nb4);
+    };
+    if (n_it > 0) prefetch(tile0);
+    cp_async_commit();
 
     for (int tile = tile0; tile < tile1; ++tile) {
-        // ---------------- gather + dequantize one tile of 64 keys
+        const int it = tile - tile0;
+        cp_async_wait<0>();                              // this tile's raw records have landed
+        __syncthreads();
+        // ---------------- dequantize one tile of 64 keys into f16
         {
-            const int key = tid >> 2, part = tid & 3;
-            const int slot = tile * kAttTile + key;
-            __half *dst = sm.kh[key];
+            const int slot = tile * kAttTile + gkey;
+            uint8_t *kh = sm.kh;
             bool valid = false;
-            if (slot < P.k && T > 0) {
-                const int ti = P.topk_idx[static_cast<int64_t>(row) * P.k + slot];
-                int64_t phys_slot = -1;
-                if (ti >= 0) {
-                    if (ti < T) {
-                        const int64_t ph = P.page_table[static_cast<int64_t>(b) * P.max_pages + (ti >> 6)];
-                        if (ph >= 0 && ph < P.num_pages) phys_slot = ph * kPage + (ti & 63);
-                        else flag_status(kStatusBounds);
-                    } else {
-                        flag_status(kStatusBounds);
-                    }
-                }
-                if (phys_slot >= 0) {
-                    valid = true;
-                    const uint8_t *src = P.kv_fp4 + phys_slot * kFp4Bytes;
-                    const uint8_t *ssrc = P.kv_scale + phys_slot * kScaleBytes;
-                    uint4 raw[5];
-                    uint32_t sc[5];
+            if (slot < P.k) {
+                valid = sm.slot[it * kAttTile + gkey] >= 0;
+                if (valid) {
+                    // Threads 2 and 3 of a key walk the four 8-channel
+                    // chunks of a record chunk in the order 2,3,0,1, so the
+                    // 8 lanes of each 128-bit store phase hit 8 bank groups.
+                    const bool rot = (gpart & 2) != 0;
+                    for (int c = gpart; c < kFp4Bytes / 16; c += 4) {   // 16-byte chunk = 32 channels
+                        const uint4 raw = *reinterpret_cast<const uint4 *>(&sm.raw[gkey][c * 16]);
+                        const uint32_t sc = *reinterpret_cast<const unsigned short *>(&sm.rsc[gkey][c * 2]);
+                        const uint32_t sf = e4m3x2_to_f16x2(sc);                 // (scale 2c, scale 2c+1)
+                        const uint32_t s_lo = __byte_perm(sf, 0, 0x1010);
+                        const uint32_t s_hi = __byte_perm(sf, 0, 0x3232);
+                        const uint32_t w[4] = {rot ? raw.z : raw.x, rot ? raw.w : raw.y,
+                                               rot ? raw.x : raw.z, rot ? raw.y : raw.w};
+                        const uint32_t sa = rot ? s_hi : s_lo, sb = rot ? s_lo : s_hi;
 #pragma unroll
-                    for (int i = 0; i < 5; ++i) {
-                        const int c = part + 4 * i;      // 16-byte chunk = 32 channels
-                        if (c < 18) {
-                            raw[i] = __ldg(reinterpret_cast<const uint4 *>(src + c * 16));
-                            sc[i] = __ldg(reinterpret_cast<const unsigned short *>(ssrc + c * 2));
-                        }
-                    }
-#pragma unroll
-                    for (int i = 0; i < 5; ++i) {
-                        const int c = part + 4 * i;
-                        if (c < 18) {
-                            const uint32_t sf = e4m3x2_to_f16x2(sc[i]);          // (scale 2c, scale 2c+1)
-                            const uint32_t s_lo = __byte_perm(sf, 0, 0x1010);     // broadcast low half
-                            const uint32_t s_hi = __byte_perm(sf, 0, 0x3232);     // broadcast high half
-                            const uint32_t wv[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-#pragma unroll
-                            for (int q4 = 0; q4 < 4; ++q4) {
-                                const uint32_t s2 = q4 < 2 ? s_lo : s_hi;
-                                uint4 h;
-                                h.x = hmul2_u32(e2m1x2_to_f16x2(wv[q4] & 0xffu), s2);
-                                h.y = hmul2_u32(e2m1x2_to_f16x2((wv[q4] >> 8) & 0xffu), s2);
-                                h.z = hmul2_u32(e2m1x2_to_f16x2((wv[q4] >> 16) & 0xffu), s2);
-                                h.w = hmul2_u32(e2m1x2_to_f16x2(wv[q4] >> 24), s2);
-                                *reinterpret_cast<uint4 *>(dst + c * 32 + q4 * 8) = h;
-                            }
+                        for (int q = 0; q < 4; ++q) {
+                            const uint32_t wv = w[q];
+                            const uint32_t s2 = q < 2 ? sa : sb;
+                            uint4 h;
+                            h.x = hmul2_u32(e2m1x2_to_f16x2(wv & 0xffu), s2);
+                            h.y = hmul2_u32(e2m1x2_to_f16x2((wv >> 8) & 0xffu), s2);
+                            h.z = hmul2_u32(e2m1x2_to_f16x2((wv >> 16) & 0xffu), s2);
+                            h.w = hmul2_u32(e2m1x2_to_f16x2(wv >> 24), s2);
+                            *reinterpret_cast<uint4 *>(kh + kh_off(gkey, 4 * c + (q ^ (rot ? 2 : 0)))) = h;
                         }
                     }
                 }
-            } else if (slot >= P.k && slot < n_slots && T > 0) {
+            } else if (slot < n_slots && T > 0) {
                 const int r = j + (slot - P.k);              // window row of this query
                 if (T - n_rows_swa + r >= 0) {
                     valid = true;
                     const uint4 *src = reinterpret_cast<const uint4 *>(
                         P.swa + (static_cast<int64_t>(b) * n_rows_swa + r) * kDim);
+                    // Thread p of a key takes chunks 8m + 2p + {0,1}: the
+                    // chunks of a store phase share their parity per key.
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
-                        uint4 raw[9];
-#pragma unroll
-                        for (int i = 0; i < 9; ++i) raw[i] = __ldg(src + part + 4 * (half * 9 + i));
+                        uint4 rv[9];
 #pragma unroll
                         for (int i = 0; i < 9; ++i) {
+                            const int e = half * 9 + i;
+                            rv[i] = __ldg(src + 8 * (e >> 1) + 2 * gpart + (e & 1));
+                        }
+#pragma unroll
+                        for (int i = 0; i < 9; ++i) {
+                            const int e = half * 9 + i;
                             uint4 h;
-                            h.x = bf16x2_to_f16x2(raw[i].x);
-                            h.y = bf16x2_to_f16x2(raw[i].y);
-                            h.z = bf16x2_to_f16x2(raw[i].z);
-                            h.w = bf16x2_to_f16x2(raw[i].w);
-                            *reinterpret_cast<uint4 *>(dst + (part + 4 * (half * 9 + i)) * 8) = h;
+                            h.x = bf16x2_to_f16x2(rv[i].x);
+                            h.y = bf16x2_to_f16x2(rv[i].y);
+                            h.z = bf16x2_to_f16x2(rv[i].z);
+                            h.w = bf16x2_to_f16x2(rv[i].w);
+                            *reinterpret_cast<uint4 *>(kh + kh_off(gkey, 8 * (e >> 1) + 2 * gpart + (e & 1))) = h;
                         }
                     }
                 }
             }
             if (!valid) {
                 const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-                for (int c = part; c < kDim / 8; c += 4) *reinterpret_cast<uint4 *>(dst + c * 8) = z;
+                for (int c = gpart; c < kDim / 8; c += 4) *reinterpret_cast<uint4 *>(kh + kh_off(gkey, c)) = z;
             }
-            if (part == 0) sm.valid[key] = valid ? 1 : 0;
+            if (gpart == 0) sm.valid[gkey] = valid ? 1 : 0;
         }
         __syncthreads();
+        if (tile + 1 < tile1) prefetch(tile + 1);        // overlaps this tile's math
+        cp_async_commit();
 
-        // ---------------- S = Q K^T over this warp's channel quarter
+        // ---------------- S = Q K^T over this warp's 32 keys x channel quarter
         {
             float acc[4][4];
 #pragma unroll
@@ -207,58 +273,67 @@ sparse_attn_kernel(const AttParams P) {
                 for (int pr = 0; pr < 2; ++pr) {
                     const int key = kg * 32 + (2 * pr + (m >> 1)) * 8 + r;
                     uint32_t b0, b1, b2, b3;
-                    ldsm_x4(b0, b1, b2, b3, &sm.kh[key][cb + (m & 1) * 8]);
+                    ldsm_x4(b0, b1, b2, b3, sm.kh + kh_off(key, (cb >> 3) + (m & 1)));
                     mma_f16_16816(acc[2 * pr], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
                     mma_f16_16816(acc[2 * pr + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
                 }
             }
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                sm.red[warp][g][nt * 8 + tig * 2] = acc[nt][0];
-                sm.red[warp][g][nt * 8 + tig * 2 + 1] = acc[nt][1];
-                sm.red[warp][g + 8][nt * 8 + tig * 2] = acc[nt][2];
-                sm.red[warp][g + 8][nt * 8 + tig * 2 + 1] = acc[nt][3];
+                const int col = nt * 8 + tig * 2;
+                *reinterpret_cast<float2 *>(&sm.red[warp][g][red_col(g, col)]) = make_float2(acc[nt][0], acc[nt][1]);
+                *reinterpret_cast<float2 *>(&sm.red[warp][g + 8][red_col(g + 8, col)]) =
+                    make_float2(acc[nt][2], acc[nt][3]);
             }
         }
         __syncthreads();
 
         // ---------------- online softmax, two heads per warp
+        {
+            float pv[2][2], alpha[2], m_new[2], psum[2];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const int h = warp * 2 + hh;
-            float s[2];
+            for (int hh = 0; hh < 2; ++hh) {
+                const int h = warp * 2 + hh;
+                float s[2];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int key = lane + 32 * u;          // key group u
-                const float v = sm.red[u * 4 + 0][h][lane] + sm.red[u * 4 + 1][h][lane] +
-                                sm.red[u * 4 + 2][h][lane] + sm.red[u * 4 + 3][h][lane];
-                s[u] = sm.valid[key] ? v * P.scale_log2 : -INFINITY;
+                for (int u = 0; u < 2; ++u) {
+                    const int key = lane + 32 * u;          // key group u
+                    const int cc = red_col(h, lane);
+                    const float v = sm.red[u * 4 + 0][h][cc] + sm.red[u * 4 + 1][h][cc] +
+                                    sm.red[u * 4 + 2][h][cc] + sm.red[u * 4 + 3][h][cc];
+                    s[u] = sm.valid[key] ? v * P.scale_log2 : -INFINITY;
+                }
+                float mx = fmaxf(s[0], s[1]);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                const float m_old = sm.m_run[h];
+                m_new[hh] = fmaxf(m_old, mx);
+                if (m_new[hh] == -INFINITY) {
+                    alpha[hh] = 1.0f;
+                    pv[hh][0] = pv[hh][1] = 0.0f;
+                } else {
+                    alpha[hh] = exp2f(m_old - m_new[hh]);
+                    pv[hh][0] = exp2f(s[0] - m_new[hh]);
+                    pv[hh][1] = exp2f(s[1] - m_new[hh]);
+                }
+                pv[hh][0] = __half2float(__float2half_rn(pv[hh][0]));
+                pv[hh][1] = __half2float(__float2half_rn(pv[hh][1]));
+                float sum = pv[hh][0] + pv[hh][1];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+                psum[hh] = sum;
             }
-            float mx = fmaxf(s[0], s[1]);
+            __syncthreads();                                  // every warp is done reading red (P overlays it)
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            const float m_old = sm.m_run[h];
-            const float m_new = fmaxf(m_old, mx);
-            float alpha, p0, p1;
-            if (m_new == -INFINITY) {
-                alpha = 1.0f;
-                p0 = p1 = 0.0f;
-            } else {
-                alpha = exp2f(m_old - m_new);
-                p0 = exp2f(s[0] - m_new);
-                p1 = exp2f(s[1] - m_new);
-            }
-            const __half h0 = __float2half_rn(p0), h1 = __float2half_rn(p1);
-            sm.p[h][lane] = h0;
-            sm.p[h][lane + 32] = h1;
-            float sum = __half2float(h0) + __half2float(h1);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-            __syncwarp();
-            if (lane == 0) {
-                sm.l_run[h] = sm.l_run[h] * alpha + sum;
-                sm.m_run[h] = m_new;
-                sm.alpha[h] = alpha;
+            for (int hh = 0; hh < 2; ++hh) {
+                const int h = warp * 2 + hh;
+                pmat[h][lane] = __float2half_rn(pv[hh][0]);
+                pmat[h][lane + 32] = __float2half_rn(pv[hh][1]);
+                if (lane == 0) {
+                    sm.l_run[h] = sm.l_run[h] * alpha[hh] + psum[hh];
+                    sm.m_run[h] = m_new[hh];
+                    sm.alpha[h] = alpha[hh];
+                }
             }
         }
         __syncthreads();
@@ -278,22 +353,23 @@ sparse_attn_kernel(const AttParams P) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 uint32_t a0, a1, a2, a3;
-                ldsm_x4(a0, a1, a2, a3, &sm.p[r + 8 * (m & 1)][kk * 16 + 8 * (m >> 1)]);
+                ldsm_x4(a0, a1, a2, a3, &pmat[r + 8 * (m & 1)][kk * 16 + 8 * (m >> 1)]);
                 const int key = kk * 16 + 8 * (m & 1) + r;
 #pragma unroll
                 for (int pr = 0; pr < 4; ++pr) {
                     uint32_t b0, b1, b2, b3;
-                    ldsm_x4_t(b0, b1, b2, b3, &sm.kh[key][c0 + pr * 16 + 8 * (m >> 1)]);
+                    ldsm_x4_t(b0, b1, b2, b3, sm.kh + kh_off(key, ((c0 + pr * 16) >> 3) + (m >> 1)));
                     mma_f16_16816(o[2 * pr], a0, a1, a2, a3, b0, b1);
                     mma_f16_16816(o[2 * pr + 1], a0, a1, a2, a3, b2, b3);
                 }
                 uint32_t b0, b1;
-                ldsm_x2_t(b0, b1, &sm.kh[key][c0 + 64]);
+                ldsm_x2_t(b0, b1, sm.kh + kh_off(key, (c0 + 64) >> 3));
                 mma_f16_16816(o[8], a0, a1, a2, a3, b0, b1);
             }
         }
-        __syncthreads();
     }
+    cp_async_wait<0>();
+    __syncthreads();
 
     // ---------------- epilogue: final output or split partial
     const int c0 = warp * 72;
@@ -327,48 +403,72 @@ sparse_attn_kernel(const AttParams P) {
 }
 
 // K5: merge split partials: O = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-constexpr int kMergeThreads = 256;
+// One CTA per (query row, group of 4 heads): the (m, l) pairs are staged in
+// shared memory by all threads at once, then each thread owns 3 float4 of the
+// group's 4 x 576 outputs and issues the split loads 4 at a time, so the
+// L2 round trips overlap instead of following one another.
+constexpr int kMergeThreads = 192;
+constexpr int kMergeHeads = 4;
+constexpr int kMergeVec = kMergeHeads * kDim / 4;        // 576 float4 per CTA
+constexpr int kMergePer = kMergeVec / kMergeThreads;    // 3
 
 __global__ void __launch_bounds__(kMergeThreads)
 attn_merge_kernel(const float *__restrict__ part_o, const float2 *__restrict__ part_ml, int n_splits,
                   float *__restrict__ out, float *__restrict__ lse) {
-    extern __shared__ float wgt[];     // [n_splits][16]
-    const int row = blockIdx.x;
-    const float2 *ml = part_ml + static_cast<int64_t>(row) * n_splits * kHeads;
-    if (threadIdx.x < kHeads) {
-        const int h = threadIdx.x;
+    extern __shared__ float2 mlw[];    // [n_splits][4]: (m, l), then (weight, -)
+    pdl_wait();
+    pdl_trigger();
+    const int row = blockIdx.x, hg = blockIdx.y, tid = threadIdx.x;
+    const float2 *ml = part_ml + static_cast<int64_t>(row) * n_splits * kHeads + hg * kMergeHeads;
+    for (int i = tid; i < n_splits * kMergeHeads; i += kMergeThreads)
+        mlw[i] = __ldcg(ml + (i / kMergeHeads) * kHeads + (i % kMergeHeads));
+    __syncthreads();
+    if (tid < kMergeHeads) {
         float M = -INFINITY;
-        for (int s = 0; s < n_splits; ++s) M = fmaxf(M, ml[s * kHeads + h].x);
+        for (int s = 0; s < n_splits; ++s) M = fmaxf(M, mlw[s * kMergeHeads + tid].x);
         float L = 0.0f;
         for (int s = 0; s < n_splits; ++s) {
-            const float2 v = ml[s * kHeads + h];
+            const float2 v = mlw[s * kMergeHeads + tid];
             const float e = (M == -INFINITY || v.y == 0.0f) ? 0.0f : exp2f(v.x - M);
-            wgt[s * kHeads + h] = e;
+            mlw[s * kMergeHeads + tid].x = e;
             L += e * v.y;
         }
         const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-        for (int s = 0; s < n_splits; ++s) wgt[s * kHeads + h] *= inv;
-        lse[static_cast<int64_t>(row) * kHeads + h] = L > 0.0f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+        for (int s = 0; s < n_splits; ++s) mlw[s * kMergeHeads + tid].x *= inv;
+        lse[static_cast<int64_t>(row) * kHeads + hg * kMergeHeads + tid] =
+            L > 0.0f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
     }
     __syncthreads();
-    const float4 *po = reinterpret_cast<const float4 *>(part_o + static_cast<int64_t>(row) * n_splits * kHeads * kDim);
-    float4 *orow = reinterpret_cast<float4 *>(out + static_cast<int64_t>(row) * kHeads * kDim);
-    constexpr int kVec = kHeads * kDim / 4;   // 2304 float4 per row
-    for (int i = threadIdx.x; i < kVec; i += kMergeThreads) {
-        const int h = (i * 4) / kDim;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = 0; s < n_splits; ++s) {
-            const float wv = wgt[s * kHeads + h];
-            if (wv != 0.0f) {
-                const float4 v = __ldcg(po + static_cast<int64_t>(s) * kVec + i);
-                acc.x += wv * v.x;
-                acc.y += wv * v.y;
-                acc.z += wv * v.z;
-                acc.w += wv * v.w;
+    constexpr int kRowVec = kHeads * kDim / 4;              // 2304 float4 per split partial
+    const float4 *po = reinterpret_cast<const float4 *>(part_o) +
+                       static_cast<int64_t>(row) * n_splits * kRowVec + hg * kMergeVec;
+    float4 acc[kMergePer];
+#pragma unroll
+    for (int c = 0; c < kMergePer; ++c) acc[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < n_splits; s0 += 4) {
+        float4 v[4][kMergePer];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int c = 0; c < kMergePer; ++c)
+                v[u][c] = s0 + u < n_splits ? __ldcg(po + static_cast<int64_t>(s0 + u) * kRowVec + c * kMergeThreads + tid)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (s0 + u >= n_splits) break;
+#pragma unroll
+            for (int c = 0; c < kMergePer; ++c) {
+                const float wv = mlw[(s0 + u) * kMergeHeads + (c * kMergeThreads + tid) / (kDim / 4)].x;
+                acc[c].x += wv * v[u][c].x;
+                acc[c].y += wv * v[u][c].y;
+                acc[c].z += wv * v[u][c].z;
+                acc[c].w += wv * v[u][c].w;
             }
         }
-        orow[i] = acc;
     }
+    float4 *orow = reinterpret_cast<float4 *>(out + static_cast<int64_t>(row) * kHeads * kDim) + hg * kMergeVec;
+#pragma unroll
+    for (int c = 0; c < kMergePer; ++c) orow[c * kMergeThreads + tid] = acc[c];
 }
 
 }  // namespace csa2

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 
 #include "attn.cuh"
 #include "common.cuh"
@@ -23,6 +24,7 @@ struct DeviceInfo {
     bool ready = false;
     int sm_count = 0;
     int att_ctas_per_sm = 0;
+    int tk_max_cluster = 1;       // largest power-of-two top-k cluster the device can co-schedule
 };
 DeviceInfo g_dev[kMaxDevices];
 
@@ -40,15 +42,55 @@ cudaError_t device_info(DeviceInfo **out) {
         e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(indexer_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(sizeof(IdxSmem)));
+                                 static_cast<int>(std::max(idx_smem_bytes(idx_shape(1)), idx_smem_bytes(idx_shape(2)))));
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(sizeof(AttSmem)));
+                                 static_cast<int>(kAttSmemBytes));
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(sizeof(TkSmem)));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+        // One shared-memory carveout for every kernel of the path, so that
+        // consecutive launches do not reconfigure the SMs' L1 / shared split.
+        const void *kernels[] = {reinterpret_cast<const void *>(quant_kv_fp4_kernel),
+                                 reinterpret_cast<const void *>(indexer_score_kernel),
+                                 reinterpret_cast<const void *>(topk_zero_kernel),
+                                 reinterpret_cast<const void *>(topk_cluster_kernel),
+                                 reinterpret_cast<const void *>(sparse_attn_kernel),
+                                 reinterpret_cast<const void *>(attn_merge_kernel)};
+        for (const void *kf : kernels) {
+            e = cudaFuncSetAttribute(kf, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+            if (e != cudaSuccess) return e;
+        }
+
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.att_ctas_per_sm, sparse_attn_kernel, kAttThreads,
-                                                          sizeof(AttSmem));
+                                                          kAttSmemBytes);
         if (e != cudaSuccess) return e;
         if (d.att_ctas_per_sm < 1) d.att_ctas_per_sm = 1;
+        // Largest top-k cluster (<= 16 CTAs) that fits on the device at once.
+        d.tk_max_cluster = 1;
+        for (int cs = kTkMaxCluster; cs > 1; cs /= 2) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(cs);
+            cfg.blockDim = dim3(kTkThreads);
+            cfg.dynamicSmemBytes = sizeof(TkSmem);
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = cs;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int n_clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&n_clusters, topk_cluster_kernel, &cfg) == cudaSuccess &&
+                n_clusters >= 1) {
+                d.tk_max_cluster = cs;
+                break;
+            }
+            (void)cudaGetLastError();                      // clear a refusal of this size
+        }
         d.ready = true;
     }
     *out = &d;
@@ -58,22 +100,17 @@ cudaError_t device_info(DeviceInfo **out) {
 // ---------------------------------------------------------------- indexer / top-k workspace
 struct IdxLayout {
     int64_t t_cap;
-    int n_chunks;
-    size_t scores, rows, hist, counters, chunk_cnt, chunk_off, total;
+    size_t scores, hist, zero_end, total;
 };
 
-IdxLayout idx_layout(int B, int Sq, int max_pages) {
+IdxLayout idx_layout(int B, int Sq, int max_pages, int k) {
     IdxLayout L{};
     const int64_t R = static_cast<int64_t>(B) * Sq;
     L.t_cap = static_cast<int64_t>(max_pages) * kPage;
-    L.n_chunks = static_cast<int>((L.t_cap + kTopkChunk - 1) / kTopkChunk);
     size_t off = 0;
     L.scores = off;    off = round_up(off + static_cast<size_t>(R * L.t_cap) * 4, 256);
-    L.rows = off;      off = round_up(off + static_cast<size_t>(R) * sizeof(TopkRow), 256);
     L.hist = off;      off = round_up(off + static_cast<size_t>(R) * kTopkBins * 4, 256);
-    L.counters = off;  off = round_up(off + static_cast<size_t>(R) * 4, 256);
-    L.chunk_cnt = off; off = round_up(off + static_cast<size_t>(R) * L.n_chunks * 8, 256);
-    L.chunk_off = off; off = round_up(off + static_cast<size_t>(R) * L.n_chunks * 8, 256);
+    L.zero_end = off;
     L.total = off;
     return L;
 }
@@ -89,9 +126,10 @@ struct AttSplit {
 // small charge per split for writing and merging its partial.
 AttSplit att_split(int R, int k, int slots) {
     const int n_tiles = (k + kWindow + kAttTile - 1) / kAttTile;
-    AttSplit best{1, n_tiles};
+    const int s_min = (n_tiles + kMaxTilesPerSplit - 1) / kMaxTilesPerSplit;
+    AttSplit best{s_min, (n_tiles + s_min - 1) / s_min};
     double best_cost = 1e30;
-    for (int s = 1; s <= n_tiles && s <= 64; ++s) {
+    for (int s = s_min; s <= n_tiles && s <= s_min + 64; ++s) {
         const int tps = (n_tiles + s - 1) / s;
         const int s_eff = (n_tiles + tps - 1) / tps;
         const int64_t ctas = static_cast<int64_t>(R) * s_eff;
@@ -143,9 +181,8 @@ csa2_status csa2_quant_kv_fp4(const void *x_bf16, int64_t n_tok, int dim, const 
 }
 
 size_t csa2_indexer_topk_workspace_bytes(int B, int Sq, int max_pages, int k) {
-    (void)k;
-    if (B <= 0 || Sq <= 0 || max_pages <= 0) return 0;
-    return idx_layout(B, Sq, max_pages).total;
+    if (B <= 0 || Sq <= 0 || max_pages <= 0 || k <= 0) return 0;
+    return idx_layout(B, Sq, max_pages, k).total;
 }
 
 csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq, int idx_heads, int idx_dim,
@@ -163,7 +200,7 @@ csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq, 
     if (!aligned(q_idx, 16) || !aligned(w, 16) || !aligned(cache->kidx, 16) || !aligned(cache->kidx_scale, 16) ||
         !aligned(page_table, 4) || !aligned(seq_lens, 4) || !aligned(out_idx, 4))
         return CSA2_ERR_ALIGNMENT;
-    const IdxLayout L = idx_layout(B, Sq, max_pages);
+    const IdxLayout L = idx_layout(B, Sq, max_pages, k);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return CSA2_ERR_WORKSPACE;
     DeviceInfo *dev = nullptr;
     cudaError_t e = device_info(&dev);
@@ -172,29 +209,47 @@ csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq, 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *base = static_cast<uint8_t *>(ws);
     float *scores = reinterpret_cast<float *>(base + L.scores);
-    TopkRow *rows = reinterpret_cast<TopkRow *>(base + L.rows);
     uint32_t *hist = reinterpret_cast<uint32_t *>(base + L.hist);
-    uint32_t *counters = reinterpret_cast<uint32_t *>(base + L.counters);
-    uint2 *chunk_cnt = reinterpret_cast<uint2 *>(base + L.chunk_cnt);
-    uint2 *chunk_off = reinterpret_cast<uint2 *>(base + L.chunk_off);
     const int R = B * Sq;
 
-    dim3 g1((max_pages + kIdxPagesPerCta - 1) / kIdxPagesPerCta, B);
-    indexer_score_kernel<<<g1, kIdxThreads, sizeof(IdxSmem), st>>>(
-        static_cast<const uint8_t *>(q_idx), w, static_cast<const uint8_t *>(cache->kidx), cache->kidx_scale,
-        cache->num_pages, page_table, max_pages, seq_lens, Sq, k, scores, L.t_cap, rows, hist, counters);
-    count_launch();
-    dim3 g2(L.n_chunks, R);
-    for (int level = 0; level < 3; ++level) {
-        topk_radix_kernel<<<g2, kTopkThreads, 0, st>>>(scores, L.t_cap, rows, hist, counters, level);
-        count_launch();
-    }
-    topk_count_kernel<<<g2, kTopkThreads, 0, st>>>(scores, L.t_cap, rows, counters, chunk_cnt, chunk_off,
-                                                   L.n_chunks);
-    count_launch();
-    topk_write_kernel<<<g2, kTopkThreads, 0, st>>>(scores, L.t_cap, rows, chunk_off, L.n_chunks, k, out_idx);
-    count_launch();
-    return cuda_status(cudaGetLastError());
+    // The level-1 histograms start at zero.
+    const int64_t n16 = static_cast<int64_t>((L.zero_end - L.hist) / 16);
+    e = launch_pdl(topk_zero_kernel, dim3(static_cast<unsigned>(std::min<int64_t>((n16 + 255) / 256, 2 * dev->sm_count))),
+                   dim3(256), 0, st, reinterpret_cast<uint4 *>(base + L.hist), n16);
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+
+    IdxArgs A;
+    A.q_idx = static_cast<const uint8_t *>(q_idx);
+    A.w = w;
+    A.kidx = static_cast<const uint8_t *>(cache->kidx);
+    A.kidx_scale = cache->kidx_scale;
+    A.num_pages = cache->num_pages;
+    A.page_table = page_table;
+    A.max_pages = max_pages;
+    A.seq_lens = seq_lens;
+    A.B = B;
+    A.Sq = Sq;
+    A.scores = scores;
+    A.t_cap = L.t_cap;
+    A.hist = hist;
+    const IdxShape shape = idx_shape(Sq);
+    A.hist_rows = shape.hist_rows;
+    A.ring = shape.ring;
+    const int64_t n_flat = static_cast<int64_t>(B) * max_pages;
+    const int grid1 = static_cast<int>(std::min<int64_t>(n_flat, dev->sm_count));
+    e = launch_pdl(indexer_score_kernel, dim3(grid1), dim3(shape.warps * 32), idx_smem_bytes(shape), st, A);
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+    // Top-k: one cluster of C CTAs per query row, C a power of two chosen so
+    // that the R * C CTAs stay within one wave and every CTA keeps at least
+    // 8192 positions.
+    int C = 1;
+    while (C * 2 <= dev->tk_max_cluster && static_cast<int64_t>(R) * C * 2 <= dev->sm_count &&
+           L.t_cap / (C * 2) >= 8192)
+        C *= 2;
+    e = launch_pdl_cluster(topk_cluster_kernel, dim3(static_cast<unsigned>(R * C)), dim3(kTkThreads), sizeof(TkSmem),
+                           st, C, static_cast<const float *>(scores), L.t_cap, static_cast<const uint32_t *>(hist),
+                           seq_lens, Sq, max_pages, k, out_idx);
+    return cuda_status(e);
 }
 
 size_t csa2_sparse_attn_workspace_bytes(int B, int Sq, int k) {
@@ -256,14 +311,15 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int B, int Sq, int H, in
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     dim3 grid(sp.n_splits, R);
-    sparse_attn_kernel<<<grid, kAttThreads, sizeof(AttSmem), st>>>(P);
-    count_launch();
+    cudaError_t e = launch_pdl(sparse_attn_kernel, grid, dim3(kAttThreads), kAttSmemBytes, st, P);
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
     if (sp.n_splits > 1) {
-        attn_merge_kernel<<<R, kMergeThreads, sp.n_splits * kHeads * sizeof(float), st>>>(
-            P.part_o, P.part_ml, sp.n_splits, out, lse);
-        count_launch();
+        e = launch_pdl(attn_merge_kernel, dim3(R, kHeads / kMergeHeads), dim3(kMergeThreads),
+                       sp.n_splits * kMergeHeads * sizeof(float2), st,
+                       static_cast<const float *>(P.part_o), static_cast<const float2 *>(P.part_ml), sp.n_splits,
+                       out, lse);
     }
-    return cuda_status(cudaGetLastError());
+    return cuda_status(e);
 }
 
 }  // extern "C"

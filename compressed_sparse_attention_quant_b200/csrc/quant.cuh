@@ -22,6 +22,8 @@ quant_kv_fp4_kernel(const uint4 *__restrict__ x, int64_t n_tok, const int32_t *_
                     uint8_t *__restrict__ kv_fp4, uint8_t *__restrict__ kv_scale,
                     uint8_t *__restrict__ kidx, float *__restrict__ kidx_scale, int64_t n_slots) {
     constexpr int kGroups = kDim / kGroup;  // 36
+    pdl_wait();
+    pdl_trigger();
     const int64_t gid = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
     const int64_t tok = gid / kGroups;
     const int g = static_cast<int>(gid - tok * kGroups);
@@ -87,12 +89,10 @@ inline cudaError_t launch_quant_kv_fp4(const void *x, int64_t n_tok, const int32
                                        const csa2_paged_cache &c, cudaStream_t stream) {
     const int64_t threads = n_tok * (kDim / kGroup);
     const int64_t blocks = (threads + kQuantThreads - 1) / kQuantThreads;
-    quant_kv_fp4_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, stream>>>(
-        static_cast<const uint4 *>(x), n_tok, slots, static_cast<const uint4 *>(kidx_in), ksig_in,
-        static_cast<uint8_t *>(c.kv_fp4), static_cast<uint8_t *>(c.kv_scale),
-        static_cast<uint8_t *>(c.kidx), c.kidx_scale, c.num_pages * kPage);
-    count_launch();
-    return cudaGetLastError();
+    return launch_pdl(quant_kv_fp4_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kQuantThreads), 0, stream,
+                      static_cast<const uint4 *>(x), n_tok, slots, static_cast<const uint4 *>(kidx_in), ksig_in,
+                      static_cast<uint8_t *>(c.kv_fp4), static_cast<uint8_t *>(c.kv_scale),
+                      static_cast<uint8_t *>(c.kidx), c.kidx_scale, c.num_pages * kPage);
 }
 
 }  // namespace csa2

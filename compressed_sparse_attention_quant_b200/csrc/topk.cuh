@@ -3,277 +3,464 @@
 // part 2: the "Top-K sparse addressing index"; page "DeepSeek V4 1-Flash
 // 架构拆解…" (blog.zulogic.cn), section 3: Full and Reindex run the selection.
 //
-// Selection rule: the k largest scores of positions 0 .. n_valid-1, ties to
-// the lower position, emitted in ascending position order, -1 padded.
+// Rule: the k largest scores of positions 0 .. n_valid-1, ties to the lower
+// position, emitted in ascending position order, -1 padded.
 //
-// Method (multi-CTA per query row, no inter-CTA waiting):
-//   1. radix levels on the order-preserving 32-bit key of each score, 11 + 11
-//      + 10 bits from the top: every CTA histograms the next digit of the
-//      keys that match the prefix resolved so far (shared-memory atomics,
-//      then one global add per non-empty bin); the last CTA of the row to
-//      arrive (atomic counter, no spin) picks the digit holding the k-th key
-//      and stops early once every element of that digit is taken.
-//   2. count: per 4096-element chunk, elements above the threshold prefix
-//      and equal to it; the last CTA scans the chunk counts into output
-//      offsets.
-//   3. write: each chunk emits its selected positions in order (block scan
-//      of per-thread counts); among keys equal to the threshold only the
-//      lowest positions, up to the number still needed, are taken.
-// Scores stay L2-resident between the passes (4 B per cached token).
+// Method: a radix select over order-preserving 32-bit keys, levels of
+// 11 + 11 + 10 bits, run by one thread-block cluster of C CTAs per query row
+// (C = 1..16). CTA r of the cluster owns the position windows
+// [(i*C + r)*W, +W) for rounds i = 0, 1, ... (a single round unless the row
+// exceeds C * 2^17 positions).
+//   level 1  the indexer already built the row's histogram of the top 11 key
+//            bits: every CTA finds the bin b1 holding the k-th largest key.
+//   pass A   one read of the CTA's scores (L2-resident): keys in bins above
+//            b1 are certainly selected and set bits of a shared-memory
+//            bitmap over the window; keys in bin b1 are candidates, counted
+//            into a histogram of their next 11 bits and kept (key, position)
+//            in shared memory while they fit.
+//   level 2/3 the CTAs sum their histograms through distributed shared
+//            memory (every CTA reads every peer's), so each CTA picks the same
+//            digit; level 3 is skipped when the level-2 bin is taken whole.
+//   emit     candidates above the threshold key join the bitmap, candidates
+//            equal to it go to a tie bitmap; one exchange of (selected, ties)
+//            counts across the cluster gives each CTA its first tie rank and
+//            output offset, ties are taken lowest position first, and each
+//            thread writes the positions of its contiguous bitmap words.
+// If some CTA's candidates overflow its shared list, or the row needs more
+// than one round, the levels and the emission re-read the scores instead of
+// the list (same result, more L2 reads). Cluster barriers are the only
+// waits, and every CTA of a cluster takes the same branches.
 #pragma once
 
 #include "common.cuh"
 #include "indexer.cuh"
 
+#include <cooperative_groups.h>
+
 namespace csa2 {
 
-constexpr int kTopkThreads = 256;
-constexpr int kTopkPerThread = 16;
-constexpr int kTopkChunk = kTopkThreads * kTopkPerThread;   // 4096
+constexpr int kTkThreads = 1024;
+constexpr int kTkWin = 1 << 17;                  // positions per CTA window
+constexpr int kTkWinWords = kTkWin / 32;
+constexpr int kTkCandCap = 12288;                // candidates kept in shared memory per CTA
+constexpr int kTkMaxCluster = 16;
+constexpr int kTkUnroll = 4;                     // float4 loads in flight per thread
 
-__device__ __forceinline__ int topk_digit_width(int level) { return level < 2 ? 11 : 10; }
+// Zeroes the per-row level-1 histograms before the indexer accumulates them.
+__global__ void __launch_bounds__(256) topk_zero_kernel(uint4 *__restrict__ p, int64_t n16) {
+    pdl_wait();                                         // the previous selection has read them
+    pdl_trigger();
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        p[i] = make_uint4(0u, 0u, 0u, 0u);
+}
 
-// Exclusive block scan of one value per thread (256 threads). Returns the
-// exclusive prefix; *total receives the block sum.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_buf, uint32_t *total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t incl = v;
+__device__ __forceinline__ int topk_n_valid(const int32_t *seq_lens, int row, int Sq, int max_pages) {
+    const int b = row / Sq, j = row % Sq;
+    const int T = seq_lens[b];
+    if (T < Sq || T > max_pages * kPage) return 0;
+    return T - Sq + j + 1;
+}
+
+// Warp-level inclusive scan helper.
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+        const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
     }
-    if (lane == 31) warp_buf[warp] = incl;
+    return v;
+}
+
+// Exclusive block scan of one value per thread. wbuf holds >= nwarps + 1
+// words. Returns the exclusive prefix; *total receives the block sum.
+template <int NT>
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *wbuf, uint32_t *total) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t incl = warp_incl_scan(v);
+    if (lane == 31) wbuf[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        uint32_t wv = lane < (kTopkThreads / 32) ? warp_buf[lane] : 0u;
-        uint32_t wi = wv;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += y;
-        }
-        if (lane < (kTopkThreads / 32)) warp_buf[lane] = wi - wv;   // exclusive warp offsets
-        if (lane == kTopkThreads / 32 - 1) warp_buf[kTopkThreads / 32] = wi;
+        const uint32_t wv = lane < NW ? wbuf[lane] : 0u;
+        const uint32_t wi = warp_incl_scan(wv);
+        if (lane < NW) wbuf[lane] = wi - wv;
+        if (lane == NW - 1) wbuf[NW] = wi;
     }
     __syncthreads();
-    const uint32_t res = warp_buf[warp] + incl - v;
-    *total = warp_buf[kTopkThreads / 32];
+    const uint32_t res = wbuf[warp] + incl - v;
+    *total = wbuf[NW];
     __syncthreads();
     return res;
 }
 
-// Loads this thread's 16 consecutive keys of the chunk; positions >= n get
-// valid = false.
-__device__ __forceinline__ void load_keys(const float *__restrict__ srow, int64_t c0, int n,
-                                          uint32_t (&key)[kTopkPerThread], uint32_t &valid_mask) {
-    const int64_t e0 = c0 + static_cast<int64_t>(threadIdx.x) * kTopkPerThread;
-    valid_mask = 0u;
-    if (e0 + kTopkPerThread <= n) {
-        const float4 *p = reinterpret_cast<const float4 *>(srow + e0);
-#pragma unroll
-        for (int v = 0; v < kTopkPerThread / 4; ++v) {
-            const float4 f = __ldcg(p + v);
-            key[4 * v + 0] = float_key(f.x);
-            key[4 * v + 1] = float_key(f.y);
-            key[4 * v + 2] = float_key(f.z);
-            key[4 * v + 3] = float_key(f.w);
-        }
-        valid_mask = 0xffffu;
-    } else {
-#pragma unroll
-        for (int i = 0; i < kTopkPerThread; ++i) {
-            if (e0 + i < n) {
-                key[i] = float_key(__ldcg(srow + e0 + i));
-                valid_mask |= 1u << i;
-            } else {
-                key[i] = 0u;
-            }
-        }
-    }
-}
-
-__device__ __forceinline__ uint32_t key_prefix(uint32_t key, int bits) {
-    return bits == 0 ? 0u : (key >> (32 - bits));
-}
-
-// One radix level: histogram of the next digit, then the last CTA picks it.
-__global__ void __launch_bounds__(kTopkThreads)
-topk_radix_kernel(const float *__restrict__ scores, int64_t t_cap, TopkRow *__restrict__ rows,
-                  uint32_t *__restrict__ hist, uint32_t *__restrict__ counters, int level) {
-    __shared__ uint32_t sh[kTopkBins];
-    __shared__ uint32_t wbuf[kTopkThreads / 32 + 1];
-    __shared__ int is_last;
-    const int row = blockIdx.y;
-    const TopkRow st = rows[row];
-    if (st.done) return;                        // uniform over the row's CTAs
-    const int width = topk_digit_width(level);
-    const int nb = 1 << width;
-    const int bits_after = st.bits + width;
-    for (int i = threadIdx.x; i < nb; i += kTopkThreads) sh[i] = 0u;
-    __syncthreads();
-
-    const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kTopkChunk;
-    if (c0 < st.n_valid) {
-        uint32_t key[kTopkPerThread];
-        uint32_t vm;
-        load_keys(scores + static_cast<int64_t>(row) * t_cap, c0, st.n_valid, key, vm);
-#pragma unroll
-        for (int i = 0; i < kTopkPerThread; ++i) {
-            if (((vm >> i) & 1u) && key_prefix(key[i], st.bits) == st.prefix) {
-                atomicAdd(&sh[(key[i] >> (32 - bits_after)) & (nb - 1)], 1u);
-            }
-        }
-    }
-    __syncthreads();
-    uint32_t *gh = hist + static_cast<int64_t>(row) * kTopkBins;
-    for (int i = threadIdx.x; i < nb; i += kTopkThreads)
-        if (sh[i]) atomicAdd(&gh[i], sh[i]);
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) is_last = (atomicAdd(&counters[row], 1u) == gridDim.x - 1);
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-
-    // Last CTA of the row: find the digit holding the remaining-th largest key.
-    const int per = nb / kTopkThreads;          // 8 or 4 bins per thread
-    // thread t owns bins [hi_t - per + 1, hi_t] counted from the top
-    const int top = nb - 1 - threadIdx.x * per;
+// From the row's 2048-bin histogram (global), the bin holding the need-th
+// largest key, and how many keys lie in higher bins. Every thread of the
+// block gets the answer.
+template <int NT>
+__device__ __forceinline__ void find_threshold_bin(const uint32_t *__restrict__ gh, uint32_t need,
+                                                   uint32_t *wbuf, int *s_bin, uint32_t *s_above,
+                                                   int *bin_out, uint32_t *above_out) {
+    constexpr int PER = kTopkBins / NT;
+    const int top = kTopkBins - 1 - threadIdx.x * PER;   // this thread's bins: top, top-1, ...
+    uint32_t c[PER];
     uint32_t local = 0u;
-    for (int i = 0; i < per; ++i) {
-        const uint32_t c = __ldcg(&gh[top - i]);
-        sh[top - i] = c;
-        local += c;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        c[i] = __ldcg(&gh[top - i]);
+        local += c[i];
     }
     uint32_t tot;
-    const uint32_t above = block_excl_scan(local, wbuf, &tot);   // keys in higher bins
-    const uint32_t need = static_cast<uint32_t>(st.remaining);
-    uint32_t run = above;
-    for (int i = 0; i < per; ++i) {
-        const int bin = top - i;
-        const uint32_t c = sh[bin];
-        if (run < need && run + c >= need) {
-            TopkRow r = st;
-            r.prefix = (st.bits == 0 ? 0u : (st.prefix << width)) | static_cast<uint32_t>(bin);
-            r.bits = bits_after;
-            r.remaining = static_cast<int32_t>(need - run);
-            r.eq_count = static_cast<int32_t>(c);
-            r.done = (c == need - run || bits_after == 32) ? 1 : 0;
-            rows[row] = r;
+    uint32_t run = block_excl_scan<NT>(local, wbuf, &tot);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        if (run < need && run + c[i] >= need) {
+            *s_bin = top - i;
+            *s_above = run;
         }
-        run += c;
+        run += c[i];
     }
-    // leave the histogram and counter zeroed for the next level
-    for (int i = threadIdx.x; i < kTopkBins; i += kTopkThreads) gh[i] = 0u;
-    if (threadIdx.x == 0) counters[row] = 0u;
+    __syncthreads();
+    *bin_out = *s_bin;
+    *above_out = *s_above;
 }
 
-// Chunk counts of keys above / equal to the threshold prefix, then offsets.
-__global__ void __launch_bounds__(kTopkThreads)
-topk_count_kernel(const float *__restrict__ scores, int64_t t_cap, const TopkRow *__restrict__ rows,
-                  uint32_t *__restrict__ counters, uint2 *__restrict__ chunk_cnt,
-                  uint2 *__restrict__ chunk_off, int n_chunks) {
-    __shared__ uint32_t wbuf[kTopkThreads / 32 + 1];
-    __shared__ int is_last;
-    const int row = blockIdx.y;
-    const TopkRow st = rows[row];
-    const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kTopkChunk;
-    uint32_t gt = 0u, eq = 0u;
-    if (c0 < st.n_valid) {
-        uint32_t key[kTopkPerThread];
-        uint32_t vm;
-        load_keys(scores + static_cast<int64_t>(row) * t_cap, c0, st.n_valid, key, vm);
+struct TkSmem {
+    uint32_t sel[kTkWinWords];          // 16 KB: selected positions of the window
+    uint32_t tie[kTkWinWords];          // 16 KB: positions whose key equals the threshold
+    uint32_t ckey[kTkCandCap];          // 48 KB: candidate keys (bin b1)
+    int32_t cpos[kTkCandCap];           // 48 KB: candidate positions
+    uint32_t hloc[2][kTopkBins];        // this CTA's level-2 / level-3 histograms (read by peers)
+    uint32_t hsum[kTopkBins];           // cluster-wide sum of the current level
+    uint32_t wbuf[kTkThreads / 32 + 1];
+    uint32_t xchg[2][2];                // per round parity: (selected before ties, ties), read by peers
+    uint32_t n_cand;
+    int s_bin;
+    uint32_t s_above;
+    uint32_t s_digit;
+    uint32_t s_cum;
+    uint32_t s_flag;
+    uint32_t s_base[4];
+};
+
+// Digit of the need-th largest element of a histogram of nbins (<= 2048)
+// bins, and the count of elements in higher bins.
+__device__ __forceinline__ void tk_pick(TkSmem &sm, const uint32_t *h, int nbins, uint32_t need, uint32_t &digit,
+                                        uint32_t &above) {
+    const int top = kTopkBins - 1 - static_cast<int>(threadIdx.x) * 2;
+    const uint32_t c0 = top < nbins ? h[top] : 0u;
+    const uint32_t c1 = top - 1 < nbins ? h[top - 1] : 0u;
+    uint32_t tot;
+    const uint32_t run = block_excl_scan<kTkThreads>(c0 + c1, sm.wbuf, &tot);
+    if (run < need && run + c0 >= need) {
+        sm.s_digit = static_cast<uint32_t>(top);
+        sm.s_cum = run;
+    } else if (run + c0 < need && run + c0 + c1 >= need) {
+        sm.s_digit = static_cast<uint32_t>(top - 1);
+        sm.s_cum = run + c0;
+    }
+    __syncthreads();
+    digit = sm.s_digit;
+    above = sm.s_cum;
+    __syncthreads();
+}
+
+// Guarded float4 of scores at positions p .. p+3 (< w1 only).
+__device__ __forceinline__ float4 tk_load(const float *srow, int64_t p, int64_t w1, bool live) {
+    if (live && p + 4 <= w1) return __ldcg(reinterpret_cast<const float4 *>(srow + p));
+    float t[4] = {0.f, 0.f, 0.f, 0.f};
+    if (live)
 #pragma unroll
-        for (int i = 0; i < kTopkPerThread; ++i) {
-            if ((vm >> i) & 1u) {
-                const uint32_t pf = key_prefix(key[i], st.bits);
-                gt += pf > st.prefix;
-                eq += pf == st.prefix;
+        for (int u = 0; u < 4; ++u)
+            if (p + u < w1) t[u] = __ldcg(srow + p + u);
+    return make_float4(t[0], t[1], t[2], t[3]);
+}
+
+// OR of a 4-bit group over the 8 lanes sharing one 32-position bitmap word.
+__device__ __forceinline__ uint32_t tk_word(uint32_t nib) {
+    uint32_t w = nib << ((threadIdx.x & 7) * 4);
+    w |= __shfl_xor_sync(0xffffffffu, w, 1);
+    w |= __shfl_xor_sync(0xffffffffu, w, 2);
+    w |= __shfl_xor_sync(0xffffffffu, w, 4);
+    return w;
+}
+
+__global__ void __launch_bounds__(kTkThreads, 1)
+topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint32_t *__restrict__ hist,
+                    const int32_t *__restrict__ seq_lens, int Sq, int max_pages, int k, int32_t *__restrict__ out) {
+    namespace cg = cooperative_groups;
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    TkSmem &sm = *reinterpret_cast<TkSmem *>(smem_raw);
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = static_cast<int>(cluster.num_blocks());
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int row = blockIdx.x / C;
+    const int tid = threadIdx.x;
+    pdl_wait();                                         // scores and histograms are complete
+    pdl_trigger();
+    const int n_valid = topk_n_valid(seq_lens, row, Sq, max_pages);
+    int32_t *orow = out + static_cast<int64_t>(row) * k;
+    if (n_valid <= k) {                                 // every valid position is selected
+        for (int i = rank * kTkThreads + tid; i < k; i += C * kTkThreads) orow[i] = i < n_valid ? i : -1;
+        return;                                         // no distributed shared memory was touched
+    }
+    const float *srow = scores + static_cast<int64_t>(row) * t_cap;
+    const int64_t per = (static_cast<int64_t>(n_valid) + C - 1) / C;
+    const int64_t Wn = min(static_cast<int64_t>(kTkWin), (per + 31) / 32 * 32);
+    const int rounds = static_cast<int>((n_valid + C * Wn - 1) / (C * Wn));
+    const bool fast = rounds == 1;
+    auto win = [&](int r, int64_t &w0, int64_t &w1, int &n_it) {
+        w0 = (static_cast<int64_t>(r) * C + rank) * Wn;
+        w1 = min(w0 + Wn, static_cast<int64_t>(n_valid));
+        n_it = w1 > w0 ? static_cast<int>((w1 - w0 + 4 * kTkThreads - 1) / (4 * kTkThreads)) : 0;
+    };
+
+    for (int i = tid; i < 2 * kTopkBins; i += kTkThreads) (&sm.hloc[0][0])[i] = 0u;
+    if (tid == 0) sm.n_cand = 0u;
+    // ---- level 1: from the indexer's histogram
+    int b1;
+    uint32_t above1;
+    find_threshold_bin<kTkThreads>(hist + static_cast<int64_t>(row) * kTopkBins, static_cast<uint32_t>(k), sm.wbuf,
+                                   &sm.s_bin, &sm.s_above, &b1, &above1);
+    uint32_t need = static_cast<uint32_t>(k) - above1;
+
+    // ---- pass A: sure bits, level-2 histogram, candidate list
+    for (int r = 0; r < rounds; ++r) {
+        int64_t w0, w1;
+        int n_it;
+        win(r, w0, w1, n_it);
+        for (int i0 = 0; i0 < n_it; i0 += kTkUnroll) {
+            float4 f[kTkUnroll];
+#pragma unroll
+            for (int u = 0; u < kTkUnroll; ++u)
+                f[u] = tk_load(srow, w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) + tid * 4, w1,
+                               i0 + u < n_it);
+            uint32_t cmask = 0u;                         // 4 bits per unrolled load
+#pragma unroll
+            for (int u = 0; u < kTkUnroll; ++u) {
+                const int64_t p = w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) + tid * 4;
+                const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+                uint32_t s4 = 0u;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t key = float_key(fv[e]);
+                    const int bin = static_cast<int>(key >> kTopkDigitShift);
+                    if (i0 + u < n_it && p + e < w1) {
+                        if (bin > b1) s4 |= 1u << e;
+                        if (bin == b1) {
+                            cmask |= 1u << (4 * u + e);
+                            atomicAdd(&sm.hloc[0][(key >> 10) & (kTopkBins - 1)], 1u);
+                        }
+                    }
+                }
+                if (fast) {
+                    const uint32_t w = tk_word(s4);
+                    if ((tid & 7) == 0 && i0 + u < n_it) sm.sel[(i0 + u) * (kTkThreads / 8) + (tid >> 3)] = w;
+                }
+            }
+            if (fast && __any_sync(0xffffffffu, cmask != 0u)) {
+                const uint32_t cnt = __popc(cmask);
+                const uint32_t incl = warp_incl_scan(cnt);
+                uint32_t base = 0u;
+                if ((tid & 31) == 31) base = atomicAdd(&sm.n_cand, incl);
+                base = __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
+                while (cmask) {
+                    const int bit = __ffs(cmask) - 1;
+                    cmask &= cmask - 1u;
+                    const int u = bit >> 2, e = bit & 3;
+                    float4 fu = f[0];
+#pragma unroll
+                    for (int uu = 1; uu < kTkUnroll; ++uu)
+                        if (u == uu) fu = f[uu];                 // register select, no local array
+                    const float v = e == 0 ? fu.x : e == 1 ? fu.y : e == 2 ? fu.z : fu.w;
+                    if (base < static_cast<uint32_t>(kTkCandCap)) {
+                        sm.ckey[base] = float_key(v);
+                        sm.cpos[base] = static_cast<int32_t>(w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) +
+                                                             tid * 4 + e);
+                    }
+                    ++base;
+                }
             }
         }
     }
-    uint32_t tgt, teq;
-    block_excl_scan(gt, wbuf, &tgt);
-    block_excl_scan(eq, wbuf, &teq);
-    uint2 *cc = chunk_cnt + static_cast<int64_t>(row) * n_chunks;
-    if (threadIdx.x == 0) cc[blockIdx.x] = make_uint2(tgt, teq);
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) is_last = (atomicAdd(&counters[row], 1u) == gridDim.x - 1);
-    __syncthreads();
-    if (!is_last) return;
-    __threadfence();
-    // Offsets: output position of each chunk's first selection, and the number
-    // of threshold-equal keys in earlier chunks.
-    uint2 *co = chunk_off + static_cast<int64_t>(row) * n_chunks;
-    uint32_t gt_before = 0u, eq_before = 0u;
-    for (int base = 0; base < n_chunks; base += kTopkThreads) {
-        const int c = base + threadIdx.x;
-        uint2 v = make_uint2(0u, 0u);
-        if (c < n_chunks) v = __ldcg(&cc[c]);
-        uint32_t sg, se;
-        const uint32_t pg = block_excl_scan(v.x, wbuf, &sg);
-        const uint32_t pe = block_excl_scan(v.y, wbuf, &se);
-        if (c < n_chunks) {
-            const uint32_t eb = eq_before + pe;
-            const uint32_t take = min(eb, static_cast<uint32_t>(st.remaining));
-            co[c] = make_uint2(gt_before + pg + take, eb);
-        }
-        gt_before += sg;
-        eq_before += se;
-    }
-    if (threadIdx.x == 0) counters[row] = 0u;
-}
+    cluster.sync();                                     // every CTA's level-2 histogram and list are complete
 
-// Emit the selected positions of each chunk in ascending order.
-__global__ void __launch_bounds__(kTopkThreads)
-topk_write_kernel(const float *__restrict__ scores, int64_t t_cap, const TopkRow *__restrict__ rows,
-                  const uint2 *__restrict__ chunk_off, int n_chunks, int k, int32_t *__restrict__ out) {
-    __shared__ uint32_t wbuf[kTopkThreads / 32 + 1];
-    const int row = blockIdx.y;
-    const TopkRow st = rows[row];
-    int32_t *orow = out + static_cast<int64_t>(row) * k;
-    if (blockIdx.x == 0) {
-        const int n_sel = min(k, st.n_valid);
-        for (int i = n_sel + threadIdx.x; i < k; i += kTopkThreads) orow[i] = -1;
+    // ---- level 2: cluster-wide histogram of the candidates' next 11 bits
+    for (int i = tid; i < kTopkBins; i += kTkThreads) {
+        uint32_t v = 0u;
+        for (int q = 0; q < C; ++q) v += cluster.map_shared_rank(&sm.hloc[0][0], q)[i];
+        sm.hsum[i] = v;
     }
-    const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kTopkChunk;
-    if (c0 >= st.n_valid) return;               // uniform over the CTA
-    const uint2 off = chunk_off[static_cast<int64_t>(row) * n_chunks + blockIdx.x];
-    uint32_t key[kTopkPerThread];
-    uint32_t vm;
-    load_keys(scores + static_cast<int64_t>(row) * t_cap, c0, st.n_valid, key, vm);
-    uint32_t gtm = 0u, eqm = 0u;
+    if (tid == 0) {
+        uint32_t of = 0u;
+        for (int q = 0; q < C; ++q) of |= *cluster.map_shared_rank(&sm.n_cand, q) > static_cast<uint32_t>(kTkCandCap);
+        sm.s_flag = of;
+    }
+    __syncthreads();
+    const bool use_list = fast && sm.s_flag == 0u;
+    uint32_t d2, above2;
+    tk_pick(sm, sm.hsum, kTopkBins, need, d2, above2);
+    const uint32_t cnt2 = sm.hsum[d2];
+    need -= above2;
+    uint32_t prefix = (static_cast<uint32_t>(b1) << 11) | d2;
+    int bits = 22;
+    if (cnt2 != need) {
+        // ---- level 3: the low 10 bits of the keys with this 22-bit prefix
+        if (use_list) {
+            const uint32_t nc = sm.n_cand;
+            for (uint32_t i = tid; i < nc; i += kTkThreads) {
+                const uint32_t key = sm.ckey[i];
+                if ((key >> 10) == prefix) atomicAdd(&sm.hloc[1][key & 1023u], 1u);
+            }
+        } else {
+            for (int r = 0; r < rounds; ++r) {
+                int64_t w0, w1;
+                int n_it;
+                win(r, w0, w1, n_it);
+                for (int i = 0; i < n_it; ++i) {
+                    const int64_t p = w0 + static_cast<int64_t>(i) * (4 * kTkThreads) + tid * 4;
+                    const float4 f = tk_load(srow, p, w1, true);
+                    const float fv[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-    for (int i = 0; i < kTopkPerThread; ++i) {
-        if ((vm >> i) & 1u) {
-            const uint32_t pf = key_prefix(key[i], st.bits);
-            if (pf > st.prefix) gtm |= 1u << i;
-            if (pf == st.prefix) eqm |= 1u << i;
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t key = float_key(fv[e]);
+                        if (p + e < w1 && (key >> 10) == prefix) atomicAdd(&sm.hloc[1][key & 1023u], 1u);
+                    }
+                }
+            }
         }
+        cluster.sync();
+        for (int i = tid; i < 1024; i += kTkThreads) {
+            uint32_t v = 0u;
+            for (int q = 0; q < C; ++q) v += cluster.map_shared_rank(&sm.hloc[1][0], q)[i];
+            sm.hsum[i] = v;
+        }
+        __syncthreads();
+        uint32_t d3, above3;
+        tk_pick(sm, sm.hsum, 1024, need, d3, above3);
+        need -= above3;
+        prefix = (prefix << 10) | d3;
+        bits = 32;
     }
-    uint32_t tot;
-    const uint32_t eq_rank0 = off.y + block_excl_scan(__popc(eqm), wbuf, &tot);
-    // threshold-equal keys are taken while their global rank < remaining
-    uint32_t selm = gtm;
-    uint32_t r = eq_rank0;
+    // Threshold: keys whose top `bits` bits exceed `prefix` are selected;
+    // among keys equal to it, the `need` lowest positions.
+
+    // ---- emission, one round at a time (positions ascend with the round)
+    uint32_t out_base = 0u, tie_base = 0u;
+    for (int r = 0; r < rounds; ++r) {
+        int64_t w0, w1;
+        int n_it;
+        win(r, w0, w1, n_it);
+        const int nw = w1 > w0 ? static_cast<int>((w1 - w0 + 31) / 32) : 0;
+        __syncthreads();                                // the previous round's bitmaps are consumed
+        if (use_list) {
+            for (int i = tid; i < nw; i += kTkThreads) sm.tie[i] = 0u;
+            __syncthreads();
+            const uint32_t nc = sm.n_cand;
+            for (uint32_t i = tid; i < nc; i += kTkThreads) {
+                const uint32_t key = sm.ckey[i];
+                const uint32_t top = bits == 32 ? key : key >> 10;
+                const int64_t rel = sm.cpos[i] - w0;
+                if (top > prefix) atomicOr(&sm.sel[rel >> 5], 1u << (rel & 31));
+                else if (top == prefix) atomicOr(&sm.tie[rel >> 5], 1u << (rel & 31));
+            }
+        } else {
+            for (int i = 0; i < n_it; ++i) {
+                const int64_t p = w0 + static_cast<int64_t>(i) * (4 * kTkThreads) + tid * 4;
+                const float4 f = tk_load(srow, p, w1, true);
+                const float fv[4] = {f.x, f.y, f.z, f.w};
+                uint32_t s4 = 0u, t4 = 0u;
 #pragma unroll
-    for (int i = 0; i < kTopkPerThread; ++i) {
-        if ((eqm >> i) & 1u) {
-            if (r < static_cast<uint32_t>(st.remaining)) selm |= 1u << i;
-            ++r;
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t key = float_key(fv[e]);
+                    const uint32_t top = bits == 32 ? key : key >> 10;
+                    if (p + e < w1) {
+                        if (top > prefix) s4 |= 1u << e;
+                        else if (top == prefix) t4 |= 1u << e;
+                    }
+                }
+                const uint32_t ws = tk_word(s4), wt = tk_word(t4);
+                if ((tid & 7) == 0) {
+                    sm.sel[i * (kTkThreads / 8) + (tid >> 3)] = ws;
+                    sm.tie[i * (kTkThreads / 8) + (tid >> 3)] = wt;
+                }
+            }
         }
-    }
-    uint32_t pos = off.x + block_excl_scan(__popc(selm), wbuf, &tot);
-    const int64_t e0 = c0 + static_cast<int64_t>(threadIdx.x) * kTopkPerThread;
-#pragma unroll
-    for (int i = 0; i < kTopkPerThread; ++i) {
-        if ((selm >> i) & 1u) {
-            if (pos < static_cast<uint32_t>(k)) orow[pos] = static_cast<int32_t>(e0 + i);
-            ++pos;
+        __syncthreads();
+        // thread t owns the contiguous words [wb, we)
+        const int wper = (nw + kTkThreads - 1) / kTkThreads;
+        const int wb = min(tid * wper, nw), we = min(wb + wper, nw);
+        uint32_t n_tie = 0u, n_sel = 0u;
+        for (int i = wb; i < we; ++i) {
+            n_tie += __popc(sm.tie[i]);
+            n_sel += __popc(sm.sel[i]);
         }
+        uint32_t cta_ties, cta_sel;
+        const uint32_t tie_off = block_excl_scan<kTkThreads>(n_tie, sm.wbuf, &cta_ties);
+        block_excl_scan<kTkThreads>(n_sel, sm.wbuf, &cta_sel);
+        if (tid == 0) {
+            sm.xchg[r & 1][0] = cta_sel;
+            sm.xchg[r & 1][1] = cta_ties;
+        }
+        cluster.sync();
+        if (tid == 0) {
+            // Walk the cluster in position order: ranks, each with its ties
+            // taken while the global tie rank is below `need`.
+            uint32_t op = out_base, tp = tie_base;
+            for (int q = 0; q < C; ++q) {
+                const uint32_t *x = cluster.map_shared_rank(&sm.xchg[r & 1][0], q);
+                const uint32_t s = x[0], t = x[1];
+                if (q == rank) {
+                    sm.s_base[0] = op;
+                    sm.s_base[1] = tp;
+                }
+                const uint32_t taken = need > tp ? min(t, need - tp) : 0u;
+                op += s + taken;
+                tp += t;
+            }
+            sm.s_base[2] = op;
+            sm.s_base[3] = tp;
+        }
+        __syncthreads();
+        uint32_t tie_rank = sm.s_base[1] + tie_off;
+        uint32_t n_out = 0u;
+        for (int i = wb; i < we; ++i) {
+            uint32_t m = sm.sel[i];
+            uint32_t tm = sm.tie[i];
+            if (tm) {
+                const uint32_t c = __popc(tm);
+                if (tie_rank + c <= need) {
+                    m |= tm;
+                } else {
+                    uint32_t tr = tie_rank;
+                    while (tm) {
+                        const uint32_t bit = tm & (0u - tm);
+                        tm ^= bit;
+                        if (tr < need) m |= bit;
+                        ++tr;
+                    }
+                }
+                tie_rank += c;
+                sm.sel[i] = m;
+            }
+            n_out += __popc(m);
+        }
+        uint32_t cta_out;
+        uint32_t pos = sm.s_base[0] + block_excl_scan<kTkThreads>(n_out, sm.wbuf, &cta_out);
+        for (int i = wb; i < we; ++i) {
+            uint32_t m = sm.sel[i];
+            while (m) {
+                const int bit = __ffs(m) - 1;
+                m &= m - 1u;
+                if (pos < static_cast<uint32_t>(k)) orow[pos] = static_cast<int32_t>(w0 + i * 32 + bit);
+                ++pos;
+            }
+        }
+        out_base = sm.s_base[2];
+        tie_base = sm.s_base[3];
     }
+    cluster.sync();                                     // no CTA leaves while a peer may read its counts
 }
 
 }  // namespace csa2

@@ -62,16 +62,52 @@ def test_decode_group_matches_oracle(mods, case):
 
 
 def test_topk_ties_go_to_lower_index(mods):
-    """All-zero indexer query: every score is 0, so the top-k are 0..k-1."""
+    """All-zero indexer query: every score is 0, so the top-k are 0..k-1. The
+    28000-token rows are split over 2 CTAs of about 14000 positions, more equal
+    scores than a CTA's candidate list holds, so they take the re-scan path."""
     lib, workload = mods
-    wl = inputs.small_workload("ties", 2, 2, [3000, 777], 100, modes=("F",))
+    wl = inputs.small_workload("ties", 3, 2, [28000, 3000, 777], 100, modes=("F",))
     dw = workload.DeviceWorkload(wl)
     dw.q_idx[0].zero_()
     dw.step()
+    assert lib.last_device_error() == 0
     idx = dw.group.index(0).cpu().numpy()
-    for b in range(2):
+    for b in range(3):
         for j in range(2):
             np.testing.assert_array_equal(idx[b, j], np.arange(100, dtype=np.int32))
+
+
+def test_topk_heavy_ties_against_oracle(mods):
+    """Indexer queries with a single non-zero channel: scores take few
+    distinct values, so the threshold bin is crowded (overflow path on the
+    long row, candidate path on the short ones); indices must match."""
+    lib, workload = mods
+    wl = inputs.small_workload("crowd", 3, 1, [30000, 6000, 2500], 700, modes=("F",), seed=5)
+    dw = workload.DeviceWorkload(wl)
+    dw.q_idx[0][:, :, :, 1:] = 0
+    dw.step()
+    assert lib.last_device_error() == 0
+    ref = OracleRun(dw, range(3))
+    idx = dw.group.index(0).cpu().numpy()
+    for b in range(3):
+        np.testing.assert_array_equal(idx[b, 0], ref.out[0][(b, 0)]["idx"], err_msg=f"b {b}")
+
+
+def test_topk_rows_longer_than_one_window(mods):
+    """80 query rows give one CTA per row, and rows longer than 2^17 positions
+    are then covered in two rounds of windows; shorter rows in the same
+    launch take one round. Sampled rows must match the oracle exactly."""
+    lib, workload = mods
+    lens = [140000 if b % 3 == 0 else (131100 if b % 3 == 1 else 5000) for b in range(80)]
+    wl = inputs.small_workload("rounds", 80, 1, lens, 2048, modes=("F",), seed=11)
+    dw = workload.DeviceWorkload(wl)
+    dw.step()
+    assert lib.last_device_error() == 0
+    rows = [0, 1, 2, 39, 79]
+    ref = OracleRun(dw, rows)
+    idx = dw.group.index(0).cpu().numpy()
+    for b in rows:
+        np.testing.assert_array_equal(idx[b, 0], ref.out[0][(b, 0)]["idx"], err_msg=f"b {b}")
 
 
 def test_topk_all_valid_when_k_covers_context(mods):
