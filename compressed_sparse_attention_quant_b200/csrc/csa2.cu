@@ -41,8 +41,11 @@ cudaError_t device_info(DeviceInfo **out) {
     if (!d.ready) {
         e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(indexer_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(std::max(idx_smem_bytes(idx_shape(1)), idx_smem_bytes(idx_shape(2)))));
+        e = cudaFuncSetAttribute(indexer_score_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(idx_smem_bytes<1>()));
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(indexer_score_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(idx_smem_bytes<0>()));
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kAttSmemBytes));
@@ -55,7 +58,8 @@ cudaError_t device_info(DeviceInfo **out) {
         // One shared-memory carveout for every kernel of the path, so that
         // consecutive launches do not reconfigure the SMs' L1 / shared split.
         const void *kernels[] = {reinterpret_cast<const void *>(quant_kv_fp4_kernel),
-                                 reinterpret_cast<const void *>(indexer_score_kernel),
+                                 reinterpret_cast<const void *>(indexer_score_kernel<1>),
+                                 reinterpret_cast<const void *>(indexer_score_kernel<0>),
                                  reinterpret_cast<const void *>(topk_zero_kernel),
                                  reinterpret_cast<const void *>(topk_cluster_kernel),
                                  reinterpret_cast<const void *>(sparse_attn_kernel),
@@ -195,6 +199,7 @@ csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq, 
     if (Sq > 4) return CSA2_ERR_UNSUPPORTED;   // 4 query tokens x 4 heads = 16 MMA columns
     if (static_cast<int64_t>(B) * Sq > 65535) return CSA2_ERR_UNSUPPORTED;
     if (static_cast<int64_t>(max_pages) * kPage > (INT64_C(1) << 30)) return CSA2_ERR_UNSUPPORTED;
+    if (cache->num_pages > INT32_MAX) return CSA2_ERR_UNSUPPORTED;   // page-table entries are int32
     if (!q_idx || !w || !page_table || !seq_lens || !out_idx || !cache->kidx || !cache->kidx_scale)
         return CSA2_ERR_INVALID_ARG;
     if (!aligned(q_idx, 16) || !aligned(w, 16) || !aligned(cache->kidx, 16) || !aligned(cache->kidx_scale, 16) ||
@@ -232,12 +237,12 @@ csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq, 
     A.scores = scores;
     A.t_cap = L.t_cap;
     A.hist = hist;
-    const IdxShape shape = idx_shape(Sq);
-    A.hist_rows = shape.hist_rows;
-    A.ring = shape.ring;
-    const int64_t n_flat = static_cast<int64_t>(B) * max_pages;
-    const int grid1 = static_cast<int>(std::min<int64_t>(n_flat, dev->sm_count));
-    e = launch_pdl(indexer_score_kernel, dim3(grid1), dim3(shape.warps * 32), idx_smem_bytes(shape), st, A);
+    const int64_t n_units = static_cast<int64_t>(B) * ((max_pages + kIdxUnitPages - 1) / kIdxUnitPages);
+    const int grid1 = static_cast<int>(std::min<int64_t>(n_units, dev->sm_count));
+    if (Sq == 1)
+        e = launch_pdl(indexer_score_kernel<1>, dim3(grid1), dim3(kIdxThreads), idx_smem_bytes<1>(), st, A);
+    else
+        e = launch_pdl(indexer_score_kernel<0>, dim3(grid1), dim3(kIdxThreads), idx_smem_bytes<0>(), st, A);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
     // Top-k: one cluster of C CTAs per query row, C a power of two chosen so
     // that the R * C CTAs stay within one wave and every CTA keeps at least

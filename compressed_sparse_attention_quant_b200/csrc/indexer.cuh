@@ -8,48 +8,95 @@
 //     s_t = sum_h w_h * max(0, sigma_t * <q_h, k_t>)
 // for every token t of the sequence's pages.
 //
-// Data path: HBM-bound streaming of 68 B per cached token. One CTA per SM;
-// each warp owns a contiguous run of the flattened (sequence, page) space and
-// runs its own three-slot ring: lane 0 issues bulk copies (cp.async.bulk, no
-// multicast) of a whole 4 KB key page and its 256 B scale row into a slot,
-// completing on that slot's mbarrier, two pages ahead of the page being
-// computed (keys marked evict-first in L2, scores evict-last), so about
-// 140 KB per SM are in flight without holding them in
-// registers and without any cross-warp synchronisation. Page-table entries
-// are resolved 32 pages at a time by one coalesced warp load, one batch
-// ahead. Compute reads the page from shared memory: lane (g, tig) loads
-// channels tig*16 .. tig*16+15 of token rows g and g+8 of each 16-token tile
-// (the page stores 8x16-byte core matrices, so a warp's load covers 512
-// contiguous bytes, free of bank conflicts). The MMA's k index
-// tig*4 + j (+16) is mapped to channel tig*16 + 8*step + j (+4) for the keys
-// and the query alike, which leaves the dot product unchanged. FP8 tensor-core
-// MMA (m16n8k32 e4m3, fp32 accumulate); columns = query token x head. The
-// epilogue applies sigma, ReLU and the head weights, stores the score and adds
-// each valid score's top 11 key bits to a shared-memory histogram per query
-// row (rows past the shared slots go straight to the global histogram).
+// Data path: HBM-bound streaming of 68 B per cached token. One CTA per SM
+// owns a contiguous run of "units" (up to eight consecutive pages of one
+// sequence, 512 tokens) and runs a warp-specialised pipeline:
+//   producer (1 warp)   resolves 32 units at a time (one coalesced
+//        page-table load per lane) and each lane with a unit copies its pages
+//        (4 KB key pages + 256 B scale rows, cp.async.bulk without multicast,
+//        L2 evict-first) into the next of S ring slots once that slot is
+//        free; the slot's "full" mbarrier completes with the bytes.
+//   MMA (1 warp)        one thread issues, per unit, eight tcgen05.mma
+//        kind::f8f6f4 (E4M3 x E4M3 -> fp32; four 128-token blocks x two
+//        32-channel steps, N = 16 query columns) from the slot straight into
+//        one of 4 TMEM accumulators, and one commit (a commit costs several
+//        MMAs' worth of issue time, so units are sized to amortise it). The key pages are stored as 8 x 16-byte core
+//        matrices (byte (t, c) at (t/8)*512 + (c/16)*128 + (t%8)*16 + c%16),
+//        which is the tensor core's no-swizzle K-major operand layout, so
+//        they are used as copied. The query (column n = query token * 4 +
+//        head) is written once per sequence into the same layout.
+//   epilogue (16 warps) 4 groups of 4 warps take the units in turn; warp q
+//        of a group reads TMEM lanes 32q .. 32q+31 of every block (one token
+//        per thread and block, all heads), applies sigma, ReLU and the head weights, stores the
+//        scores (128-byte coalesced, L2 evict-last: the selection re-reads
+//        them) and adds each valid score's top 11 key bits to a shared-memory
+//        histogram per query row (rows past the shared slots go straight to
+//        the global histogram).
+// Every wait is a bounded mbarrier wait; a timeout sets the status word,
+// stops the pipeline and the producer waits (bounded) for its copies before
+// the CTA exits.
 #pragma once
 
 #include "common.cuh"
 
 namespace csa2 {
 
-constexpr int kIdxMaxRing = 4;
 constexpr int kTopkBins = 2048;                 // top 11 bits of the key
 constexpr int kTopkDigitShift = 21;
-constexpr int kIdxSlotBytes = kKidxPageBytes + kPage * 4;
+constexpr int kIdxUnitPages = 8;                           // pages per unit
+constexpr int kIdxBlocks = kIdxUnitPages / 2;               // M = 128-token MMA blocks per unit
+constexpr int kIdxSlotKeys = kIdxUnitPages * kKidxPageBytes;   // 32 KB of keys
+constexpr int kIdxSlotBytes = kIdxSlotKeys + kIdxUnitPages * kPage * 4;   // + scale rows
+constexpr int kIdxEpiWarps = 16;
+constexpr int kIdxGroups = kIdxEpiWarps / 4;
+constexpr int kIdxAccBufs = kIdxGroups;                   // TMEM accumulators, one per group
+constexpr int kIdxAccCols = 16;                           // N = 16 fp32 columns per block
+constexpr int kIdxBufCols = kIdxBlocks * kIdxAccCols;      // one accumulator = all blocks of a unit
+constexpr int kIdxTmemCols = kIdxAccBufs * kIdxBufCols;    // 256
+constexpr int kIdxMmaWarp = kIdxEpiWarps;
+constexpr int kIdxProdWarp = kIdxEpiWarps + 1;
+constexpr int kIdxThreads = (kIdxEpiWarps + 2) * 32;
+constexpr int kIdxQBytes = 16 * kIdxDim;                  // N = 16 rows x 64 B query operand
 
-// Launch shapes: one query token per sequence -> 16 warps and 2 histogram
-// rows; more query tokens -> 12 warps and 8 histogram rows; 3-slot rings.
-struct IdxShape {
-    int warps;
-    int ring;
-    int hist_rows;
+// Ring slots and shared histogram rows per launch shape (one query token per
+// sequence, or more).
+template <int Sq1>
+struct IdxShape;
+template <>
+struct IdxShape<1> {
+    static constexpr int kSlots = 6;
+    static constexpr int kHistRows = 2;
 };
-inline IdxShape idx_shape(int Sq) { return Sq == 1 ? IdxShape{16, 3, 2} : IdxShape{12, 3, 8}; }
-inline size_t idx_smem_bytes(const IdxShape &s) {
-    return static_cast<size_t>(s.warps) * s.ring * (kIdxSlotBytes + 16) +
-           static_cast<size_t>(s.hist_rows) * kTopkBins * 4;
-}
+template <>
+struct IdxShape<0> {
+    static constexpr int kSlots = 4;
+    static constexpr int kHistRows = 8;
+};
+
+struct IdxUnitMeta {
+    int b;          // sequence, or -1: stop mark
+    int p0;         // first logical page
+    int np;         // pages present (1 .. 8)
+    int slot;       // ring slot
+};
+
+template <int Sq1>
+struct IdxSmem {
+    static constexpr int S = IdxShape<Sq1>::kSlots;
+    alignas(128) uint8_t slot[S][kIdxSlotBytes];
+    alignas(128) uint8_t qop[kIdxQBytes];
+    uint32_t hist[IdxShape<Sq1>::kHistRows * kTopkBins];
+    IdxUnitMeta meta[S];
+    IdxUnitMeta acc_meta[kIdxAccBufs];
+    uint64_t full[S];
+    uint64_t empty[S];
+    uint64_t acc_full[kIdxAccBufs];
+    uint64_t acc_empty[kIdxAccBufs];
+    uint64_t q_free;
+    uint32_t tmem_base;
+};
+template <int Sq1>
+constexpr size_t idx_smem_bytes() { return sizeof(IdxSmem<Sq1>) + 128; }
 
 struct IdxArgs {
     const uint8_t *q_idx;        // [B][Sq][4][64]
@@ -65,8 +112,6 @@ struct IdxArgs {
     float *scores;               // [B*Sq][t_cap]
     int64_t t_cap;
     uint32_t *hist;              // [B*Sq][kTopkBins], zero on entry
-    int hist_rows;               // shared-memory histogram rows per CTA
-    int ring;                    // ring slots per warp (<= kIdxMaxRing)
 };
 
 __device__ __forceinline__ int idx_seq_len(const int32_t *seq_lens, int b, int Sq, int max_pages) {
@@ -75,185 +120,331 @@ __device__ __forceinline__ int idx_seq_len(const int32_t *seq_lens, int b, int S
     return T;
 }
 
-__global__ void __launch_bounds__(512, 1)
+// D[tmem] (+)= A[smem] * B[smem] with E4M3 operands, one thread issues.
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// 32 lanes x 4 columns of 32-bit TMEM data: thread i gets lane (base + i).
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
+    uint32_t r[4];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Bounded wait by lane 0 for the whole warp (the result and the memory
+// ordering reach every lane through the broadcast and __syncwarp).
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok;
+}
+
+
+template <int Sq1>
+__global__ void __launch_bounds__(kIdxThreads, 1)
 indexer_score_kernel(const IdxArgs A) {
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    const int n_warps = blockDim.x >> 5;
+    using Sm = IdxSmem<Sq1>;
+    constexpr int S = Sm::S;
+    constexpr int kRows = IdxShape<Sq1>::kHistRows;
+    constexpr int kCols = Sq1 ? 4 : 16;                  // accumulator columns read per token
+    extern __shared__ uint8_t smem_raw[];
+    Sm &sm = *reinterpret_cast<Sm *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~static_cast<uintptr_t>(127));
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, tig = lane & 3;
     const int Sq = A.Sq;
-    const int ring = A.ring;
-    // shared layout: [warps][ring] slots (keys then scales), barriers, meta, histogram
-    uint8_t *slots = smem_raw;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + static_cast<size_t>(n_warps) * ring * kIdxSlotBytes);
-    int2 *metas = reinterpret_cast<int2 *>(bars + n_warps * ring);
-    uint32_t *hist = reinterpret_cast<uint32_t *>(metas + n_warps * ring);
-    uint8_t *my_slots = slots + static_cast<size_t>(warp) * ring * kIdxSlotBytes;
-    uint64_t *my_bars = bars + warp * ring;
-    int2 *my_meta = metas + warp * ring;
 
-    const int64_t n_flat = static_cast<int64_t>(A.B) * A.max_pages;
-    const int64_t cta0 = n_flat * blockIdx.x / gridDim.x;
-    const int64_t cta1 = n_flat * (blockIdx.x + 1) / gridDim.x;
-    const int64_t f_begin = cta0 + (cta1 - cta0) * warp / n_warps;
-    const int64_t f_end = cta0 + (cta1 - cta0) * (warp + 1) / n_warps;
-    const int b_first = static_cast<int>(cta0 / A.max_pages);
+    const int ups = (A.max_pages + kIdxUnitPages - 1) / kIdxUnitPages;   // units per sequence
+    const int64_t n_units = static_cast<int64_t>(A.B) * ups;
+    const int64_t cta0 = n_units * blockIdx.x / gridDim.x;
+    const int64_t cta1 = n_units * (blockIdx.x + 1) / gridDim.x;
+    const int b_first = static_cast<int>(cta0 / ups);
 
-    if (lane == 0) {
-        for (int s = 0; s < ring; ++s) mbar_init(&my_bars[s], 1);
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 4);
+        }
+        for (int i = 0; i < kIdxAccBufs; ++i) {
+            mbar_init(&sm.acc_full[i], 2);
+            mbar_init(&sm.acc_empty[i], 4);
+        }
+        mbar_init(&sm.q_free, 1);
         fence_mbar_init();
     }
-    for (int i = tid; i < A.hist_rows * kTopkBins; i += blockDim.x) hist[i] = 0u;
+    for (int i = tid; i < kRows * kTopkBins; i += blockDim.x) sm.hist[i] = 0u;
+    for (int i = tid; i < kIdxQBytes / 16; i += blockDim.x)
+        reinterpret_cast<uint4 *>(sm.qop)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();                           // the zero rows are read by the tensor core
+    if (warp == kIdxMmaWarp) {
+        tmem_alloc(&sm.tmem_base, kIdxTmemCols);
+        tmem_relinquish();
+    }
     pdl_wait();                                         // cache pages and zeroed histograms are ready
     pdl_trigger();
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
 
-    const int n_tiles = (4 * Sq + 7) / 8;
-    uint4 bq[2];                 // query operand per n-tile: row n = nt*8 + g, channels tig*16 .. +15
-    float wq[2][2];              // head weights of this lane's two accumulator columns
-    int cur_b = -1, cur_T = 0;
-    auto load_query = [&](int b) {
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int n = nt * 8 + g;
-            const int qq = n >> 2, h = n & 3;
-            bq[nt] = make_uint4(0u, 0u, 0u, 0u);
-            if (nt < n_tiles && qq < Sq)
-                bq[nt] = *reinterpret_cast<const uint4 *>(
-                    A.q_idx + ((static_cast<int64_t>(b) * Sq + qq) * kIdxHeads + h) * kIdxDim + tig * 16);
-            const int nc = nt * 8 + tig * 2;
-            const int qc = nc >> 2;
-            wq[nt][0] = wq[nt][1] = 0.0f;
-            if (nt < n_tiles && qc < Sq) {
-                const float *wp = A.w + (static_cast<int64_t>(b) * Sq + qc) * kIdxHeads + (nc & 3);
-                wq[nt][0] = wp[0];
-                wq[nt][1] = wp[1];
-            }
-        }
-    };
-
-    // Per-lane resolution of the 32 pages of batch bi: physical page (-2: no
-    // page to score, -1: bad page-table entry), sequence and logical page.
-    const int64_t n_batches = (f_end - f_begin + 31) / 32;
-    auto resolve = [&](int64_t bi, int64_t &phys, int &pb, int &pp) {
-        phys = -2;
-        pb = 0;
-        pp = 0;
-        const int64_t f = f_begin + bi * 32 + lane;
-        if (bi < n_batches && f < f_end) {
-            pb = static_cast<int>(f / A.max_pages);
-            pp = static_cast<int>(f - static_cast<int64_t>(pb) * A.max_pages);
-            const int T = idx_seq_len(A.seq_lens, pb, Sq, A.max_pages);
+    if (warp == kIdxProdWarp) {
+        // ------------------------------------------------ producer
+        const uint64_t pol_stream = l2_policy_evict_first();
+        int64_t n_issued = 0;                           // units placed in the ring so far
+        bool ok = true;
+        auto slot_wait = [&](int64_t i) -> bool {       // the slot of ring index i is free
+            if (i < S) return true;
+            return mbar_wait_bounded(&sm.empty[i % S], static_cast<uint32_t>((i / S - 1) & 1));
+        };
+        // Lane-parallel resolution of unit u: sequence, first page, pages
+        // present (the prefix below T with good page-table entries) and their
+        // physical pages.
+        struct Unit {
+            int b, p0, np;
+            int32_t ph[kIdxUnitPages];
+        };
+        auto resolve = [&](int64_t u, Unit &r) {
+            r.b = 0;
+            r.p0 = 0;
+            r.np = 0;
+            if (u >= cta1) return;
+            r.b = static_cast<int>(u / ups);
+            r.p0 = static_cast<int>(u - static_cast<int64_t>(r.b) * ups) * kIdxUnitPages;
+            const int T = idx_seq_len(A.seq_lens, r.b, Sq, A.max_pages);
             if (T < 0) {
-                if (pp == 0) flag_status(kStatusBounds);
-            } else if (pp * kPage < T) {
-                const int64_t ph = A.page_table[static_cast<int64_t>(pb) * A.max_pages + pp];
-                if (ph >= 0 && ph < A.num_pages) {
-                    phys = ph;
-                } else {
-                    phys = -1;
-                    flag_status(kStatusBounds);
+                if (r.p0 == 0) flag_status(kStatusBounds);
+                return;
+            }
+            int32_t e[kIdxUnitPages];
+#pragma unroll
+            for (int pg = 0; pg < kIdxUnitPages; ++pg) {       // loads first, checks after
+                const int p = r.p0 + pg;
+                e[pg] = (p < A.max_pages && p * kPage < T) ? A.page_table[static_cast<int64_t>(r.b) * A.max_pages + p]
+                                                           : -2;
+            }
+#pragma unroll
+            for (int pg = 0; pg < kIdxUnitPages; ++pg) {
+                r.ph[pg] = e[pg];
+                if (r.np == pg && e[pg] != -2) {
+                    if (e[pg] >= 0 && e[pg] < A.num_pages) ++r.np;
+                    else flag_status(kStatusBounds);
                 }
             }
+        };
+        Unit cur, nxt;
+        resolve(cta0 + lane, cur);
+        for (int64_t u0 = cta0; u0 < cta1 && ok; u0 += 32) {
+            resolve(u0 + 32 + lane, nxt);               // the next batch's loads overlap this batch's copies
+            const bool live = cur.np > 0;
+            const uint32_t todo = __ballot_sync(0xffffffffu, live);
+            const int rank = __popc(todo & ((1u << lane) - 1u));
+            // Issue in chunks of S ring positions: a lane only waits on a slot
+            // filled by an earlier chunk.
+            for (int c0 = 0; c0 < __popc(todo); c0 += S) {
+                if (live && rank >= c0 && rank < c0 + S) {
+                    const int64_t i = n_issued + rank;
+                    const int s = static_cast<int>(i % S);
+                    if (slot_wait(i)) {
+                        sm.meta[s] = IdxUnitMeta{cur.b, cur.p0, cur.np, s};
+                        uint8_t *dst = sm.slot[s];
+                        mbar_arrive_expect_tx(&sm.full[s], static_cast<uint32_t>((kKidxPageBytes + kPage * 4) * cur.np));
+#pragma unroll
+                        for (int pg = 0; pg < kIdxUnitPages; ++pg) {
+                            if (pg < cur.np) {
+                                const int64_t ph = cur.ph[pg];
+                                bulk_g2s(dst + pg * kKidxPageBytes, A.kidx + ph * kKidxPageBytes, kKidxPageBytes,
+                                         &sm.full[s], pol_stream);
+                                bulk_g2s(dst + kIdxSlotKeys + pg * kPage * 4, A.kidx_scale + ph * kPage, kPage * 4,
+                                         &sm.full[s], pol_stream);
+                            }
+                        }
+                    } else {
+                        ok = false;
+                    }
+                }
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+            }
+            n_issued += __popc(todo);
+            cur = nxt;
         }
-    };
-    int64_t ph_c, ph_n;
-    int pb_c, pp_c, pb_n, pp_n;
-    resolve(0, ph_c, pb_c, pp_c);
-    resolve(1, ph_n, pb_n, pp_n);
-    int64_t bi_issue = 0;
-    uint32_t todo = __ballot_sync(0xffffffffu, ph_c != -2);
-    int issued = 0, consumed = 0;
-    // Keys stream through L2 once; scores are re-read by the selection.
-    const uint64_t pol_stream = l2_policy_evict_first();
-    const uint64_t pol_keep = l2_policy_evict_last();
-
-    auto try_issue = [&]() {
-        while (todo == 0u && bi_issue + 1 < n_batches) {
-            ++bi_issue;
-            ph_c = ph_n;
-            pb_c = pb_n;
-            pp_c = pp_n;
-            resolve(bi_issue + 1, ph_n, pb_n, pp_n);
-            todo = __ballot_sync(0xffffffffu, ph_c != -2);
-        }
-        if (todo == 0u || issued - consumed >= ring) return;
-        const int li = __ffs(todo) - 1;
-        todo &= todo - 1u;
-        const int64_t ph = __shfl_sync(0xffffffffu, ph_c, li);
-        const int b = __shfl_sync(0xffffffffu, pb_c, li);
-        const int p = __shfl_sync(0xffffffffu, pp_c, li);
-        const int slot = issued % ring;
-        if (lane == 0) {
-            my_meta[slot] = make_int2(b, p);
-            uint8_t *dst = my_slots + slot * kIdxSlotBytes;
-            mbar_arrive_expect_tx(&my_bars[slot], ph >= 0 ? static_cast<uint32_t>(kIdxSlotBytes) : 0u);
-            if (ph >= 0) {
-                bulk_g2s(dst, A.kidx + ph * kKidxPageBytes, kKidxPageBytes, &my_bars[slot], pol_stream);
-                bulk_g2s(dst + kKidxPageBytes, A.kidx_scale + ph * kPage, kPage * 4, &my_bars[slot], pol_stream);
+        // One stop mark per epilogue group; the MMA warp forwards them.
+        if (ok && lane < kIdxGroups) {
+            const int64_t i = n_issued + lane;
+            const int s = static_cast<int>(i % S);
+            if (slot_wait(i)) {
+                sm.meta[s] = IdxUnitMeta{-1, 0, 0, s};
+                mbar_arrive(&sm.full[s]);
+            } else {
+                ok = false;
             }
         }
-        ++issued;
-    };
-
-    for (int s = 0; s < ring; ++s) try_issue();
-    while (consumed < issued) {
-        const int slot = consumed % ring;
-        mbar_wait_bounded(&my_bars[slot], (consumed / ring) & 1);
-        __syncwarp();
-        const int2 meta = my_meta[slot];
-        if (meta.x != cur_b) {
-            cur_b = meta.x;
-            cur_T = A.seq_lens[cur_b];
-            load_query(cur_b);
+        // No copy may be in flight when the CTA exits: wait (bounded) for the
+        // last filled phase of every slot.
+        const int64_t n_total = n_issued + kIdxGroups;
+        bool drain = true;                              // after a timeout give up at the first failure
+        for (int s = lane; s < S && s < n_total && drain; s += 32) {
+            const int64_t last = s + (n_total - 1 - s) / S * S;         // last ring index using slot s
+            drain = mbar_wait_bounded(&sm.full[s], static_cast<uint32_t>((last / S) & 1));
         }
-        const uint8_t *kp = my_slots + slot * kIdxSlotBytes;
-        const float *sp = reinterpret_cast<const float *>(kp + kKidxPageBytes);
-        const int hrow0 = (cur_b - b_first) * Sq;          // shared histogram row of query 0
+    } else if (warp == kIdxMmaWarp) {
+        // ------------------------------------------------ MMA issue
+        constexpr uint32_t idesc = umma_idesc_f16(128, kIdxAccCols, false, false);   // E4M3 codes are 0
+        const uint32_t q_addr = smem_u32(sm.qop);
+        int cur_b = -1, stops = 0;
+        uint32_t q_phase = 0u;
+        for (int64_t i = 0; stops < kIdxGroups; ++i) {
+            const int s = static_cast<int>(i % S);
+            const int buf = static_cast<int>(i % kIdxAccBufs);
+            if (!warp_wait(&sm.full[s], static_cast<uint32_t>((i / S) & 1))) break;
+            const IdxUnitMeta m = sm.meta[s];
+            if (i >= kIdxAccBufs && !warp_wait(&sm.acc_empty[buf], static_cast<uint32_t>((i / kIdxAccBufs - 1) & 1)))
+                break;
+            tc_fence_after();
+            if (m.b >= 0 && m.b != cur_b) {
+                // New sequence: every MMA reading the old query must be done
+                // before the operand is rewritten.
+                if (cur_b >= 0) {
+                    if (lane == 0) umma_commit(&sm.q_free);
+                    if (!warp_wait(&sm.q_free, q_phase)) break;
+                    q_phase ^= 1u;
+                }
+                cur_b = m.b;
+                // column n = query token * 4 + head; 16 B chunk c of its 64 channels
+                for (int k = lane; k < 4 * Sq * (kIdxDim / 16); k += 32) {
+                    const int n = k >> 2, c = k & 3;
+                    const uint4 v = *reinterpret_cast<const uint4 *>(
+                        A.q_idx + (static_cast<int64_t>(cur_b) * Sq * kIdxHeads + n) * kIdxDim + c * 16);
+                    *reinterpret_cast<uint4 *>(sm.qop + (n >> 3) * 512 + c * 128 + (n & 7) * 16) = v;
+                }
+                fence_proxy_async_smem();               // generic writes -> tensor-core reads
+                __syncwarp();
+            }
+            if (lane == 0) {
+                sm.acc_meta[buf] = m;
+                if (m.b >= 0) {
+                    const uint32_t a_addr = smem_u32(sm.slot[s]);
 #pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
-            const uint4 r0 = *reinterpret_cast<const uint4 *>(kp + (2 * mt) * 512 + tig * 128 + g * 16);
-            const uint4 r1 = *reinterpret_cast<const uint4 *>(kp + (2 * mt + 1) * 512 + tig * 128 + g * 16);
-            const float s0 = sp[mt * 16 + g], s1 = sp[mt * 16 + g + 8];
-            const int t_lo = meta.y * kPage + mt * 16 + g;
+                    for (int hf = 0; hf < kIdxBlocks; ++hf) {
+                        if (2 * hf < m.np) {
+                            const uint32_t d = tmem + buf * kIdxBufCols + hf * kIdxAccCols;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                if (nt < n_tiles) {
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_e4m3_16832(acc, r0.x, r1.x, r0.y, r1.y, bq[nt].x, bq[nt].y);
-                    mma_e4m3_16832(acc, r0.z, r1.z, r0.w, r1.w, bq[nt].z, bq[nt].w);
-                    const float part0 = wq[nt][0] * fmaxf(0.0f, s0 * acc[0]) + wq[nt][1] * fmaxf(0.0f, s0 * acc[1]);
-                    const float part1 = wq[nt][0] * fmaxf(0.0f, s1 * acc[2]) + wq[nt][1] * fmaxf(0.0f, s1 * acc[3]);
-                    const float oth0 = __shfl_xor_sync(0xffffffffu, part0, 1);
-                    const float oth1 = __shfl_xor_sync(0xffffffffu, part1, 1);
-                    const int qq = nt * 2 + (tig >> 1);
-                    // even tig: token t_lo (heads 0,1 + heads 2,3); odd tig: token t_lo + 8
-                    const int t = t_lo + ((tig & 1) ? 8 : 0);
-                    const float score = (tig & 1) ? oth1 + part1 : part0 + oth0;
+                            for (int ks = 0; ks < kIdxDim / 32; ++ks) {
+                                const uint64_t ad = umma_desc(a_addr + hf * 2 * kKidxPageBytes + ks * 256, 128, 512, 0);
+                                const uint64_t bd = umma_desc(q_addr + ks * 256, 128, 512, 0);
+                                umma_e4m3(d, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                            }
+                        }
+                    }
+                    umma_commit(&sm.acc_full[buf]);
+                } else {
+                    ++stops;
+                    mbar_arrive(&sm.acc_full[buf]);     // stands in for the commit
+                }
+                mbar_arrive(&sm.acc_full[buf]);          // orders acc_meta for the epilogue
+            }
+            stops = __shfl_sync(0xffffffffu, stops, 0);
+        }
+    } else {
+        // ------------------------------------------------ epilogue
+        const int grp = warp >> 2, q = warp & 3;         // TMEM lanes 32q .. 32q+31
+        const uint64_t pol_keep = l2_policy_evict_last();
+        int cur_b = -1, cur_T = 0, hrow0 = 0;
+        float wq[4][4];
+        for (int64_t i = grp;; i += kIdxGroups) {
+            const int buf = static_cast<int>(i % kIdxAccBufs);
+            if (!warp_wait(&sm.acc_full[buf], static_cast<uint32_t>((i / kIdxAccBufs) & 1))) break;
+            tc_fence_after();
+            const IdxUnitMeta m = sm.acc_meta[buf];
+            if (m.b < 0) {
+                if (lane == 0) mbar_arrive(&sm.empty[m.slot]);
+                break;
+            }
+            // this thread: token j of page 2*hf + (q >> 1) of the unit, for every block hf
+            const int j = (q & 1) * 32 + lane;
+            const float *sgp = reinterpret_cast<const float *>(sm.slot[m.slot] + kIdxSlotKeys);
+            float sig[kIdxBlocks];
+#pragma unroll
+            for (int hf = 0; hf < kIdxBlocks; ++hf) sig[hf] = sgp[(2 * hf + (q >> 1)) * kPage + j];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.empty[m.slot]);
+            if (m.b != cur_b) {
+                cur_b = m.b;
+                cur_T = A.seq_lens[cur_b];
+                hrow0 = (cur_b - b_first) * Sq;
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
+                        wq[qq][h] = qq < Sq ? A.w[(static_cast<int64_t>(cur_b) * Sq + qq) * kIdxHeads + h] : 0.0f;
+            }
+            // Scores of this thread's token in block hf from its accumulator row.
+            auto emit = [&](int hf, const float *acc) {
+                const int pg = 2 * hf + (q >> 1);
+                if (pg >= m.np) return;
+                const int t = (m.p0 + pg) * kPage + j;
+                float *srow = A.scores + static_cast<int64_t>(cur_b) * Sq * A.t_cap + t;
+#pragma unroll
+                for (int qq = 0; qq < kCols / 4; ++qq) {
                     if (qq < Sq) {
-                        st_policy(&A.scores[(static_cast<int64_t>(cur_b) * Sq + qq) * A.t_cap + t], score, pol_keep);
+                        float score = 0.0f;
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) score += wq[qq][h] * fmaxf(0.0f, sig[hf] * acc[qq * 4 + h]);
+                        st_policy(srow + qq * A.t_cap, score, pol_keep);
                         if (t <= cur_T - Sq + qq) {
                             const uint32_t bin = float_key(score) >> kTopkDigitShift;
                             const int hr = hrow0 + qq;
-                            if (hr < A.hist_rows) atomicAdd(&hist[hr * kTopkBins + bin], 1u);
+                            if (hr < kRows) atomicAdd(&sm.hist[hr * kTopkBins + bin], 1u);
                             else atomicAdd(&A.hist[(static_cast<int64_t>(cur_b) * Sq + qq) * kTopkBins + bin], 1u);
                         }
                     }
                 }
+            };
+            const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16) + buf * kIdxBufCols;
+            if constexpr (kCols == 4) {
+                // all blocks to registers, release the accumulator, then score
+                float acc[kIdxBlocks][4];
+#pragma unroll
+                for (int hf = 0; hf < kIdxBlocks; ++hf) tmem_ld4(trow + hf * kIdxAccCols, acc[hf]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
+#pragma unroll
+                for (int hf = 0; hf < kIdxBlocks; ++hf) emit(hf, acc[hf]);
+            } else {
+                // 16 columns per block: one block at a time keeps registers low
+#pragma unroll
+                for (int hf = 0; hf < kIdxBlocks; ++hf) {
+                    float acc[16];
+                    tmem_ld16(trow + hf * kIdxAccCols, acc);
+                    emit(hf, acc);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
             }
         }
-        __syncwarp();                                   // every lane is done with the slot
-        ++consumed;
-        try_issue();
     }
-
+    tc_fence_before();
     __syncthreads();
+    if (warp == kIdxMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kIdxTmemCols);
+    }
     // Flush the shared histograms of the rows this CTA touched.
-    const int b_last = static_cast<int>((cta1 > cta0 ? cta1 - 1 : cta0) / A.max_pages);
-    const int n_rows = min(A.hist_rows, (b_last - b_first + 1) * Sq);
+    const int b_last = static_cast<int>((cta1 > cta0 ? cta1 - 1 : cta0) / ups);
+    const int n_rows = min(kRows, (b_last - b_first + 1) * Sq);
     for (int i = tid; i < n_rows * kTopkBins; i += blockDim.x) {
-        const uint32_t c = hist[i];
+        const uint32_t c = sm.hist[i];
         if (c) atomicAdd(&A.hist[static_cast<int64_t>(b_first) * Sq * kTopkBins + i], c);
     }
 }

@@ -111,6 +111,10 @@ __device__ __forceinline__ void find_threshold_bin(const uint32_t *__restrict__ 
         c[i] = __ldcg(&gh[top - i]);
         local += c[i];
     }
+    if (threadIdx.x == 0) {                 // stays if the counts fall short of need (corrupt input)
+        *s_bin = 0;
+        *s_above = 0u;
+    }
     uint32_t tot;
     uint32_t run = block_excl_scan<NT>(local, wbuf, &tot);
 #pragma unroll
@@ -149,6 +153,10 @@ struct TkSmem {
 __device__ __forceinline__ void tk_pick(TkSmem &sm, const uint32_t *h, int nbins, uint32_t need, uint32_t &digit,
                                         uint32_t &above) {
     const int top = kTopkBins - 1 - static_cast<int>(threadIdx.x) * 2;
+    if (threadIdx.x == 0) {                 // stays if the counts fall short of need (corrupt input)
+        sm.s_digit = 0u;
+        sm.s_cum = 0u;
+    }
     const uint32_t c0 = top < nbins ? h[top] : 0u;
     const uint32_t c1 = top - 1 < nbins ? h[top - 1] : 0u;
     uint32_t tot;
