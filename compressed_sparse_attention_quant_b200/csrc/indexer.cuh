@@ -16,7 +16,9 @@
 //        (4 KB key pages + 256 B scale rows, cp.async.bulk without multicast,
 //        L2 evict-first) into the next of S ring slots once that slot is
 //        free; the slot's "full" mbarrier completes with the bytes.
-//   MMA (1 warp)        one thread issues, per unit, eight tcgen05.mma
+//   MMA (2 warps)       units alternate between two issuing threads (the
+//        per-unit waits and the commit, not the tensor core, bound one
+//        thread); each issues, per unit, eight tcgen05.mma
 //        kind::f8f6f4 (E4M3 x E4M3 -> fp32; four 128-token blocks x two
 //        32-channel steps, N = 16 query columns) from the slot straight into
 //        one of 4 TMEM accumulators, and one commit (a commit costs several
@@ -53,9 +55,10 @@ constexpr int kIdxAccBufs = kIdxGroups;                   // TMEM accumulators, 
 constexpr int kIdxAccCols = 16;                           // N = 16 fp32 columns per block
 constexpr int kIdxBufCols = kIdxBlocks * kIdxAccCols;      // one accumulator = all blocks of a unit
 constexpr int kIdxTmemCols = kIdxAccBufs * kIdxBufCols;    // 256
-constexpr int kIdxMmaWarp = kIdxEpiWarps;
-constexpr int kIdxProdWarp = kIdxEpiWarps + 1;
-constexpr int kIdxThreads = (kIdxEpiWarps + 2) * 32;
+constexpr int kIdxMmaWarps = 2;
+constexpr int kIdxMmaWarp = kIdxEpiWarps;                 // first MMA warp
+constexpr int kIdxProdWarp = kIdxEpiWarps + kIdxMmaWarps;
+constexpr int kIdxThreads = (kIdxEpiWarps + kIdxMmaWarps + 1) * 32;
 constexpr int kIdxQBytes = 16 * kIdxDim;                  // N = 16 rows x 64 B query operand
 
 // Ring slots and shared histogram rows per launch shape (one query token per
@@ -84,7 +87,7 @@ template <int Sq1>
 struct IdxSmem {
     static constexpr int S = IdxShape<Sq1>::kSlots;
     alignas(128) uint8_t slot[S][kIdxSlotBytes];
-    alignas(128) uint8_t qop[kIdxQBytes];
+    alignas(128) uint8_t qop[kIdxMmaWarps][kIdxQBytes];   // query operand per MMA warp
     uint32_t hist[IdxShape<Sq1>::kHistRows * kTopkBins];
     IdxUnitMeta meta[S];
     IdxUnitMeta acc_meta[kIdxAccBufs];
@@ -92,7 +95,7 @@ struct IdxSmem {
     uint64_t empty[S];
     uint64_t acc_full[kIdxAccBufs];
     uint64_t acc_empty[kIdxAccBufs];
-    uint64_t q_free;
+    uint64_t q_free[kIdxMmaWarps];
     uint32_t tmem_base;
 };
 template <int Sq1>
@@ -178,12 +181,12 @@ indexer_score_kernel(const IdxArgs A) {
             mbar_init(&sm.acc_full[i], 2);
             mbar_init(&sm.acc_empty[i], 4);
         }
-        mbar_init(&sm.q_free, 1);
+        for (int i = 0; i < kIdxMmaWarps; ++i) mbar_init(&sm.q_free[i], 1);
         fence_mbar_init();
     }
     for (int i = tid; i < kRows * kTopkBins; i += blockDim.x) sm.hist[i] = 0u;
-    for (int i = tid; i < kIdxQBytes / 16; i += blockDim.x)
-        reinterpret_cast<uint4 *>(sm.qop)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = tid; i < kIdxMmaWarps * kIdxQBytes / 16; i += blockDim.x)
+        reinterpret_cast<uint4 *>(&sm.qop[0][0])[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();                           // the zero rows are read by the tensor core
     if (warp == kIdxMmaWarp) {
         tmem_alloc(&sm.tmem_base, kIdxTmemCols);
@@ -296,13 +299,15 @@ indexer_score_kernel(const IdxArgs A) {
             const int64_t last = s + (n_total - 1 - s) / S * S;         // last ring index using slot s
             drain = mbar_wait_bounded(&sm.full[s], static_cast<uint32_t>((last / S) & 1));
         }
-    } else if (warp == kIdxMmaWarp) {
-        // ------------------------------------------------ MMA issue
+    } else if (warp >= kIdxMmaWarp) {
+        // ------------------------------------------------ MMA issue: units i = mw, mw + 2, ...
+        const int mw = warp - kIdxMmaWarp;
         constexpr uint32_t idesc = umma_idesc_f16(128, kIdxAccCols, false, false);   // E4M3 codes are 0
-        const uint32_t q_addr = smem_u32(sm.qop);
+        uint8_t *qop = sm.qop[mw];
+        const uint32_t q_addr = smem_u32(qop);
         int cur_b = -1, stops = 0;
         uint32_t q_phase = 0u;
-        for (int64_t i = 0; stops < kIdxGroups; ++i) {
+        for (int64_t i = mw; stops < kIdxGroups / kIdxMmaWarps; i += kIdxMmaWarps) {
             const int s = static_cast<int>(i % S);
             const int buf = static_cast<int>(i % kIdxAccBufs);
             if (!warp_wait(&sm.full[s], static_cast<uint32_t>((i / S) & 1))) break;
@@ -314,8 +319,8 @@ indexer_score_kernel(const IdxArgs A) {
                 // New sequence: every MMA reading the old query must be done
                 // before the operand is rewritten.
                 if (cur_b >= 0) {
-                    if (lane == 0) umma_commit(&sm.q_free);
-                    if (!warp_wait(&sm.q_free, q_phase)) break;
+                    if (lane == 0) umma_commit(&sm.q_free[mw]);
+                    if (!warp_wait(&sm.q_free[mw], q_phase)) break;
                     q_phase ^= 1u;
                 }
                 cur_b = m.b;
@@ -324,7 +329,7 @@ indexer_score_kernel(const IdxArgs A) {
                     const int n = k >> 2, c = k & 3;
                     const uint4 v = *reinterpret_cast<const uint4 *>(
                         A.q_idx + (static_cast<int64_t>(cur_b) * Sq * kIdxHeads + n) * kIdxDim + c * 16);
-                    *reinterpret_cast<uint4 *>(sm.qop + (n >> 3) * 512 + c * 128 + (n & 7) * 16) = v;
+                    *reinterpret_cast<uint4 *>(qop + (n >> 3) * 512 + c * 128 + (n & 7) * 16) = v;
                 }
                 fence_proxy_async_smem();               // generic writes -> tensor-core reads
                 __syncwarp();
@@ -436,7 +441,7 @@ indexer_score_kernel(const IdxArgs A) {
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == kIdxMmaWarp) {
+    if (warp == kIdxMmaWarp) {                         // the allocating warp frees TMEM
         tc_fence_after();
         tmem_dealloc(tmem, kIdxTmemCols);
     }
