@@ -29,7 +29,7 @@ if ROOT not in sys.path:
 
 import torch  # noqa: E402
 
-from compressed_sparse_attention_quant_b200 import inputs  # noqa: E402
+from compressed_sparse_attention_quant_b200 import inputs, replicas  # noqa: E402
 
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
@@ -211,7 +211,7 @@ def cpu_baseline(wl: inputs.Workload, n_seqs: int, budget_s: float) -> dict:
 
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    if not replicas.reports(rank):
         return                      # the oracle arm runs on rank 0 only
     arm = OracleArm(wl, args.ref_seqs)
     arm.prepare()
@@ -250,7 +250,7 @@ def run_gpu(args, wl):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     # Each rank runs its own replica (different seed): weak scaling.
-    wl_r = inputs.Workload(**{**wl.__dict__, "seed": wl.seed + 1000 * rank}) if rank else wl
+    wl_r = replicas.replica_workload(wl, rank)
     dw = workload.DeviceWorkload(wl_r, dev)
     g = dw.group
     stream = torch.cuda.current_stream(dev)
@@ -339,13 +339,10 @@ def run_gpu(args, wl):
     torch.cuda.synchronize(dev)
     e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_events) / args.steps
 
-    times = torch.tensor([step_ms, idx_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    step_ms, idx_ms, e2e_ms = times.tolist()
+    step_ms, idx_ms, e2e_ms = replicas.max_over_ranks([step_ms, idx_ms, e2e_ms], dist, dev)
 
     tokens_per_rank = wl.batch * wl.q_tokens
-    value = tokens_per_rank * world / (step_ms * 1e-3)
+    value = replicas.job_throughput(tokens_per_rank, world, step_ms)
     hbm, peak_kind = peaks()
     idx_bytes = (acct["indexer"] + acct["topk_io"]) / max(n_idx_calls, 1)
     achieved = idx_bytes / (idx_ms * 1e-3) / 1e9
@@ -365,7 +362,7 @@ def run_gpu(args, wl):
                      "achieved": achieved, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic, "ms_per_launch": idx_ms,
                      "algorithmic_bytes_per_launch": idx_bytes},
-        "e2e": {"value": tokens_per_rank * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": replicas.job_throughput(tokens_per_rank, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "device_status": lib.status_string(status),
@@ -378,7 +375,7 @@ def run_gpu(args, wl):
     if dist:
         dist.barrier()
         dist.destroy_process_group()
-    if rank == 0:
+    if replicas.reports(rank):
         print(json.dumps(line), flush=True)
 
 
