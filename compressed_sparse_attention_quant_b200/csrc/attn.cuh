@@ -8,7 +8,7 @@
 //
 // One CTA (8 warps, two CTAs per SM) per (query token, split of its key
 // list). The key list is the k selected positions followed by the 128 window
-// rows; a split owns a run of at most 6 tiles of 64 keys.
+// rows; a split owns a run of at most 12 tiles of 64 keys.
 //   set-up   the split's selected positions are resolved once to physical
 //            cache slots (top-k index -> page table) in a shared table;
 //   prefetch right after a tile is dequantized, cp.async (16-byte and 4-byte
@@ -38,14 +38,14 @@ constexpr int kAttThreads = 256;
 constexpr int kAttTile = 64;
 constexpr int kKhRow = kDim * 2;            // 1152 bytes per f16 key row (no padding: swizzled chunks)
 constexpr int kPPitch = kAttTile + 8;       // halfs per probability row
-constexpr int kMaxTilesPerSplit = 6;
+constexpr int kMaxTilesPerSplit = 12;
 
 struct AttSmem {
     alignas(128) uint8_t kh[kAttTile * kKhRow];            // 73,728: f16 keys / values
     alignas(16) float red[8][16][32];                      // 16,384: QK partials; P reuses the start
     alignas(16) uint8_t raw[kAttTile][kFp4Bytes];          // 18,432: staged packed FP4 of the next tile
     alignas(16) uint8_t rsc[kAttTile][kScaleBytes];        // 2,304: staged scales of the next tile
-    int slot[kMaxTilesPerSplit * kAttTile];                // 1,536: physical slot of each selected key
+    int slot[kMaxTilesPerSplit * kAttTile];                // 3,072: physical slot of each selected key
     float m_run[16];
     float l_run[16];
     float alpha[16];
@@ -118,7 +118,7 @@ sparse_attn_kernel(const AttParams P) {
     // Physical slots of this split's selected keys: all index loads first,
     // then all page-table loads, so only two load latencies are exposed.
     {
-        constexpr int kPer = (kMaxTilesPerSplit * kAttTile + kAttThreads - 1) / kAttThreads;   // 2
+        constexpr int kPer = (kMaxTilesPerSplit * kAttTile + kAttThreads - 1) / kAttThreads;   // 3
         int ti[kPer];
 #pragma unroll
         for (int u = 0; u < kPer; ++u) {
