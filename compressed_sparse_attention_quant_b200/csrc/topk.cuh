@@ -234,6 +234,13 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     uint32_t need = static_cast<uint32_t>(k) - above1;
 
     // ---- pass A: sure bits, level-2 histogram, candidate list
+    // With a positive threshold bin (1024 < b1 < 2047) a score is above b1,
+    // or in b1, exactly when its IEEE bits as a signed integer are at least
+    // hi_bits, or in [lo_bits, hi_bits): negative scores and -0 fall below
+    // both. That skips the key transform for all but the candidates.
+    const bool pos = b1 > 1024 && b1 < kTopkBins - 1;
+    const int32_t lo_bits = (b1 - 1024) << kTopkDigitShift;
+    const int32_t hi_bits = (b1 - 1023) << kTopkDigitShift;
     for (int r = 0; r < rounds; ++r) {
         int64_t w0, w1;
         int n_it;
@@ -250,15 +257,30 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
                 const int64_t p = w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) + tid * 4;
                 const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
                 uint32_t s4 = 0u;
+                if (pos) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const uint32_t key = float_key(fv[e]);
-                    const int bin = static_cast<int>(key >> kTopkDigitShift);
-                    if (i0 + u < n_it && p + e < w1) {
-                        if (bin > b1) s4 |= 1u << e;
-                        if (bin == b1) {
-                            cmask |= 1u << (4 * u + e);
-                            atomicAdd(&sm.hloc[0][(key >> 10) & (kTopkBins - 1)], 1u);
+                    for (int e = 0; e < 4; ++e) {
+                        const int32_t bits = __float_as_int(fv[e]);
+                        if (i0 + u < n_it && p + e < w1 && bits >= lo_bits) {
+                            if (bits >= hi_bits) {
+                                s4 |= 1u << e;
+                            } else {
+                                cmask |= 1u << (4 * u + e);
+                                atomicAdd(&sm.hloc[0][(static_cast<uint32_t>(bits) >> 10) & (kTopkBins - 1)], 1u);
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t key = float_key(fv[e]);
+                        const int bin = static_cast<int>(key >> kTopkDigitShift);
+                        if (i0 + u < n_it && p + e < w1) {
+                            if (bin > b1) s4 |= 1u << e;
+                            if (bin == b1) {
+                                cmask |= 1u << (4 * u + e);
+                                atomicAdd(&sm.hloc[0][(key >> 10) & (kTopkBins - 1)], 1u);
+                            }
                         }
                     }
                 }
