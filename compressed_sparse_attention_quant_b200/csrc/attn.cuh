@@ -199,10 +199,23 @@ sparse_attn_kernel(const AttParams P) {
                     // chunks of a record chunk in the order 2,3,0,1, so the
                     // 8 lanes of each 128-bit store phase hit 8 bank groups.
                     const bool rot = (gpart & 2) != 0;
-                    for (int c = gpart; c < kFp4Bytes / 16; c += 4) {   // 16-byte chunk = 32 channels
-                        const uint4 raw = *reinterpret_cast<const uint4 *>(&sm.raw[gkey][c * 16]);
-                        const uint32_t sc = *reinterpret_cast<const unsigned short *>(&sm.rsc[gkey][c * 2]);
-                        const uint32_t sf = e4m3x2_to_f16x2(sc);                 // (scale 2c, scale 2c+1)
+                    // Record chunks c = gpart + 4i, software-pipelined: the
+                    // next chunk's shared loads are issued before this one is
+                    // converted.
+                    constexpr int kCh = (kFp4Bytes / 16 + 3) / 4;           // 5
+                    uint4 raw_n = *reinterpret_cast<const uint4 *>(&sm.raw[gkey][gpart * 16]);
+                    uint32_t sc_n = *reinterpret_cast<const unsigned short *>(&sm.rsc[gkey][gpart * 2]);
+#pragma unroll
+                    for (int i = 0; i < kCh; ++i) {
+                        const int c = gpart + 4 * i;
+                        if (c >= kFp4Bytes / 16) break;
+                        const uint4 raw = raw_n;
+                        const uint32_t scv = sc_n;
+                        if (c + 4 < kFp4Bytes / 16) {
+                            raw_n = *reinterpret_cast<const uint4 *>(&sm.raw[gkey][(c + 4) * 16]);
+                            sc_n = *reinterpret_cast<const unsigned short *>(&sm.rsc[gkey][(c + 4) * 2]);
+                        }
+                        const uint32_t sf = e4m3x2_to_f16x2(scv);                // (scale 2c, scale 2c+1)
                         const uint32_t s_lo = __byte_perm(sf, 0, 0x1010);
                         const uint32_t s_hi = __byte_perm(sf, 0, 0x3232);
                         const uint32_t w[4] = {rot ? raw.z : raw.x, rot ? raw.w : raw.y,
