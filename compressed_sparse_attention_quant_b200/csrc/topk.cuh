@@ -95,6 +95,38 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *wbuf, 
     return res;
 }
 
+// Exclusive block scan of a pair of counts packed in 64 bits (one scan for
+// two quantities). wbuf holds >= nwarps + 1 entries.
+template <int NT>
+__device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t *wbuf, uint64_t *total) {
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint64_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) wbuf[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const uint64_t wv = lane < NW ? wbuf[lane] : 0ull;
+        uint64_t wi = wv;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint64_t y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += y;
+        }
+        if (lane < NW) wbuf[lane] = wi - wv;
+        if (lane == NW - 1) wbuf[NW] = wi;
+    }
+    __syncthreads();
+    const uint64_t res = wbuf[warp] + incl - v;
+    *total = wbuf[NW];
+    __syncthreads();
+    return res;
+}
+
 // From the row's 2048-bin histogram (global), the bin holding the need-th
 // largest key, and how many keys lie in higher bins. Every thread of the
 // block gets the answer.
@@ -138,6 +170,7 @@ struct TkSmem {
     uint32_t hloc[2][kTopkBins];        // this CTA's level-2 / level-3 histograms (read by peers)
     uint32_t hsum[kTopkBins];           // cluster-wide sum of the current level
     uint32_t wbuf[kTkThreads / 32 + 1];
+    uint64_t wbuf64[kTkThreads / 32 + 1];
     uint32_t xchg[2][2];                // per round parity: (selected before ties, ties), read by peers
     uint32_t n_cand;
     int s_bin;
@@ -257,7 +290,22 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
                 const int64_t p = w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) + tid * 4;
                 const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
                 uint32_t s4 = 0u;
-                if (pos) {
+                // one bounds check per float4; per element only on the ragged tail
+                const bool full4 = i0 + u < n_it && p + 4 <= w1;
+                if (pos && full4) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int32_t bits = __float_as_int(fv[e]);
+                        if (bits >= lo_bits) {
+                            if (bits >= hi_bits) {
+                                s4 |= 1u << e;
+                            } else {
+                                cmask |= 1u << (4 * u + e);
+                                atomicAdd(&sm.hloc[0][(static_cast<uint32_t>(bits) >> 10) & (kTopkBins - 1)], 1u);
+                            }
+                        }
+                    }
+                } else if (pos) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int32_t bits = __float_as_int(fv[e]);
@@ -426,9 +474,10 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
             n_tie += __popc(sm.tie[i]);
             n_sel += __popc(sm.sel[i]);
         }
-        uint32_t cta_ties, cta_sel;
-        const uint32_t tie_off = block_excl_scan<kTkThreads>(n_tie, sm.wbuf, &cta_ties);
-        block_excl_scan<kTkThreads>(n_sel, sm.wbuf, &cta_sel);
+        uint64_t tot2;                                   // (ties, selected) in one scan
+        const uint32_t tie_off = static_cast<uint32_t>(
+            block_excl_scan64<kTkThreads>((static_cast<uint64_t>(n_tie) << 32) | n_sel, sm.wbuf64, &tot2) >> 32);
+        const uint32_t cta_ties = static_cast<uint32_t>(tot2 >> 32), cta_sel = static_cast<uint32_t>(tot2);
         if (tid == 0) {
             sm.xchg[r & 1][0] = cta_sel;
             sm.xchg[r & 1][1] = cta_ties;
