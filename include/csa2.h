@@ -157,6 +157,10 @@ csa2_status csa2_quant_kv_fp4(const void *x_bf16, int64_t n_tok, int dim,
  *   ws          device workspace of at least csa2_indexer_topk_workspace_bytes()
  *               bytes, 256-byte aligned; contents need no initialisation and
  *               are clobbered.
+ *
+ * Limits (else CSA2_ERR_UNSUPPORTED): 4 indexer heads x 64 channels,
+ * Sq <= 4, B * Sq <= 65535, 64 * max_pages <= 2^30, cache->num_pages <=
+ * INT32_MAX (physical page indices are int32).
  */
 size_t csa2_indexer_topk_workspace_bytes(int B, int Sq, int max_pages, int k);
 csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq,

@@ -93,6 +93,24 @@ def test_topk_heavy_ties_against_oracle(mods):
         np.testing.assert_array_equal(idx[b, 0], ref.out[0][(b, 0)]["idx"], err_msg=f"b {b}")
 
 
+def test_topk_negative_scores_against_oracle(mods):
+    """Negative head weights make every score <= 0, so the threshold bin lies
+    among negative keys (the selection's general key path, not the
+    positive-bits shortcut); -0 and +0 scores must tie. Indices must match
+    the oracle exactly."""
+    lib, workload = mods
+    wl = inputs.small_workload("negw", 3, 2, [9000, 4000, 700], 300, modes=("F",), seed=21)
+    dw = workload.DeviceWorkload(wl)
+    dw.w[0].neg_()
+    dw.step()
+    assert lib.last_device_error() == 0
+    ref = OracleRun(dw, range(3))
+    idx = dw.group.index(0).cpu().numpy()
+    for b in range(3):
+        for j in range(2):
+            np.testing.assert_array_equal(idx[b, j], ref.out[0][(b, j)]["idx"], err_msg=f"b {b} j {j}")
+
+
 def test_topk_rows_longer_than_one_window(mods):
     """80 query rows give one CTA per row, and rows longer than 2^17 positions
     are then covered in two rounds of windows; shorter rows in the same
