@@ -53,7 +53,8 @@ class LayerGroup:
 
     def step(self, page_table: torch.Tensor, seq_lens: torch.Tensor, q: List[torch.Tensor],
              swa: List[torch.Tensor], q_idx: Dict[int, torch.Tensor], w: Dict[int, torch.Tensor],
-             append: Optional[Dict[int, tuple]] = None) -> None:
+             append: Optional[Dict[int, tuple]] = None, out: Optional[List[torch.Tensor]] = None,
+             lse: Optional[List[torch.Tensor]] = None) -> None:
         """One decode step over every layer of the group, on the current stream.
 
         q[l], swa[l]: layer l's attention query and window rows.
@@ -61,7 +62,10 @@ class LayerGroup:
         append[l] = (x_new [n,576] bf16, slots [n] int32, kidx_new [n,64] u8,
                      ksig_new [n] f32): the new tokens a Full layer writes into
                      its cache before it indexes (None: cache already holds them).
+        out[l], lse[l]: where layer l writes its output (default self.out, self.lse).
         """
+        out = self.out if out is None else out
+        lse = self.lse if lse is None else lse
         for li, mode in enumerate(self.modes):
             cache = self.cache(li)
             if mode == "F" and append is not None and li in append:
@@ -71,4 +75,4 @@ class LayerGroup:
                 lib.indexer_topk(q_idx[li], w[li], cache, page_table, seq_lens, self.k,
                                  out=self._index[li], ws=self.ws_idx)
             lib.sparse_attn_decode(q[li], cache, page_table, seq_lens, self.index(li), swa[li], self.scale,
-                                   out=self.out[li], lse=self.lse[li], ws=self.ws_att)
+                                   out=out[li], lse=lse[li], ws=self.ws_att)
