@@ -74,6 +74,11 @@ struct AttParams {
     int tiles_per_split;
 };
 
+// Pull the 128-byte line holding p into L2 (no register result).
+__device__ __forceinline__ void prefetch_l2_line(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Byte offset of 8-channel chunk `chunk` (0..71) of key row `key`: chunks are
 // XOR-swizzled by the key's low 3 bits so that the 8 rows an ldmatrix reads
 // fall in 8 different bank groups.
@@ -97,10 +102,30 @@ sparse_attn_kernel(const AttParams P) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, tig = lane & 3;
     const int n_rows_swa = kWindow + P.Sq - 1;
+
+    // Inputs that no earlier kernel of the step writes are read before the
+    // wait for the selection: the query fragments, the sequence length and
+    // (into L2) the sequence's page-table row.
+    // Query fragments for QK: warp (kg, cq) covers channels cq*144 .. +143.
+    const int kg = warp >> 2, cq = warp & 3;
+    uint32_t qa[9][4];
+    {
+        const __nv_bfloat16 *qrow = P.q + static_cast<int64_t>(row) * kHeads * kDim;
+#pragma unroll
+        for (int ks = 0; ks < 9; ++ks) {
+            const int cb = cq * 144 + ks * 16 + tig * 2;
+            qa[ks][0] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + g * kDim + cb));
+            qa[ks][1] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + (g + 8) * kDim + cb));
+            qa[ks][2] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + g * kDim + cb + 8));
+            qa[ks][3] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + (g + 8) * kDim + cb + 8));
+        }
+    }
+    int T = P.seq_lens[b];
+    for (int i = tid * 32; i < P.max_pages; i += kAttThreads * 32)           // 128-byte lines of the row
+        prefetch_l2_line(P.page_table + static_cast<int64_t>(b) * P.max_pages + i);
     pdl_wait();                                         // the selection's indices are ready
     pdl_trigger();
 
-    int T = P.seq_lens[b];
     if (T < P.Sq || T > P.max_pages * kPage) {
         if (tid == 0 && split == 0) flag_status(kStatusBounds);
         T = -1;                                          // no valid key at all
@@ -150,20 +175,6 @@ sparse_attn_kernel(const AttParams P) {
         }
     }
 
-    // Query fragments for QK: warp (kg, cq) covers channels cq*144 .. +143.
-    const int kg = warp >> 2, cq = warp & 3;
-    uint32_t qa[9][4];
-    {
-        const __nv_bfloat16 *qrow = P.q + static_cast<int64_t>(row) * kHeads * kDim;
-#pragma unroll
-        for (int ks = 0; ks < 9; ++ks) {
-            const int cb = cq * 144 + ks * 16 + tig * 2;
-            qa[ks][0] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + g * kDim + cb));
-            qa[ks][1] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + (g + 8) * kDim + cb));
-            qa[ks][2] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + g * kDim + cb + 8));
-            qa[ks][3] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + (g + 8) * kDim + cb + 8));
-        }
-    }
     float o[9][4];
 #pragma unroll
     for (int nt = 0; nt < 9; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.0f;
