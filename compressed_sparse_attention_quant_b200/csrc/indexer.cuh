@@ -192,6 +192,45 @@ indexer_score_kernel(const IdxArgs A) {
         tmem_alloc(&sm.tmem_base, kIdxTmemCols);
         tmem_relinquish();
     }
+    // Lane-parallel resolution of unit u: sequence, first page, pages
+    // present (the prefix below T with good page-table entries) and their
+    // physical pages.
+    struct Unit {
+        int b, p0, np;
+        int32_t ph[kIdxUnitPages];
+    };
+    auto resolve = [&](int64_t u, Unit &r) {
+        r.b = 0;
+        r.p0 = 0;
+        r.np = 0;
+        if (u >= cta1) return;
+        r.b = static_cast<int>(u / ups);
+        r.p0 = static_cast<int>(u - static_cast<int64_t>(r.b) * ups) * kIdxUnitPages;
+        const int T = idx_seq_len(A.seq_lens, r.b, Sq, A.max_pages);
+        if (T < 0) {
+            if (r.p0 == 0) flag_status(kStatusBounds);
+            return;
+        }
+        int32_t e[kIdxUnitPages];
+#pragma unroll
+        for (int pg = 0; pg < kIdxUnitPages; ++pg) {       // loads first, checks after
+            const int p = r.p0 + pg;
+            e[pg] = (p < A.max_pages && p * kPage < T) ? A.page_table[static_cast<int64_t>(r.b) * A.max_pages + p]
+                                                       : -2;
+        }
+#pragma unroll
+        for (int pg = 0; pg < kIdxUnitPages; ++pg) {
+            r.ph[pg] = e[pg];
+            if (r.np == pg && e[pg] != -2) {
+                if (e[pg] >= 0 && e[pg] < A.num_pages) ++r.np;
+                else flag_status(kStatusBounds);
+            }
+        }
+    };
+    // The page table and sequence lengths are inputs no earlier kernel of the
+    // step writes: the producer resolves its first batch before the wait.
+    Unit cur;
+    if (warp == kIdxProdWarp) resolve(cta0 + lane, cur);
     pdl_wait();                                         // cache pages and zeroed histograms are ready
     pdl_trigger();
     tc_fence_before();
@@ -208,43 +247,7 @@ indexer_score_kernel(const IdxArgs A) {
             if (i < S) return true;
             return mbar_wait_bounded(&sm.empty[i % S], static_cast<uint32_t>((i / S - 1) & 1));
         };
-        // Lane-parallel resolution of unit u: sequence, first page, pages
-        // present (the prefix below T with good page-table entries) and their
-        // physical pages.
-        struct Unit {
-            int b, p0, np;
-            int32_t ph[kIdxUnitPages];
-        };
-        auto resolve = [&](int64_t u, Unit &r) {
-            r.b = 0;
-            r.p0 = 0;
-            r.np = 0;
-            if (u >= cta1) return;
-            r.b = static_cast<int>(u / ups);
-            r.p0 = static_cast<int>(u - static_cast<int64_t>(r.b) * ups) * kIdxUnitPages;
-            const int T = idx_seq_len(A.seq_lens, r.b, Sq, A.max_pages);
-            if (T < 0) {
-                if (r.p0 == 0) flag_status(kStatusBounds);
-                return;
-            }
-            int32_t e[kIdxUnitPages];
-#pragma unroll
-            for (int pg = 0; pg < kIdxUnitPages; ++pg) {       // loads first, checks after
-                const int p = r.p0 + pg;
-                e[pg] = (p < A.max_pages && p * kPage < T) ? A.page_table[static_cast<int64_t>(r.b) * A.max_pages + p]
-                                                           : -2;
-            }
-#pragma unroll
-            for (int pg = 0; pg < kIdxUnitPages; ++pg) {
-                r.ph[pg] = e[pg];
-                if (r.np == pg && e[pg] != -2) {
-                    if (e[pg] >= 0 && e[pg] < A.num_pages) ++r.np;
-                    else flag_status(kStatusBounds);
-                }
-            }
-        };
-        Unit cur, nxt;
-        resolve(cta0 + lane, cur);
+        Unit nxt;
         for (int64_t u0 = cta0; u0 < cta1 && ok; u0 += 32) {
             resolve(u0 + 32 + lane, nxt);               // the next batch's loads overlap this batch's copies
             const bool live = cur.np > 0;
