@@ -305,7 +305,7 @@ indexer_score_kernel(const IdxArgs A) {
     } else if (warp >= kIdxMmaWarp) {
         // ------------------------------------------------ MMA issue: units i = mw, mw + 2, ...
         const int mw = warp - kIdxMmaWarp;
-        constexpr uint32_t idesc = umma_idesc_f16(128, kIdxAccCols, false, false);   // E4M3 codes are 0
+        constexpr uint32_t idesc = umma_idesc(128, kIdxAccCols, false, false);   // E4M3 x E4M3, fp32
         uint8_t *qop = sm.qop[mw];
         const uint32_t q_addr = smem_u32(qop);
         int cur_b = -1, stops = 0;
