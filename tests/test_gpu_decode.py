@@ -79,8 +79,9 @@ def test_topk_ties_go_to_lower_index(mods):
 
 def test_topk_heavy_ties_against_oracle(mods):
     """Indexer queries with a single non-zero channel: scores take few
-    distinct values, so the threshold bin is crowded (overflow path on the
-    long row, candidate path on the short ones); indices must match."""
+    distinct values, so the threshold bin is crowded and many positions tie
+    at the threshold key (tie ranking across the CTAs of a row); indices
+    must match the oracle."""
     lib, workload = mods
     wl = inputs.small_workload("crowd", 3, 1, [30000, 6000, 2500], 700, modes=("F",), seed=5)
     dw = workload.DeviceWorkload(wl)
