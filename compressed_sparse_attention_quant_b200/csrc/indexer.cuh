@@ -11,32 +11,35 @@
 // Data path: HBM-bound streaming of 68 B per cached token. One CTA per SM
 // owns a contiguous run of "units" (up to eight consecutive pages of one
 // sequence, 512 tokens) and runs a warp-specialised pipeline:
-//   producer (1 warp)   resolves 32 units at a time (one coalesced
-//        page-table load per lane) and each lane with a unit copies its pages
-//        (4 KB key pages + 256 B scale rows, cp.async.bulk without multicast,
-//        L2 evict-first) into the next of S ring slots once that slot is
-//        free; the slot's "full" mbarrier completes with the bytes.
+//   producer (1 warp)   resolves 32 units at a time, one batch ahead (one
+//        coalesced page-table load per lane; the first batch before the
+//        wait on the previous kernel, since the page table is an input),
+//        and each lane with a unit copies its pages (4 KB key pages + 256 B
+//        scale rows, cp.async.bulk without multicast, L2 evict-first) into
+//        the next of S ring slots once that slot is free; the slot's "full"
+//        mbarrier completes with the bytes.
 //   MMA (2 warps)       units alternate between two issuing threads (the
 //        per-unit waits and the commit, not the tensor core, bound one
-//        thread); each issues, per unit, eight tcgen05.mma
-//        kind::f8f6f4 (E4M3 x E4M3 -> fp32; four 128-token blocks x two
-//        32-channel steps, N = 16 query columns) from the slot straight into
-//        one of 4 TMEM accumulators, and one commit (a commit costs several
-//        MMAs' worth of issue time, so units are sized to amortise it). The key pages are stored as 8 x 16-byte core
-//        matrices (byte (t, c) at (t/8)*512 + (c/16)*128 + (t%8)*16 + c%16),
-//        which is the tensor core's no-swizzle K-major operand layout, so
-//        they are used as copied. The query (column n = query token * 4 +
-//        head) is written once per sequence into the same layout.
+//        thread); each issues, per unit, eight tcgen05.mma kind::f8f6f4
+//        (E4M3 x E4M3 -> fp32; four 128-token blocks x two 32-channel steps,
+//        N = 16 query columns) from the slot straight into one of 4 TMEM
+//        accumulators, and one commit (a commit costs several MMAs' worth
+//        of issue time, so units are sized to amortise it). The key pages
+//        are stored as 8 x 16-byte core matrices (byte (t, c) at
+//        (t/8)*512 + (c/16)*128 + (t%8)*16 + c%16), the tensor core's
+//        no-swizzle K-major operand layout, so they are used as copied. The
+//        query (column n = query token * 4 + head) is written once per
+//        sequence into the same layout.
 //   epilogue (16 warps) 4 groups of 4 warps take the units in turn; warp q
 //        of a group reads TMEM lanes 32q .. 32q+31 of every block (one token
-//        per thread and block, all heads), applies sigma, ReLU and the head weights, stores the
-//        scores (128-byte coalesced, L2 evict-last: the selection re-reads
-//        them) and adds each valid score's top 11 key bits to a shared-memory
-//        histogram per query row (rows past the shared slots go straight to
-//        the global histogram).
-// Every wait is a bounded mbarrier wait; a timeout sets the status word,
-// stops the pipeline and the producer waits (bounded) for its copies before
-// the CTA exits.
+//        per thread and block, all heads), applies sigma, ReLU and the head
+//        weights, stores the scores (128-byte coalesced, L2 evict-last: the
+//        selection re-reads them) and adds each valid score's top 11 key
+//        bits to a shared-memory histogram per query row (rows past the
+//        shared slots go straight to the global histogram).
+// Every wait is a bounded mbarrier wait that sleeps between probes; a
+// timeout sets the status word, stops the pipeline and the producer waits
+// (bounded) for its copies before the CTA exits.
 #pragma once
 
 #include "common.cuh"
