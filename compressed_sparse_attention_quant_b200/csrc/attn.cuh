@@ -9,21 +9,29 @@
 // One CTA (8 warps, two CTAs per SM) per (query token, split of its key
 // list). The key list is the k selected positions followed by the 128 window
 // rows; a split owns a run of at most 12 tiles of 64 keys.
-//   set-up   the split's selected positions are resolved once to physical
-//            cache slots (top-k index -> page table) in a shared table;
-//   prefetch right after a tile is dequantized, cp.async (16-byte and 4-byte
-//            LDGSTS, zero-filled for empty slots) fetches the next tile's
-//            packed FP4 records and scales, overlapping the tile's math;
-//   dequant  4 threads per key: hardware E2M1x2 -> f16x2 and E4M3x2 -> f16x2
-//            conversion and one exact f16 multiply into a [64][576] f16 tile
-//            whose 16-byte chunks are XOR-swizzled by key (conflict-free
-//            ldmatrix); window rows: bf16 loads rounded to f16;
-//   QK       warp (32-key group, 144-channel quarter): 4 n-tiles x 9 k-steps of
-//            m16n8k16 f16 MMA with the query fragments resident in registers;
-//            the quarters are summed through shared memory;
+//   set-up   the query row is read with 16-byte loads, rounded to f16 and
+//            stored in shared memory in the QK operand order (qk_pos), from
+//            where each warp takes its fragments with ldmatrix; the split's
+//            selected positions are resolved once to physical cache slots
+//            (top-k index -> page table) in a shared table;
+//   prefetch cp.async (16-byte and 4-byte LDGSTS, zero-filled for empty
+//            slots) fetches the next tile's packed FP4 records and scales as
+//            soon as the current tile's QK has consumed them, overlapping the
+//            softmax and PV;
+//   QK       warp (32-key group, 144-channel quarter): each lane converts the
+//            FP4 bytes of its key (hardware E2M1x2 -> f16x2, E4M3 -> f16 and
+//            one exact f16 multiply) directly into m16n8k16 B fragments, and
+//            stores the same f16 values into a [64][576] tile whose 16-byte
+//            chunks are XOR-swizzled by key; the query fragments stay in
+//            registers; the quarters are summed through shared memory. Tiles
+//            holding window rows (bf16 loads rounded to f16), padding, or the
+//            end of the selected list are first written to the f16 tile by
+//            all threads, and QK reads its fragments from there;
 //   softmax  two heads per warp, warp-shuffle max / sum in the exp2 domain,
-//            probabilities rounded to f16 (the same values feed the sum);
-//   PV       warp w owns 72 output channels; ldmatrix.trans of the same tile
+//            probabilities rounded to f16 (the same values feed the sum) and
+//            written over partial rows that no other warp reads, so three
+//            CTA barriers per tile remain (data in, QK done, P ready);
+//   PV       warp w owns 72 output channels; ldmatrix.trans of the f16 tile
 //            is the value operand.
 // Warp-level mma.sync is used deliberately: with 16 heads the MMA N extent is
 // 16, and at that width the warp MMAs issue faster than tcgen05 single-thread
@@ -37,7 +45,6 @@ namespace csa2 {
 constexpr int kAttThreads = 256;
 constexpr int kAttTile = 64;
 constexpr int kKhRow = kDim * 2;            // 1152 bytes per f16 key row (no padding: swizzled chunks)
-constexpr int kPPitch = kAttTile + 8;       // halfs per probability row
 constexpr int kMaxTilesPerSplit = 12;
 
 struct AttSmem {
@@ -91,11 +98,91 @@ __device__ __forceinline__ uint32_t kh_off(int key, int chunk) {
 // half-warp's float2 fragment stores touch land in four different bank groups.
 __device__ __forceinline__ int red_col(int head, int col) { return col ^ ((head & 3) << 3); }
 
+// f16 probabilities of head h for the tile's 64 keys: the 128 bytes of
+// red[0][h] (a row only the softmax warp of head h reads), with 16-byte chunks
+// XOR-swizzled by the head so the 8 rows an ldmatrix reads hit 8 bank groups.
+__device__ __forceinline__ uint8_t *p_row(AttSmem &sm, int h) {
+    return reinterpret_cast<uint8_t *>(&sm.red[0][h][0]);
+}
+__device__ __forceinline__ int p_off(int h, int key) { return (((key >> 3) ^ (h & 7)) << 4) + (key & 7) * 2; }
+
+// Position, in the operand order of the QK phase, of the physical channel
+// pair (c, c + 1), c even. Warp quarter cq of the QK phase owns channels
+// [144 cq, 144 cq + 144): two 64-channel units in which lane quad tig holds
+// channels 16 tig .. 16 tig + 15 of its key (one scale group, four k-steps),
+// then a 16-channel tail in which lane quad tig holds channels 4 tig .. 4 tig + 3.
+// k-step s of a unit puts channels 16 tig + 4 s + {0, 1} on MMA rows
+// k = 2 tig + {0, 1} and 16 tig + 4 s + {2, 3} on rows 2 tig + 8 + {0, 1}.
+// The query is stored in the same order, so every product q_c k_c is still
+// summed exactly once.
+__device__ __forceinline__ int qk_pos(int c) {
+    const int cq = c / 144, r = c - cq * 144;
+    const int ks = r < 128 ? (r >> 6) * 4 + ((r >> 2) & 3) : 8;
+    const int tig = r < 128 ? (r >> 4) & 3 : (r - 128) >> 2;
+    const int y = r & 3;
+    return cq * 144 + ks * 16 + 2 * tig + (y & 1) + ((y >> 1) << 3);
+}
+
+// QK over one warp's 32 keys x 144-channel quarter, in the operand order of
+// qk_pos. kFused: every key of the tile is a selected cache entry; the lane
+// converts its FP4 bytes straight into B fragments and also writes them to
+// the f16 tile for PV. Otherwise every key row is already in the f16 tile.
+template <bool kFused>
+__device__ __forceinline__ void qk_quarter(AttSmem &sm, const uint32_t (&qa)[9][4], float (&acc)[4][4], int kg,
+                                           int cq, int g, int tig) {
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        const int key = kg * 32 + nt * 8 + g;
+        const uint8_t *rrow = sm.raw[key];
+        const uint8_t *srow = sm.rsc[key];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int cb = cq * 144 + u * 64 + tig * 16;            // physical channel of h[0]
+            uint4 *d0 = reinterpret_cast<uint4 *>(sm.kh + kh_off(key, cb >> 3));
+            uint4 *d1 = reinterpret_cast<uint4 *>(sm.kh + kh_off(key, (cb >> 3) + 1));
+            uint32_t h[8];
+            if (kFused) {
+                const uint2 rv = *reinterpret_cast<const uint2 *>(rrow + (cb >> 1));
+                const uint32_t s2 = e4m3x2_to_f16x2(static_cast<uint32_t>(srow[cb >> 4]) * 0x0101u);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    h[i] = hmul2_u32(e2m1x2_to_f16x2(((i < 4 ? rv.x : rv.y) >> (8 * (i & 3))) & 0xffu), s2);
+                *d0 = make_uint4(h[0], h[1], h[2], h[3]);
+                *d1 = make_uint4(h[4], h[5], h[6], h[7]);
+            } else {
+                const uint4 a = *d0, b = *d1;
+                h[0] = a.x; h[1] = a.y; h[2] = a.z; h[3] = a.w;
+                h[4] = b.x; h[5] = b.y; h[6] = b.z; h[7] = b.w;
+            }
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_f16_16816(acc[nt], qa[4 * u + s][0], qa[4 * u + s][1], qa[4 * u + s][2], qa[4 * u + s][3],
+                              h[2 * s], h[2 * s + 1]);
+        }
+        {
+            const int cb = cq * 144 + 128 + tig * 4;
+            uint2 *d = reinterpret_cast<uint2 *>(sm.kh + kh_off(key, cb >> 3) + (cb & 7) * 2);
+            uint32_t h0, h1;
+            if (kFused) {
+                const uint32_t rv = *reinterpret_cast<const unsigned short *>(rrow + (cb >> 1));
+                const uint32_t s2 = e4m3x2_to_f16x2(static_cast<uint32_t>(srow[cb >> 4]) * 0x0101u);
+                h0 = hmul2_u32(e2m1x2_to_f16x2(rv & 0xffu), s2);
+                h1 = hmul2_u32(e2m1x2_to_f16x2(rv >> 8), s2);
+                *d = make_uint2(h0, h1);
+            } else {
+                const uint2 v = *d;
+                h0 = v.x;
+                h1 = v.y;
+            }
+            mma_f16_16816(acc[nt], qa[8][0], qa[8][1], qa[8][2], qa[8][3], h0, h1);
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kAttThreads, 2)
 sparse_attn_kernel(const AttParams P) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     AttSmem &sm = *reinterpret_cast<AttSmem *>(smem_raw);
-    __half (*pmat)[kPPitch] = reinterpret_cast<__half (*)[kPPitch]>(&sm.red[0][0][0]);   // P overlays red
     const int row = blockIdx.y;
     const int split = blockIdx.x;
     const int b = row / P.Sq, j = row % P.Sq;
@@ -104,21 +191,29 @@ sparse_attn_kernel(const AttParams P) {
     const int n_rows_swa = kWindow + P.Sq - 1;
 
     // Inputs that no earlier kernel of the step writes are read before the
-    // wait for the selection: the query fragments, the sequence length and
-    // (into L2) the sequence's page-table row.
-    // Query fragments for QK: warp (kg, cq) covers channels cq*144 .. +143.
+    // wait for the selection: the query, the sequence length and (into L2)
+    // the sequence's page-table row. The query goes through the (still free)
+    // f16 tile: 16-byte loads, f16 rounding, a scatter into the QK operand
+    // order, then one ldmatrix per k-step. Warp (kg, cq) covers channels
+    // cq*144 .. +143.
     const int kg = warp >> 2, cq = warp & 3;
     uint32_t qa[9][4];
     {
-        const __nv_bfloat16 *qrow = P.q + static_cast<int64_t>(row) * kHeads * kDim;
+        const uint4 *qg = reinterpret_cast<const uint4 *>(P.q + static_cast<int64_t>(row) * kHeads * kDim);
+        for (int i = tid; i < kHeads * kDim / 8; i += kAttThreads) {
+            const int h = i / (kDim / 8), c = (i - h * (kDim / 8)) * 8;
+            const uint4 v = __ldg(qg + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int ks = 0; ks < 9; ++ks) {
-            const int cb = cq * 144 + ks * 16 + tig * 2;
-            qa[ks][0] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + g * kDim + cb));
-            qa[ks][1] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + (g + 8) * kDim + cb));
-            qa[ks][2] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + g * kDim + cb + 8));
-            qa[ks][3] = bf16x2_to_f16x2(*reinterpret_cast<const uint32_t *>(qrow + (g + 8) * kDim + cb + 8));
+            for (int p = 0; p < 4; ++p) {
+                const int L = qk_pos(c + 2 * p);
+                *reinterpret_cast<uint32_t *>(sm.kh + kh_off(h, L >> 3) + (L & 7) * 2) = bf16x2_to_f16x2(w[p]);
+            }
         }
+        __syncthreads();
+#pragma unroll
+        for (int ks = 0; ks < 9; ++ks)
+            ldsm_x4(qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], sm.kh + kh_off(lane & 15, 18 * cq + 2 * ks + (lane >> 4)));
     }
     int T = P.seq_lens[b];
     for (int i = tid * 32; i < P.max_pages; i += kAttThreads * 32)           // 128-byte lines of the row
@@ -198,8 +293,12 @@ sparse_attn_kernel(const AttParams P) {
         const int it = tile - tile0;
         cp_async_wait<0>();                              // this tile's raw records have landed
         __syncthreads();
-        // ---------------- dequantize one tile of 64 keys into f16
-        {
+        // Every key of the tile is a selected cache entry: QK converts the FP4
+        // records itself. Otherwise all threads first write the tile's key
+        // rows (FP4 -> f16, window bf16 -> f16, or zeros) to the f16 tile.
+        const bool fused = (tile + 1) * kAttTile <= P.k;
+        if (fused && gpart == 0) sm.valid[gkey] = sm.slot[it * kAttTile + gkey] >= 0 ? 1 : 0;
+        if (!fused) {
             const int slot = tile * kAttTile + gkey;
             uint8_t *kh = sm.kh;
             bool valid = false;
@@ -254,16 +353,16 @@ sparse_attn_kernel(const AttParams P) {
                     // Thread p of a key takes chunks 8m + 2p + {0,1}: the
                     // chunks of a store phase share their parity per key.
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        uint4 rv[9];
+                    for (int third = 0; third < 3; ++third) {
+                        uint4 rv[6];
 #pragma unroll
-                        for (int i = 0; i < 9; ++i) {
-                            const int e = half * 9 + i;
+                        for (int i = 0; i < 6; ++i) {
+                            const int e = third * 6 + i;
                             rv[i] = __ldg(src + 8 * (e >> 1) + 2 * gpart + (e & 1));
                         }
 #pragma unroll
-                        for (int i = 0; i < 9; ++i) {
-                            const int e = half * 9 + i;
+                        for (int i = 0; i < 6; ++i) {
+                            const int e = third * 6 + i;
                             uint4 h;
                             h.x = bf16x2_to_f16x2(rv[i].x);
                             h.y = bf16x2_to_f16x2(rv[i].y);
@@ -280,28 +379,15 @@ sparse_attn_kernel(const AttParams P) {
             }
             if (gpart == 0) sm.valid[gkey] = valid ? 1 : 0;
         }
-        __syncthreads();
-        if (tile + 1 < tile1) prefetch(tile + 1);        // overlaps this tile's math
-        cp_async_commit();
+        if (!fused) __syncthreads();
 
         // ---------------- S = Q K^T over this warp's 32 keys x channel quarter
         {
             float acc[4][4];
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
-            const int m = lane >> 3, r = lane & 7;
-#pragma unroll
-            for (int ks = 0; ks < 9; ++ks) {
-                const int cb = cq * 144 + ks * 16;
-#pragma unroll
-                for (int pr = 0; pr < 2; ++pr) {
-                    const int key = kg * 32 + (2 * pr + (m >> 1)) * 8 + r;
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(b0, b1, b2, b3, sm.kh + kh_off(key, (cb >> 3) + (m & 1)));
-                    mma_f16_16816(acc[2 * pr], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
-                    mma_f16_16816(acc[2 * pr + 1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
-                }
-            }
+            if (fused) qk_quarter<true>(sm, qa, acc, kg, cq, g, tig);
+            else qk_quarter<false>(sm, qa, acc, kg, cq, g, tig);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
                 const int col = nt * 8 + tig * 2;
@@ -310,7 +396,9 @@ sparse_attn_kernel(const AttParams P) {
                     make_float2(acc[nt][2], acc[nt][3]);
             }
         }
-        __syncthreads();
+        __syncthreads();                                 // partials and the f16 tile are complete; raw is free
+        if (tile + 1 < tile1) prefetch(tile + 1);        // overlaps this tile's softmax and PV
+        cp_async_commit();
 
         // ---------------- online softmax, two heads per warp
         {
@@ -347,12 +435,16 @@ sparse_attn_kernel(const AttParams P) {
                 for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
                 psum[hh] = sum;
             }
-            __syncthreads();                                  // every warp is done reading red (P overlays it)
+            // Row h of every partial block is read by this warp alone, so the
+            // probabilities of head h go into the 128 bytes of red[0][h]
+            // without a CTA barrier (the warp's own reads are complete: the
+            // shuffles above consumed them).
+            __syncwarp();
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int h = warp * 2 + hh;
-                pmat[h][lane] = __float2half_rn(pv[hh][0]);
-                pmat[h][lane + 32] = __float2half_rn(pv[hh][1]);
+                *reinterpret_cast<__half *>(p_row(sm, h) + p_off(h, lane)) = __float2half_rn(pv[hh][0]);
+                *reinterpret_cast<__half *>(p_row(sm, h) + p_off(h, lane + 32)) = __float2half_rn(pv[hh][1]);
                 if (lane == 0) {
                     sm.l_run[h] = sm.l_run[h] * alpha[hh] + psum[hh];
                     sm.m_run[h] = m_new[hh];
@@ -377,7 +469,7 @@ sparse_attn_kernel(const AttParams P) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 uint32_t a0, a1, a2, a3;
-                ldsm_x4(a0, a1, a2, a3, &pmat[r + 8 * (m & 1)][kk * 16 + 8 * (m >> 1)]);
+                ldsm_x4(a0, a1, a2, a3, p_row(sm, r + 8 * (m & 1)) + p_off(r + 8 * (m & 1), kk * 16 + 8 * (m >> 1)));
                 const int key = kk * 16 + 8 * (m & 1) + r;
 #pragma unroll
                 for (int pr = 0; pr < 4; ++pr) {
