@@ -37,6 +37,11 @@ METRIC = "decode tokens/s and achieved HBM GB/s (% of 8 TB/s) for CSA2 FP4 spars
 KERNEL_SOURCES = ("csrc/common.cuh", "csrc/indexer.cuh", "csrc/topk.cuh")
 
 
+# Algorithmic bytes of one row of the indexer FP8 quantiser: 64 bf16 in,
+# 64 E4M3 codes + one fp32 scale out.
+Q8_BYTES_PER_ROW = 64 * 2 + 64 + 4
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -381,7 +386,31 @@ def run_gpu(args, wl):
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / args.steps
 
-    step_ms, idx_ms, e2e_ms = replicas.max_over_ranks([step_ms, idx_ms, e2e_ms], dist, dev)
+    # The indexer FP8 quantiser (csa2_quant_indexer_fp8) over the keys of the
+    # whole cache: B x T rows of 64 bf16 channels (seeded N(0, 1), generated
+    # on the device), far larger than L2, so no flush. Events around each
+    # launch on its stream.
+    q8_rows = wl.batch * wl.context
+    q8_gen = torch.Generator(device=dev).manual_seed(1000 + rank)
+    q8_x = torch.randn(q8_rows, lib.IDX_DIM, generator=q8_gen, device=dev, dtype=torch.bfloat16)
+    q8_codes = torch.empty(q8_rows, lib.IDX_DIM, dtype=torch.uint8, device=dev)
+    q8_sigma = torch.empty(q8_rows, dtype=torch.float32, device=dev)
+    for _ in range(2):
+        lib.quant_indexer_fp8(q8_x, q8_codes, q8_sigma)
+    torch.cuda.synchronize(dev)
+    q8_events = []
+    for _ in range(args.steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        lib.quant_indexer_fp8(q8_x, q8_codes, q8_sigma)
+        e1.record(stream)
+        q8_events.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    q8_ms = sum(a.elapsed_time(b) for a, b in q8_events) / args.steps
+    del q8_x, q8_codes, q8_sigma
+
+    step_ms, idx_ms, e2e_ms, q8_ms = replicas.max_over_ranks([step_ms, idx_ms, e2e_ms, q8_ms], dist, dev)
 
     tokens_per_rank = wl.batch * wl.q_tokens
     value = replicas.job_throughput(tokens_per_rank, world, step_ms)
@@ -410,6 +439,12 @@ def run_gpu(args, wl):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "device_status": lib.status_string(status),
+        "indexer_fp8_quant": {"kernel": "csa2_quant_indexer_fp8", "rows": q8_rows,
+                              "bytes_per_row": Q8_BYTES_PER_ROW, "ms_per_launch": q8_ms,
+                              "achieved": q8_rows * Q8_BYTES_PER_ROW / (q8_ms * 1e-3) / 1e9, "peak": hbm,
+                              "unit": "GB/s",
+                              "frac": q8_rows * Q8_BYTES_PER_ROW / (q8_ms * 1e-3) / 1e9 / hbm,
+                              "input": "B x T rows of 64 bf16 channels, N(0,1) seeded, > L2"},
     }
     clocks = clk.summary()
     if clocks:

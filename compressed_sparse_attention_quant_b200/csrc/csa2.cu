@@ -184,6 +184,20 @@ csa2_status csa2_quant_kv_fp4(const void *x_bf16, int64_t n_tok, int dim, const 
                                            static_cast<cudaStream_t>(stream)));
 }
 
+csa2_status csa2_quant_indexer_fp8(const void *x_bf16, int64_t n_rows, int dim, void *codes_e4m3, float *sigma,
+                                   void *stream) {
+    if (n_rows < 0) return CSA2_ERR_INVALID_ARG;
+    if (dim != kIdxDim) return CSA2_ERR_UNSUPPORTED;
+    if (n_rows == 0) return CSA2_OK;
+    if (!x_bf16 || !codes_e4m3 || !sigma) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(x_bf16, 16) || !aligned(codes_e4m3, 16) || !aligned(sigma, 4)) return CSA2_ERR_ALIGNMENT;
+    if (n_rows > (INT64_C(1) << 40)) return CSA2_ERR_INVALID_ARG;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return CSA2_ERR_CUDA;
+    return cuda_status(launch_quant_index_fp8(x_bf16, n_rows, codes_e4m3, sigma, dev->sm_count,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 size_t csa2_indexer_topk_workspace_bytes(int B, int Sq, int max_pages, int k) {
     if (B <= 0 || Sq <= 0 || max_pages <= 0 || k <= 0) return 0;
     return idx_layout(B, Sq, max_pages, k).total;

@@ -24,7 +24,7 @@ STATUS = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_UNSUPPORTED", 3:
           7: "CSA2_ERR_WORKSPACE", 8: "CSA2_ERR_ALIGNMENT"}
 
 # Every function include/csa2.h declares (checked by the CPU test suite).
-EXPORTS = ("csa2_quant_kv_fp4", "csa2_indexer_topk_workspace_bytes", "csa2_indexer_topk",
+EXPORTS = ("csa2_quant_kv_fp4", "csa2_quant_indexer_fp8", "csa2_indexer_topk_workspace_bytes", "csa2_indexer_topk",
            "csa2_sparse_attn_workspace_bytes", "csa2_sparse_attn_decode",
            "csa2_sparse_attn_decode_noalloc", "csa2_plan",
            "csa2_last_device_error", "csa2_status_string", "csa2_launch_count")
@@ -53,6 +53,7 @@ def _load():
     L = ctypes.CDLL(path)
     sig = {
         "csa2_quant_kv_fp4": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp, _cp, _vp]),
+        "csa2_quant_indexer_fp8": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp]),
         "csa2_indexer_topk_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
         "csa2_indexer_topk": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _cp, _vp, _i32, _vp, _i32, _vp,
                                      _vp, _sz, _vp]),
@@ -140,6 +141,27 @@ def quant_kv_fp4(x: torch.Tensor, slots: torch.Tensor, cache: PagedCache,
     rc = _L.csa2_quant_kv_fp4(_ptr(x), n, DIM, _ptr(slots), _ptr(kidx_in), _ptr(kidx_scale_in),
                               ctypes.byref(cache.desc), _stream())
     _check("csa2_quant_kv_fp4", rc)
+
+
+def quant_indexer_fp8(x: torch.Tensor, codes: Optional[torch.Tensor] = None,
+                      sigma: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """bf16 rows of 64 channels -> (E4M3FN codes uint8 [..., 64], sigma f32 [...])."""
+    if x.shape[-1] != IDX_DIM:
+        raise ValueError(f"x: last dimension must be {IDX_DIM}, got {tuple(x.shape)}")
+    lead = tuple(x.shape[:-1])
+    n = 1
+    for d in lead:
+        n *= int(d)
+    _req(x, torch.bfloat16, "x")
+    if codes is None:
+        codes = torch.empty(*lead, IDX_DIM, dtype=torch.uint8, device=x.device)
+    if sigma is None:
+        sigma = torch.empty(*lead, dtype=torch.float32, device=x.device)
+    _req(codes, torch.uint8, "codes", lead + (IDX_DIM,))
+    _req(sigma, torch.float32, "sigma", lead)
+    rc = _L.csa2_quant_indexer_fp8(_ptr(x), n, IDX_DIM, _ptr(codes), _ptr(sigma), _stream())
+    _check("csa2_quant_indexer_fp8", rc)
+    return codes, sigma
 
 
 def indexer_topk_workspace_bytes(B: int, Sq: int, max_pages: int, k: int) -> int:

@@ -131,6 +131,30 @@ csa2_status csa2_quant_kv_fp4(const void *x_bf16, int64_t n_tok, int dim,
                               const csa2_paged_cache *cache, void *stream);
 
 /*
+ * csa2_quant_indexer_fp8 -- indexer key / query quantiser ([ZUL section 3]:
+ * the KV owner hands "indexer K / scale" to its consumer layers; [NEO part 2]:
+ * the indexer scores with FP8 operands).
+ *
+ * For each of n_rows rows of 64 bf16 channels:
+ *     sigma[r]    = amax_r / 448                 (IEEE binary32 division)
+ *     codes[r][c] = E4M3FN(x[r][c] / sigma[r])   (binary32 division, then round
+ *                   to nearest even, saturating at +-448, canonical +0)
+ * An all-zero row gives sigma = 0 and zero codes. Inputs must be finite. The
+ * pages print no scale rule; this is the plainest one (the row maximum lands
+ * on the top E4M3 value). Keys: codes and sigma are the kidx_in and
+ * kidx_scale_in of csa2_quant_kv_fp4. Queries: one row per (token, indexer
+ * head); since sigma > 0 can be taken out of the ReLU, the head weight passed
+ * to csa2_indexer_topk becomes w * sigma.
+ *
+ *   x_bf16      device bf16 [n_rows][dim], 16-byte aligned; dim must be 64
+ *   codes_e4m3  device uint8 [n_rows][64], 16-byte aligned
+ *   sigma       device float [n_rows], 4-byte aligned
+ * HBM-bound: 128 B read and 68 B written per row.
+ */
+csa2_status csa2_quant_indexer_fp8(const void *x_bf16, int64_t n_rows, int dim,
+                                   void *codes_e4m3, float *sigma, void *stream);
+
+/*
  * csa2_indexer_topk -- Full / Reindex: score every cached token with the
  * lightweight indexer and select the top-k ([NEO part 2] "Top-K sparse
  * addressing index"; [ZUL section 3]: Full and Reindex compute the index).

@@ -56,6 +56,10 @@ def lib():
         L.orc_quant_fp4.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int, _u8p, _u8p]
         L.orc_dequant_fp4.restype = None
         L.orc_dequant_fp4.argtypes = [_u8p, _u8p, ctypes.c_int64, ctypes.c_int, _f64p]
+        L.orc_e4m3_code.restype = ctypes.c_uint8
+        L.orc_e4m3_code.argtypes = [ctypes.c_float]
+        L.orc_quant_index_fp8.restype = None
+        L.orc_quant_index_fp8.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int, _u8p, _f32p]
         L.orc_indexer_scores.restype = None
         L.orc_indexer_scores.argtypes = [_u8p, _f32p, ctypes.c_int, ctypes.c_int, _u8p, _f32p,
                                          ctypes.c_int64, ctypes.c_int, _f64p]
@@ -136,6 +140,22 @@ def dequant_fp4(codes, scales) -> np.ndarray:
     out = np.zeros((n, dim), np.float64)
     lib().orc_dequant_fp4(_p(codes, _u8p), _p(scales, _u8p), n, dim, _p(out, _f64p))
     return out
+
+
+# ---------------------------------------------------------------- indexer FP8 quantiser
+def e4m3_code(r: float) -> int:
+    """E4M3FN code of the binary32 value nearest r (the argument is passed as a C float)."""
+    return int(lib().orc_e4m3_code(float(r)))
+
+
+def quant_index_fp8(x_bf16_bits) -> Tuple[np.ndarray, np.ndarray]:
+    """x: uint16 bf16 bits [n, dim] -> (codes uint8 [n, dim] E4M3FN, sigma f32 [n])."""
+    x = _c(x_bf16_bits, np.uint16)
+    n, dim = x.shape
+    codes = np.zeros((n, dim), np.uint8)
+    sigma = np.zeros(n, np.float32)
+    lib().orc_quant_index_fp8(_p(x, _u16p), n, dim, _p(codes, _u8p), _p(sigma, _f32p))
+    return codes, sigma
 
 
 # ---------------------------------------------------------------- indexer

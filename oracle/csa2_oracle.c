@@ -212,6 +212,79 @@ void orc_dequant_fp4(const uint8_t *codes, const uint8_t *scales, int64_t n,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Indexer FP8 quantiser                                                     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * E4M3FN code of a binary32 value r, round to nearest with ties to the even
+ * mantissa, saturating at +-448, canonical +0 when the magnitude rounds to 0.
+ * Method as in orc_group_scale: the grid step in the binade [2^E, 2^(E+1))
+ * is 2^(E-3) for E >= -6, and the subnormal step 2^-9 continues below 2^-6.
+ * r is a binary32 value, exact in fp64, so r / step is exact and nearbyint
+ * performs the one rounding.
+ */
+uint8_t orc_e4m3_code(float r)
+{
+    double a = fabs((double)r);
+    double mag;
+    if (a >= 448.0) {
+        mag = 448.0;
+    } else if (a == 0.0) {
+        mag = 0.0;
+    } else {
+        int e;
+        frexp(a, &e);
+        int E = e - 1;
+        if (E < -6)
+            E = -6;
+        double step = ldexp(1.0, E - 3);
+        mag = nearbyint(a / step) * step;   /* may carry to 2^(E+1): still on the grid */
+        if (mag > 448.0)
+            mag = 448.0;
+    }
+    if (mag == 0.0)
+        return 0;
+    uint8_t code = e4m3_encode_exact(mag);
+    return (r < 0.0f) ? (uint8_t)(code | 0x80) : code;
+}
+
+/*
+ * Indexer key / query quantiser. [ZUL section 3] lists "indexer K / scale"
+ * among the state a KV owner hands to its consumer layers, and [NEO part 2]
+ * has the indexer read FP8 operands; the pages give no rule for the scale.
+ * Reading: one binary32 scale per row of `dim` channels,
+ *     sigma = amax / 448   (binary32 division; 0 for an all-zero row),
+ * and code_c = E4M3FN nearest to x_c / sigma (binary32 division, then one
+ * round to nearest even, saturating; all codes 0 when sigma = 0). Both
+ * divisions are binary32 so that a kernel dividing in fp32 takes the same
+ * integer decisions; the dequantised value is sigma * e4m3(code).
+ */
+void orc_quant_index_fp8(const uint16_t *x_bf16, int64_t n_rows, int dim,
+                         uint8_t *codes, float *sigma)
+{
+    for (int64_t t = 0; t < n_rows; ++t) {
+        const uint16_t *row = x_bf16 + t * dim;
+        double amax = 0.0;
+        for (int c = 0; c < dim; ++c) {
+            double v = fabs(orc_bf16_value(row[c]));
+            if (v > amax)
+                amax = v;
+        }
+        float sg = (float)amax / 448.0f;      /* amax is a bf16 value: exact in binary32 */
+        sigma[t] = sg;
+        for (int c = 0; c < dim; ++c) {
+            if (sg == 0.0f) {
+                codes[t * dim + c] = 0;
+                continue;
+            }
+            float x = (float)orc_bf16_value(row[c]);
+            float r = x / sg;
+            codes[t * dim + c] = orc_e4m3_code(r);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Indexer                                                                   */
 /* ------------------------------------------------------------------------ */
 

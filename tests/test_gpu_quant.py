@@ -126,3 +126,69 @@ def test_quant_out_of_range_slot_sets_device_status(lib):
     assert lib.last_device_error() == 6            # CSA2_ERR_DEVICE_BOUNDS
     assert lib.last_device_error() == 0            # cleared by the read
     assert torch.any(cache.kv_scale.view(-1, 36)[0] != 0)
+
+
+# ------------------------------------------------------------------ K1b: indexer FP8 quantiser
+def _index_rows(rng, n):
+    """Wide-magnitude rows plus the rows where a rounding decision is close:
+    zero rows, bf16 subnormals, near the bf16 maximum, E4M3 midpoints (ties)
+    and their bf16 neighbours under sigma = 1."""
+    x = rng.standard_normal((n, 64)) * np.exp2(rng.integers(-60, 60, (n, 1)))
+    x[0] = 0.0
+    x[1] = -0.0
+    x[2] = rng.standard_normal(64) * 1e-39
+    x[3, :] = 3.3e38
+    x[3, 1::2] *= -1
+    x[4] = 0.0
+    x[4, 63] = -2.0e-38
+    ev = torch.arange(127, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mids = (ev[:-1] + ev[1:]) / 2
+    rows = []
+    for k in range(0, len(mids), 63):
+        r = np.zeros(64)
+        r[0] = 448.0
+        m = mids[k:k + 63]
+        r[1:1 + len(m)] = m * np.where(np.arange(len(m)) % 2 == 0, 1, -1)
+        rows.append(r)
+    x[5:5 + len(rows)] = np.array(rows)
+    bits = oracle.bf16_bits(torch.from_numpy(x).to(torch.bfloat16))
+    # bf16 neighbours of the midpoint rows (one ulp up and down, same row maximum)
+    nb = bits[5:5 + len(rows)].copy()
+    up, down = nb.copy(), nb.copy()
+    up[:, 1:] += (nb[:, 1:] & 0x7FFF) != 0
+    down[:, 1:] -= (nb[:, 1:] & 0x7FFF) != 0
+    return np.concatenate([bits, up, down])
+
+
+@pytest.mark.parametrize("n", [1, 37, 75813])
+def test_quant_indexer_fp8_bit_exact(lib, n):
+    """Codes and sigma bit-exact against the oracle; 75813 rows run the
+    grid-stride loop twice per thread with a ragged tail."""
+    rng = np.random.default_rng(n)
+    bits = _index_rows(rng, max(n, 16))[:n] if n >= 16 else oracle.bf16_bits(
+        torch.from_numpy(rng.standard_normal((n, 64))).to(torch.bfloat16))
+    x = _bf16_from_bits(bits).cuda()
+    codes, sigma = lib.quant_indexer_fp8(x)
+    assert lib.last_device_error() == 0
+    rc, rs = oracle.quant_index_fp8(bits)
+    np.testing.assert_array_equal(codes.cpu().numpy(), rc)
+    np.testing.assert_array_equal(sigma.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+
+
+def test_quant_indexer_fp8_feeds_the_cache_and_indexer(lib):
+    """Quantised keys go through K1's indexer-key path unchanged, and an empty
+    call is a no-op."""
+    rng = np.random.default_rng(5)
+    bits = oracle.bf16_bits(torch.from_numpy(rng.standard_normal((200, 64))).to(torch.bfloat16))
+    kc, ks = lib.quant_indexer_fp8(_bf16_from_bits(bits).cuda())
+    cache = lib.PagedCache(4)
+    slots = torch.arange(200, dtype=torch.int32, device="cuda")
+    xkv = torch.zeros(200, 576, dtype=torch.bfloat16, device="cuda")
+    lib.quant_kv_fp4(xkv, slots, cache, kc, ks)
+    assert lib.last_device_error() == 0
+    got = cache.kidx_logical().reshape(-1, 64)[:200].cpu().numpy()
+    np.testing.assert_array_equal(got, kc.cpu().numpy())
+    np.testing.assert_array_equal(cache.kidx_scale.reshape(-1)[:200].cpu().numpy(), ks.cpu().numpy())
+    e = torch.empty(0, 64, dtype=torch.bfloat16, device="cuda")
+    c0, s0 = lib.quant_indexer_fp8(e)
+    assert c0.shape == (0, 64) and s0.shape == (0,)

@@ -92,6 +92,13 @@ def test_unsupported_shapes_rejected_on_host(lib):
     assert L.csa2_quant_kv_fp4(16, -1, 576, 16, None, None, ctypes.byref(cache), None) == 1
     assert L.csa2_quant_kv_fp4(16, 4, 576, 16, None, None, None, None) == 1
     assert L.csa2_plan(None, 3, None, None) == 1
+    # indexer FP8 quantiser: 64 channels only; null / negative; 16-byte alignment; empty is a no-op
+    assert L.csa2_quant_indexer_fp8(16, 4, 128, 16, 16, None) == 2
+    assert L.csa2_quant_indexer_fp8(None, 4, 64, 16, 16, None) == 1
+    assert L.csa2_quant_indexer_fp8(16, -1, 64, 16, 16, None) == 1
+    assert L.csa2_quant_indexer_fp8(24, 4, 64, 16, 16, None) == 8
+    assert L.csa2_quant_indexer_fp8(16, 4, 64, 24, 16, None) == 8
+    assert L.csa2_quant_indexer_fp8(16, 0, 64, None, None, None) == 0
     assert lib.launch_count() == 0
 
 

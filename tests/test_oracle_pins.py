@@ -10,6 +10,14 @@ What pins each oracle function:
                   finite E4M3 scale: brute-force argmin of |x - s*m|
   quant_fp4       group/nibble layout against a composition written here from
                   the pinned pieces; error bound; idempotence; bytes per token
+  e4m3_code       torch's RNE float8_e4m3fn cast (library) and a brute-force
+                  nearest search over every finite bf16 value in range and
+                  every E4M3 midpoint with its binary32 neighbours;
+                  saturation; canonical +0
+  quant_index_fp8 sigma against numpy binary32 division (library); codes
+                  against brute force on wide-magnitude rows; idempotence on
+                  E4M3-grid rows; power-of-two equivariance; error bound;
+                  zero rows
   indexer_scores  one-hot head weights reduce to an integer matmul (numpy);
                   linearity in w; ReLU placement with negative sigma; q = 0.
                   The formula itself is a reading (parity unpinned).
@@ -106,6 +114,104 @@ def test_group_scale_matches_torch_rne_cast():
     t = torch.from_numpy(amax / 6.0).to(torch.float32)   # exact side argued in the oracle
     ref = t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     np.testing.assert_array_equal(oracle.group_scale_n(amax), ref)
+
+
+# ------------------------------------------------------------------ indexer FP8 quantiser
+def e4m3_nearest_bruteforce(r: np.ndarray) -> np.ndarray:
+    """Nearest finite E4M3FN byte to each binary32 value (fp64 distances are
+    exact here), ties to the even byte, saturating, canonical +0."""
+    ev = e4m3_finite_values()[:127]                  # 0x00 .. 0x7E, ascending
+    a = np.minimum(np.abs(r.astype(np.float64)), 448.0)
+    dist = np.abs(ev[None, :] - a[:, None])
+    best = dist.min(axis=1, keepdims=True)
+    cand = dist == best
+    even = cand & (np.arange(127) % 2 == 0)[None, :]
+    pick = np.where(even.any(axis=1), even.argmax(axis=1), cand.argmax(axis=1)).astype(np.uint8)
+    return np.where((r < 0) & (pick != 0), pick | 0x80, pick).astype(np.uint8)
+
+
+def test_e4m3_code_against_torch_cast_and_bruteforce():
+    _, vals = all_finite_bf16_bits()
+    ev = e4m3_finite_values()[:127]
+    mids = ((ev[:-1] + ev[1:]) / 2).astype(np.float32)          # exact: at most 5 significant bits
+    assert np.all(mids.astype(np.float64) == (ev[:-1] + ev[1:]) / 2)
+    up = np.nextafter(mids, np.float32(np.inf))
+    down = np.nextafter(mids, np.float32(0))
+    r = np.concatenate([vals[np.abs(vals) <= 448].astype(np.float32), mids, up, down, -mids, -up, -down])
+    got = np.array([oracle.e4m3_code(float(x)) for x in r], np.uint8)
+    ref = torch.from_numpy(r).to(torch.float8_e4m3fn).view(torch.uint8).numpy().copy()
+    ref[(ref & 0x7F) == 0] = 0                                    # canonical +0
+    np.testing.assert_array_equal(got, ref)
+    np.testing.assert_array_equal(got, e4m3_nearest_bruteforce(r))
+    # saturation above the largest finite value, both signs
+    for x in (448.5, 464.0, 1e6, 3.0e38):
+        assert oracle.e4m3_code(x) == 0x7E and oracle.e4m3_code(-x) == 0xFE
+
+
+def bf16_rows(x: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def test_quant_index_fp8_rows_against_bruteforce():
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((300, 64)) * np.exp2(rng.integers(-60, 60, (300, 1)))
+    x[0] = 0.0
+    x[1] = -0.0
+    x[2] = 0.0
+    x[2, 17] = -3.0e-38                                           # one tiny non-zero channel
+    x[3] = rng.standard_normal(64) * 1e-39                        # bf16 subnormals
+    x[4, :] = 3.3e38                                              # near the bf16 maximum
+    x[4, ::2] *= -1
+    bits = bf16_rows(x)
+    codes, sigma = oracle.quant_index_fp8(bits)
+    xv = bits_to_f32(bits)
+    amax = np.abs(xv).max(axis=1)
+    np.testing.assert_array_equal(sigma, amax / np.float32(448.0))          # numpy binary32 division
+    assert sigma[0] == 0 and sigma[1] == 0 and np.all(codes[:2] == 0)
+    nz = sigma > 0
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = (xv[nz] / sigma[nz, None]).astype(np.float32)
+    np.testing.assert_array_equal(codes[nz], e4m3_nearest_bruteforce(r.ravel()).reshape(r.shape))
+    # the largest magnitude of a row lands on 448 (up to the rounding of sigma)
+    top = np.abs(xv).argmax(axis=1)
+    assert np.all((codes[nz, top[nz]] & 0x7F) >= 0x7D)
+
+
+def test_quant_index_fp8_idempotent_on_grid_rows():
+    rng = np.random.default_rng(12)
+    ev = e4m3_finite_values()
+    b = rng.integers(0, 0x7F, (50, 64)).astype(np.uint8) | (rng.integers(0, 2, (50, 64)) * 0x80).astype(np.uint8)
+    b[:, 5] = 0x7E                                                # row maximum 448 -> sigma = 1
+    x = ev[b]
+    bits = bf16_rows(x)
+    assert np.all(bits_to_f32(bits).astype(np.float64) == x)    # E4M3 values are exact in bf16
+    codes, sigma = oracle.quant_index_fp8(bits)
+    assert np.all(sigma == 1.0)
+    want = np.where((b & 0x7F) == 0, 0, b).astype(np.uint8)
+    np.testing.assert_array_equal(codes, want)
+
+
+def test_quant_index_fp8_power_of_two_equivariance_and_error_bound():
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((100, 64)).astype(np.float32)
+    bits = bf16_rows(x)
+    codes, sigma = oracle.quant_index_fp8(bits)
+    xv = bits_to_f32(bits).astype(np.float64)
+    for k in (-40, -9, 9, 40):
+        c2, s2 = oracle.quant_index_fp8(bf16_rows(xv * 2.0 ** k))
+        np.testing.assert_array_equal(c2, codes)
+        np.testing.assert_array_equal(s2.astype(np.float64), sigma.astype(np.float64) * 2.0 ** k)
+    ev = e4m3_finite_values()
+    deq = np.where(codes >= 0x80, -ev[codes & 0x7F], ev[codes & 0x7F]) * sigma[:, None].astype(np.float64)
+    r = np.abs(xv) / sigma[:, None]
+    e = np.floor(np.log2(np.maximum(r, 2.0 ** -6)))
+    half_ulp = np.exp2(e - 4)                                     # half the E4M3 step at r (2^-10 below 2^-6)
+    bound = sigma[:, None] * (half_ulp + r * 2.0 ** -23)          # + the binary32 rounding of the quotient
+    assert np.all(np.abs(xv - deq) <= bound)
 
 
 # ------------------------------------------------------------------ codes
