@@ -65,6 +65,8 @@ def lib():
                                          ctypes.c_int64, ctypes.c_int, _f64p]
         L.orc_topk.restype = ctypes.c_int
         L.orc_topk.argtypes = [_f64p, ctypes.c_int64, ctypes.c_int, _i32p]
+        L.orc_pool_topk.restype = ctypes.c_int
+        L.orc_pool_topk.argtypes = [_f64p, _i32p, ctypes.c_int, ctypes.c_int, _i32p]
         L.orc_sparse_attn.restype = None
         L.orc_sparse_attn.argtypes = [_u16p, ctypes.c_int, ctypes.c_int, _u8p, _u8p,
                                       ctypes.c_int64, _i32p, ctypes.c_int, _u16p, ctypes.c_int,
@@ -180,6 +182,26 @@ def topk(scores, n_valid: int, k: int) -> np.ndarray:
     return out
 
 
+def pool_topk(scores, pool, k: int) -> np.ndarray:
+    """Top-k of a candidate pool: scores f64 [n], pool int32 token indices [n] (-1 skipped)."""
+    s = _c(scores, np.float64)
+    p = _c(pool, np.int32)
+    out = np.full(max(k, 0), -1, np.int32)
+    if k > 0:
+        lib().orc_pool_topk(_p(s, _f64p), _p(p, _i32p), len(p), int(k), _p(out, _i32p))
+    return out
+
+
+def pool_reindex(q, w, kidx, ksig, pool, k: int) -> np.ndarray:
+    """A Reindex layer under the hierarchical sparse indexer: score only the
+    pool's tokens (kidx uint8 [T, DI], ksig f32 [T] of the owner's cache) with
+    this layer's q, w, then take the pool top-k."""
+    pool = _c(pool, np.int32)
+    valid = pool[pool >= 0]
+    s = indexer_scores(q, w, kidx[valid], ksig[valid]) if len(valid) else np.zeros(0)
+    return pool_topk(s, valid, k)
+
+
 # ---------------------------------------------------------------- attention
 def sparse_attn(q_bits, codes, scales, idx, swa_bits, softmax_scale: float
                 ) -> Tuple[np.ndarray, np.ndarray]:
@@ -224,7 +246,8 @@ def bf16_bits(t) -> np.ndarray:
 
 def decode_group(q_tokens: int, modes: Sequence[str], seqs: Sequence[int], lens: Sequence[int],
                  owner_cache: Dict[int, Dict[int, dict]], layer_in: Dict[int, dict], top_k: int,
-                 softmax_scale: float, queries: Sequence[int] = None) -> Dict[int, dict]:
+                 softmax_scale: float, queries: Sequence[int] = None,
+                 pool_size: int = None) -> Dict[int, dict]:
     """Run the whole layer group for the given sequences and query tokens.
 
     owner_cache[owner][b] = {"codes": [T,288], "scales": [T,36], "kidx": [T,64],
@@ -232,6 +255,9 @@ def decode_group(q_tokens: int, modes: Sequence[str], seqs: Sequence[int], lens:
     layer_in[layer][b] = {"q": uint16 [Sq,16,576], "swa": uint16 [W+Sq-1,576],
                           "qidx": uint8 [Sq,4,64], "w": f32 [Sq,4]} (qidx/w for F, R)
     Returns out[layer][(b, j)] = {"idx": int32 [k], "o": f64 [16,576], "lse": f64 [16]}.
+    pool_size: when given, each Full layer also keeps its top-pool_size positions
+    as the candidate pool ("pool" in its output), and a Reindex layer scores only
+    its KV owner's pool (hierarchical sparse indexer).
     """
     own, src = plan(modes)
     queries = range(q_tokens) if queries is None else queries
@@ -243,10 +269,16 @@ def decode_group(q_tokens: int, modes: Sequence[str], seqs: Sequence[int], lens:
             cache = owner_cache[own[li]][b]
             for j in queries:
                 pos = T - q_tokens + j
-                if mode in ("F", "R"):
+                pool = None
+                if mode == "R" and pool_size is not None:
+                    idx = pool_reindex(layer_in[li][b]["qidx"][j], layer_in[li][b]["w"][j], cache["kidx"],
+                                       cache["ksig"], out[own[li]][(b, j)]["pool"], top_k)
+                elif mode in ("F", "R"):
                     s = indexer_scores(layer_in[li][b]["qidx"][j], layer_in[li][b]["w"][j],
                                        cache["kidx"][:pos + 1], cache["ksig"][:pos + 1])
                     idx = topk(s, pos + 1, top_k)
+                    if mode == "F" and pool_size is not None:
+                        pool = topk(s, pos + 1, pool_size)
                 else:
                     idx = out[src[li]][(b, j)]["idx"]
                 # SWA rows j .. j+W-1 hold positions pos-W+1 .. pos; skip negatives.
@@ -256,4 +288,6 @@ def decode_group(q_tokens: int, modes: Sequence[str], seqs: Sequence[int], lens:
                 o, lse = sparse_attn(layer_in[li][b]["q"][j], cache["codes"], cache["scales"],
                                      idx, swa, softmax_scale)
                 out[li][(b, j)] = {"idx": idx, "o": o, "lse": lse}
+                if pool is not None:
+                    out[li][(b, j)]["pool"] = pool
     return out

@@ -371,6 +371,41 @@ int orc_topk(const double *s, int64_t n_valid, int k, int32_t *out)
     return k;
 }
 
+/*
+ * Top-k inside a candidate pool ([NEO part 2]: the hierarchical sparse
+ * indexer lets later indexing layers filter only within the candidate pool
+ * built by the first Full layer, so their cost no longer grows with the
+ * context). pool[i] is a token index (-1 entries are skipped) and s[i] its
+ * score under the filtering layer's own indexer query. The k best pool
+ * entries by (score desc, token index asc) are emitted in ascending token
+ * order, -1 padded when the pool holds fewer than k valid entries. Reading:
+ * the pool is the Full layer's top-C under its own scores (C >= k, a
+ * parameter: the pages give no size).
+ */
+int orc_pool_topk(const double *s, const int32_t *pool, int n_pool, int k, int32_t *out)
+{
+    if (k <= 0)
+        return 0;
+    scored_t *all = (scored_t *)malloc((size_t)(n_pool > 0 ? n_pool : 1) * sizeof *all);
+    int n = 0;
+    for (int i = 0; i < n_pool; ++i) {
+        if (pool[i] < 0)
+            continue;
+        all[n].score = s[i] + 0.0;
+        all[n].index = pool[i];
+        ++n;
+    }
+    qsort(all, (size_t)n, sizeof *all, by_score_desc_index_asc);
+    int m = n < k ? n : k;
+    for (int i = 0; i < m; ++i)
+        out[i] = all[i].index;
+    free(all);
+    qsort(out, (size_t)m, sizeof *out, by_int_asc);
+    for (int i = m; i < k; ++i)
+        out[i] = -1;
+    return m;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Sparse attention + sliding window                                         */
 /* ------------------------------------------------------------------------ */

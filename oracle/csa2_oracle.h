@@ -96,6 +96,13 @@ void orc_indexer_scores(const uint8_t *q, const float *w, int n_heads,
  * n_valid < k. Returns the number of valid indices written. */
 int orc_topk(const double *s, int64_t n_valid, int k, int32_t *out);
 
+/* Top-k inside a candidate pool (hierarchical sparse indexer, [NEO part 2]):
+ * pool: [n_pool] token indices (-1 skipped), s: [n_pool] their scores. The k
+ * best by (score desc, token index asc), ascending, -1 padded. Returns the
+ * number of valid indices written. */
+int orc_pool_topk(const double *s, const int32_t *pool, int n_pool, int k,
+                  int32_t *out);
+
 /* ---- sparse attention over FP4 entries plus the SWA window -------------
  * ([NEO part 2]: attention over the top-k selected entries; [ZUL section 4]:
  * a per-layer sliding window of recent tokens kept beside the global KV.)

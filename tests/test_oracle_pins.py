@@ -23,6 +23,11 @@ What pins each oracle function:
                   The formula itself is a reading (parity unpinned).
   topk            numpy lexsort on tie-heavy inputs; rank-count brute force;
                   k >= n; padding
+  pool_topk       rank-count brute force on tie-heavy pools; pool order
+                  invariance; -1 entries; a pool of exactly k; the Full
+                  layer's own pool under its own scores gives its top-k
+  pool_reindex    a pool holding every valid position reduces to the full
+  (decode_group)  scan (topk); the pool is the Full layer's top-C
   sparse_attn     top-k covering every entry = dense attention computed with
                   torch's scaled_dot_product_attention in fp64 (library);
                   single key; equal logits; k = 0 (window only); no keys;
@@ -532,3 +537,64 @@ def test_decode_group_reuse_carries_full_indices_and_window_rows():
     o, lse = oracle.sparse_attn(layers[2][b]["q"][j], caches[0][b]["codes"], caches[0][b]["scales"],
                                 out[0][(b, j)]["idx"], rows, 1 / math.sqrt(576))
     np.testing.assert_array_equal(o, out[2][(b, j)]["o"])
+
+
+# ------------------------------------------------------------------ hierarchical sparse indexer
+def test_pool_topk_rank_count_bruteforce_and_order_invariance():
+    rng = np.random.default_rng(21)
+    for trial in range(200):
+        n = int(rng.integers(1, 40))
+        k = int(rng.integers(1, 12))
+        pool = rng.choice(5000, n, replace=False).astype(np.int32)
+        s = rng.integers(-3, 4, n).astype(np.float64)          # heavy ties
+        got = oracle.pool_topk(s, pool, k)
+        # rank count: an entry is kept iff fewer than k entries beat it by
+        # (score desc, token index asc)
+        beats = (s[None, :] > s[:, None]) | ((s[None, :] == s[:, None]) & (pool[None, :] < pool[:, None]))
+        keep = np.sort(pool[beats.sum(axis=1) < k])
+        want = np.full(k, -1, np.int32)
+        want[:len(keep)] = keep
+        np.testing.assert_array_equal(got, want)
+        perm = rng.permutation(n)
+        np.testing.assert_array_equal(oracle.pool_topk(s[perm], pool[perm], k), got)
+        holes = np.concatenate([pool, -np.ones(3, np.int32)])
+        np.testing.assert_array_equal(oracle.pool_topk(np.concatenate([s, [9.0, 9.0, 9.0]]), holes, k), got)
+    # a pool of exactly k entries is returned whole, sorted
+    pool = np.array([40, 3, 17, 8], np.int32)
+    np.testing.assert_array_equal(oracle.pool_topk([0.1, 0.9, 0.5, 0.2], pool, 4), np.sort(pool))
+
+
+def test_full_layer_pool_is_consistent_with_its_topk():
+    rng = np.random.default_rng(22)
+    s = rng.integers(0, 50, 3000).astype(np.float64)
+    for k, C in ((16, 64), (100, 100), (7, 2999)):
+        pool = oracle.topk(s, 3000, C)
+        np.testing.assert_array_equal(oracle.pool_topk(s[pool], pool, k), oracle.topk(s, 3000, k))
+
+
+def test_pool_reindex_with_every_position_is_the_full_scan():
+    wl = inputs.small_workload("pool", 2, 2, [700, 150], 40, modes=("F", "R", "U"))
+    caches, layers = _logical_inputs(wl)
+    scale = 1 / math.sqrt(576)
+    plain = oracle.decode_group(wl.q_tokens, wl.modes, range(wl.batch), wl.lens(), caches, layers, wl.top_k, scale)
+    big = oracle.decode_group(wl.q_tokens, wl.modes, range(wl.batch), wl.lens(), caches, layers, wl.top_k, scale,
+                              pool_size=1000)
+    small = oracle.decode_group(wl.q_tokens, wl.modes, range(wl.batch), wl.lens(), caches, layers, wl.top_k, scale,
+                                pool_size=64)
+    for key in plain[0]:
+        # a pool holding every valid position reduces to the full scan
+        np.testing.assert_array_equal(big[1][key]["idx"], plain[1][key]["idx"])
+        np.testing.assert_array_equal(big[1][key]["o"], plain[1][key]["o"])
+        # with a smaller pool the Reindex layer picks only pool members,
+        # the Full layer and its Reuse consumer are unchanged
+        pool = small[0][key]["pool"]
+        sel = small[1][key]["idx"]
+        assert set(sel[sel >= 0]) <= set(pool[pool >= 0])
+        np.testing.assert_array_equal(small[0][key]["idx"], plain[0][key]["idx"])
+        np.testing.assert_array_equal(small[2][key]["idx"], plain[2][key]["idx"])
+        b, j = key
+        pos = wl.lens()[b] - wl.q_tokens + j
+        # the pool is the Full layer's top-64 under its own scores
+        sc = oracle.indexer_scores(layers[0][b]["qidx"][j], layers[0][b]["w"][j],
+                                   caches[0][b]["kidx"][:pos + 1], caches[0][b]["ksig"][:pos + 1])
+        np.testing.assert_array_equal(pool, oracle.topk(sc, pos + 1, 64))
