@@ -11,6 +11,7 @@
 #include "indexer.cuh"
 #include "quant.cuh"
 #include "topk.cuh"
+#include "pool.cuh"
 
 namespace csa2 {
 
@@ -55,6 +56,9 @@ cudaError_t device_info(DeviceInfo **out) {
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(pool_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(pool_smem_bytes(kPoolMax)));
+        if (e != cudaSuccess) return e;
         // One shared-memory carveout for every kernel of the path, so that
         // consecutive launches do not reconfigure the SMs' L1 / shared split.
         const void *kernels[] = {reinterpret_cast<const void *>(quant_kv_fp4_kernel),
@@ -63,7 +67,9 @@ cudaError_t device_info(DeviceInfo **out) {
                                  reinterpret_cast<const void *>(topk_zero_kernel),
                                  reinterpret_cast<const void *>(topk_cluster_kernel),
                                  reinterpret_cast<const void *>(sparse_attn_kernel),
-                                 reinterpret_cast<const void *>(attn_merge_kernel)};
+                                 reinterpret_cast<const void *>(attn_merge_kernel),
+                                 reinterpret_cast<const void *>(quant_index_fp8_kernel),
+                                 reinterpret_cast<const void *>(pool_topk_kernel)};
         for (const void *kf : kernels) {
             e = cudaFuncSetAttribute(kf, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
             if (e != cudaSuccess) return e;
@@ -269,6 +275,40 @@ csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq, 
                            st, C, static_cast<const float *>(scores), L.t_cap, static_cast<const uint32_t *>(hist),
                            seq_lens, Sq, max_pages, k, out_idx);
     return cuda_status(e);
+}
+
+csa2_status csa2_indexer_pool_topk(const void *q_idx, const float *w, int B, int Sq, int idx_heads, int idx_dim,
+                                   const csa2_paged_cache *cache, const int32_t *page_table, int max_pages,
+                                   const int32_t *seq_lens, const int32_t *pool, int pool_size, int k,
+                                   int32_t *out_idx, void *stream) {
+    if (idx_heads != kIdxHeads || idx_dim != kIdxDim) return CSA2_ERR_UNSUPPORTED;
+    if (B <= 0 || Sq <= 0 || max_pages <= 0 || k <= 0 || pool_size <= 0 || !cache_ok(cache))
+        return CSA2_ERR_INVALID_ARG;
+    if (pool_size > kPoolMax || static_cast<int64_t>(B) * Sq > 65535) return CSA2_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(max_pages) * kPage > (INT64_C(1) << 30)) return CSA2_ERR_UNSUPPORTED;
+    if (cache->num_pages > INT32_MAX) return CSA2_ERR_UNSUPPORTED;
+    if (!q_idx || !w || !page_table || !seq_lens || !pool || !out_idx || !cache->kidx || !cache->kidx_scale)
+        return CSA2_ERR_INVALID_ARG;
+    if (!aligned(cache->kidx, 16) || !aligned(cache->kidx_scale, 4) || !aligned(w, 4) || !aligned(page_table, 4) ||
+        !aligned(seq_lens, 4) || !aligned(pool, 4) || !aligned(out_idx, 4))
+        return CSA2_ERR_ALIGNMENT;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return CSA2_ERR_CUDA;
+    PoolArgs A;
+    A.q_idx = static_cast<const uint8_t *>(q_idx);
+    A.w = w;
+    A.kidx = static_cast<const uint8_t *>(cache->kidx);
+    A.kidx_scale = cache->kidx_scale;
+    A.num_pages = cache->num_pages;
+    A.page_table = page_table;
+    A.max_pages = max_pages;
+    A.seq_lens = seq_lens;
+    A.Sq = Sq;
+    A.pool = pool;
+    A.C = pool_size;
+    A.k = k;
+    A.out = out_idx;
+    return cuda_status(launch_pool_topk(A, B * Sq, static_cast<cudaStream_t>(stream)));
 }
 
 size_t csa2_sparse_attn_workspace_bytes(int B, int Sq, int k) {

@@ -24,8 +24,8 @@ STATUS = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_UNSUPPORTED", 3:
           7: "CSA2_ERR_WORKSPACE", 8: "CSA2_ERR_ALIGNMENT"}
 
 # Every function include/csa2.h declares (checked by the CPU test suite).
-EXPORTS = ("csa2_quant_kv_fp4", "csa2_quant_indexer_fp8", "csa2_indexer_topk_workspace_bytes", "csa2_indexer_topk",
-           "csa2_sparse_attn_workspace_bytes", "csa2_sparse_attn_decode",
+EXPORTS = ("csa2_quant_kv_fp4", "csa2_quant_indexer_fp8", "csa2_indexer_topk_workspace_bytes",
+           "csa2_indexer_topk", "csa2_indexer_pool_topk", "csa2_sparse_attn_workspace_bytes", "csa2_sparse_attn_decode",
            "csa2_sparse_attn_decode_noalloc", "csa2_plan",
            "csa2_last_device_error", "csa2_status_string", "csa2_launch_count")
 
@@ -57,6 +57,8 @@ def _load():
         "csa2_indexer_topk_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
         "csa2_indexer_topk": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _cp, _vp, _i32, _vp, _i32, _vp,
                                      _vp, _sz, _vp]),
+        "csa2_indexer_pool_topk": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _cp, _vp, _i32, _vp, _vp, _i32, _i32,
+                                          _vp, _vp]),
         "csa2_sparse_attn_workspace_bytes": (_sz, [_i32, _i32, _i32]),
         "csa2_sparse_attn_decode": (_i32, [_vp, _i32, _i32, _i32, _i32, _cp, _vp, _i32, _vp, _vp, _i32,
                                            _vp, _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
@@ -195,6 +197,28 @@ def indexer_topk(q_idx: torch.Tensor, w: torch.Tensor, cache: PagedCache, page_t
                               _ptr(page_table), max_pages, _ptr(seq_lens), k, _ptr(out), _ptr(ws),
                               ws.numel() * ws.element_size(), _stream())
     _check("csa2_indexer_topk", rc)
+    return out
+
+
+def indexer_pool_topk(q_idx: torch.Tensor, w: torch.Tensor, cache: PagedCache, page_table: torch.Tensor,
+                      seq_lens: torch.Tensor, pool: torch.Tensor, k: int,
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Top-k of each query row's candidate pool [B, Sq, C] (ascending token indices, -1 skipped)."""
+    B, Sq = q_idx.shape[0], q_idx.shape[1]
+    max_pages = page_table.shape[1]
+    C = pool.shape[2]
+    _req(q_idx, torch.uint8, "q_idx", (B, Sq, IDX_HEADS, IDX_DIM))
+    _req(w, torch.float32, "w", (B, Sq, IDX_HEADS))
+    _req(page_table, torch.int32, "page_table", (B, max_pages))
+    _req(seq_lens, torch.int32, "seq_lens", (B,))
+    _req(pool, torch.int32, "pool", (B, Sq, C))
+    if out is None:
+        out = torch.empty(B, Sq, k, dtype=torch.int32, device=q_idx.device)
+    _req(out, torch.int32, "out_idx", (B, Sq, k))
+    rc = _L.csa2_indexer_pool_topk(_ptr(q_idx), _ptr(w), B, Sq, IDX_HEADS, IDX_DIM, ctypes.byref(cache.desc),
+                                   _ptr(page_table), max_pages, _ptr(seq_lens), _ptr(pool), C, k, _ptr(out),
+                                   _stream())
+    _check("csa2_indexer_pool_topk", rc)
     return out
 
 

@@ -195,6 +195,38 @@ csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq,
                               void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * csa2_indexer_pool_topk -- Reindex under the hierarchical sparse indexer
+ * ([NEO part 2]: later indexing layers filter only within the candidate pool
+ * built by the first Full layer, so their cost does not grow with the
+ * context).
+ *
+ * For query row (b, j), scores only the tokens of pool[b][j] with the same
+ * formula as csa2_indexer_topk (this layer's q_idx and w, the owner's indexer
+ * keys and sigma) and writes to out_idx[b][j] the k best by (score desc,
+ * token index asc), in ascending token order, -1 padded when the pool holds
+ * fewer than k valid entries. The pool is typically the Full layer's
+ * csa2_indexer_topk output for k = pool_size (its top-C); with this layer's
+ * own q and w over its own pool the call returns exactly its top-k.
+ *
+ *   q_idx, w, cache, page_table, seq_lens, max_pages: as csa2_indexer_topk
+ *   pool        device int32 [B][Sq][pool_size]: token indices in ascending
+ *               order, -1 entries skipped; an entry >= seq_lens[b], a bad
+ *               page-table entry or a descending pair sets
+ *               CSA2_ERR_DEVICE_BOUNDS (the entry is skipped)
+ *   pool_size   1 <= pool_size <= 32768 (CSA2_ERR_UNSUPPORTED above)
+ *   k           k >= 1
+ *   out_idx     device int32 [B][Sq][k]
+ * No workspace. Limits: 4 indexer heads x 64 channels, B * Sq <= 65535.
+ */
+csa2_status csa2_indexer_pool_topk(const void *q_idx, const float *w, int B, int Sq,
+                                   int idx_heads, int idx_dim,
+                                   const csa2_paged_cache *cache,
+                                   const int32_t *page_table, int max_pages,
+                                   const int32_t *seq_lens, const int32_t *pool,
+                                   int pool_size, int k, int32_t *out_idx,
+                                   void *stream);
+
+/*
  * csa2_sparse_attn_decode -- all modes: attention over the selected FP4
  * entries plus the sliding window ([NEO part 2]; [ZUL section 4]).
  *

@@ -99,6 +99,14 @@ def test_unsupported_shapes_rejected_on_host(lib):
     assert L.csa2_quant_indexer_fp8(24, 4, 64, 16, 16, None) == 8
     assert L.csa2_quant_indexer_fp8(16, 4, 64, 24, 16, None) == 8
     assert L.csa2_quant_indexer_fp8(16, 0, 64, None, None, None) == 0
+    # candidate-pool top-k: indexer shape, pool size limit, bad sizes, null pointers
+    assert L.csa2_indexer_pool_topk(16, 16, 1, 1, 8, 64, ctypes.byref(cache), 16, 1, 16, 16, 64, 8, 16, None) == 2
+    assert L.csa2_indexer_pool_topk(16, 16, 1, 1, 4, 64, ctypes.byref(cache), 16, 1, 16, 16, 40000, 8, 16,
+                                    None) == 2
+    assert L.csa2_indexer_pool_topk(16, 16, 1, 1, 4, 64, ctypes.byref(cache), 16, 1, 16, 16, 64, 0, 16, None) == 1
+    assert L.csa2_indexer_pool_topk(16, 16, 1, 1, 4, 64, ctypes.byref(cache), 16, 1, 16, 16, 0, 8, 16, None) == 1
+    assert L.csa2_indexer_pool_topk(16, 16, 1, 1, 4, 64, ctypes.byref(cache), 16, 1, 16, None, 64, 8, 16,
+                                    None) == 1
     assert lib.launch_count() == 0
 
 
