@@ -9,6 +9,11 @@ reused across layers.
 No device work happens here beyond calling the library: a Reuse layer's index
 tensor IS its source layer's tensor (same storage, no copy), and every layer
 of an owner reads that owner's PagedCache.
+
+With pool_size set (the hierarchical sparse indexer, neodrop.ai architecture
+part 2), a Full layer keeps its top-pool_size positions as a candidate pool
+and takes its own top-k inside it. A Reindex layer then scores only its KV
+owner's pool instead of the whole context.
 """
 from __future__ import annotations
 
@@ -24,7 +29,8 @@ DEFAULT_SCALE = 1.0 / math.sqrt(lib.DIM)
 
 class LayerGroup:
     def __init__(self, modes: Sequence[str], batch: int, q_tokens: int, max_pages: int,
-                 num_pages: int, top_k: int, device="cuda", softmax_scale: float = DEFAULT_SCALE):
+                 num_pages: int, top_k: int, device="cuda", softmax_scale: float = DEFAULT_SCALE,
+                 pool_size: Optional[int] = None):
         self.modes = tuple(modes)
         self.kv_owner, self.index_src = lib.plan(self.modes)
         self.B, self.Sq, self.k = batch, q_tokens, top_k
@@ -41,6 +47,12 @@ class LayerGroup:
                     for _ in range(n)]
         self.lse = [torch.empty(batch, q_tokens, lib.HEADS, dtype=torch.float32, device=device)
                     for _ in range(n)]
+        self.pool_size = pool_size
+        if pool_size is not None and pool_size < top_k:
+            raise ValueError(f"pool_size {pool_size} must be at least top_k {top_k}")
+        self._pool: Dict[int, torch.Tensor] = {} if pool_size is None else {
+            i: torch.full((batch, q_tokens, pool_size), -1, dtype=torch.int32, device=device)
+            for i, m in enumerate(self.modes) if m == "F"}
         self.ws_idx = lib.workspace(lib.indexer_topk_workspace_bytes(batch, q_tokens, max_pages, top_k), device)
         self.ws_att = lib.workspace(lib.sparse_attn_workspace_bytes(batch, q_tokens, top_k), device)
 
@@ -50,6 +62,10 @@ class LayerGroup:
 
     def cache(self, layer: int) -> lib.PagedCache:
         return self.caches[self.kv_owner[layer]]
+
+    def pool(self, layer: int) -> torch.Tensor:
+        """The candidate pool a layer's selection reads (its KV owner's), when pool_size is set."""
+        return self._pool[self.kv_owner[layer]]
 
     def step(self, page_table: torch.Tensor, seq_lens: torch.Tensor, q: List[torch.Tensor],
              swa: List[torch.Tensor], q_idx: Dict[int, torch.Tensor], w: Dict[int, torch.Tensor],
@@ -71,7 +87,13 @@ class LayerGroup:
             if mode == "F" and append is not None and li in append:
                 x_new, slots, kidx_new, ksig_new = append[li]
                 lib.quant_kv_fp4(x_new, slots, cache, kidx_new, ksig_new)
-            if mode in ("F", "R"):
+            if mode in ("F", "R") and self.pool_size is not None:
+                if mode == "F":
+                    lib.indexer_topk(q_idx[li], w[li], cache, page_table, seq_lens, self.pool_size,
+                                     out=self._pool[li], ws=self.ws_idx)
+                lib.indexer_pool_topk(q_idx[li], w[li], cache, page_table, seq_lens, self.pool(li), self.k,
+                                      out=self._index[li])
+            elif mode in ("F", "R"):
                 lib.indexer_topk(q_idx[li], w[li], cache, page_table, seq_lens, self.k,
                                  out=self._index[li], ws=self.ws_idx)
             lib.sparse_attn_decode(q[li], cache, page_table, seq_lens, self.index(li), swa[li], self.scale,
