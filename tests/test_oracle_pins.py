@@ -598,3 +598,32 @@ def test_pool_reindex_with_every_position_is_the_full_scan():
         sc = oracle.indexer_scores(layers[0][b]["qidx"][j], layers[0][b]["w"][j],
                                    caches[0][b]["kidx"][:pos + 1], caches[0][b]["ksig"][:pos + 1])
         np.testing.assert_array_equal(pool, oracle.topk(sc, pos + 1, 64))
+
+
+# ------------------------------------------------------------------ replay (window-only, many query tokens)
+def test_window_only_queries_are_banded_causal_attention():
+    """L query tokens with no selected entries, each over its 128 window rows
+    (rows j .. j+127 of a [127 + L]-row window tensor; rows at negative
+    positions skipped), equal banded causal attention computed by torch's
+    scaled_dot_product_attention in fp64 with a band mask (library)."""
+    g = torch.Generator().manual_seed(31)
+    W, L = 128, 40
+    scale = 1 / math.sqrt(576)
+    q = torch.randn(L, 16, 576, generator=g).to(torch.bfloat16)
+    rows = torch.randn(W + L - 1, 576, generator=g).to(torch.bfloat16)
+    empty = np.zeros((0, 288), np.uint8), np.zeros((0, 36), np.uint8)
+    for T in (W + L - 1, 60):                       # full window, and a short sequence
+        first = T - (W + L - 1)                     # position of window row 0
+        q64 = q.to(torch.float64).transpose(0, 1)   # [16, L, 576]
+        kv64 = rows.to(torch.float64)
+        r = torch.arange(W + L - 1)
+        j = torch.arange(L)[:, None]
+        band = (r[None, :] >= j) & (r[None, :] <= j + W - 1) & (first + r[None, :] >= 0)
+        ro = F.scaled_dot_product_attention(q64, kv64[None], kv64[None], attn_mask=band[None], scale=scale)
+        for jj in (0, 17, L - 1):
+            sel = [x for x in range(jj, jj + W) if first + x >= 0]
+            o, lse = oracle.sparse_attn(oracle.bf16_bits(q[jj]), *empty, np.zeros(0, np.int32),
+                                        oracle.bf16_bits(rows)[sel], scale)
+            np.testing.assert_allclose(o, ro[:, jj].numpy(), rtol=0, atol=1e-12)
+            logits = (q64[:, jj] @ kv64[band[jj]].T) * scale
+            np.testing.assert_allclose(lse, torch.logsumexp(logits, dim=-1).numpy(), rtol=0, atol=1e-12)
