@@ -36,7 +36,7 @@ struct PoolSmemFixed {
     uint32_t hist[kPoolBins];
     uint64_t wbuf64[kPoolThreads / 32 + 1];
     uint32_t wbuf[kPoolThreads / 32 + 1];
-    uint32_t s_bin, s_above, s_valid;
+    uint32_t s_bin, s_above;
 };
 
 constexpr size_t pool_smem_bytes(int pool_size) {
@@ -108,7 +108,6 @@ pool_topk_kernel(const PoolArgs A) {
         (&fs.q[0][0])[2 * tid + 1] = f.y;
     }
     if (tid < kIdxHeads) fs.w[tid] = A.w[static_cast<int64_t>(row) * kIdxHeads + tid];
-    if (tid == 0) fs.s_valid = 0u;
     int T = A.seq_lens[b];
     pdl_wait();                                  // the pool is written by the previous kernel
     pdl_trigger();
