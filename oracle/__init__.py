@@ -202,6 +202,33 @@ def pool_reindex(q, w, kidx, ksig, pool, k: int) -> np.ndarray:
     return pool_topk(s, valid, k)
 
 
+# ---------------------------------------------------------------- context-parallel merges
+def merge_topk_candidates(scores: Sequence[np.ndarray], idx: Sequence[np.ndarray], k: int) -> np.ndarray:
+    """Global top-k from per-shard candidate lists (scores f64, global token
+    indices int32, -1 entries skipped): the k best of their union by (score
+    desc, token index asc), ascending, -1 padded. Each shard's own top-k holds
+    every one of its positions that belongs to the global top-k, so this is
+    the top-k of the whole context (plan of the scope table's multi-GPU part)."""
+    s = np.concatenate([np.asarray(x, np.float64) for x in scores]) if scores else np.zeros(0)
+    p = np.concatenate([np.asarray(x, np.int32) for x in idx]) if idx else np.zeros(0, np.int32)
+    return pool_topk(s, p, k)
+
+
+def lse_merge(outs: Sequence[np.ndarray], lses: Sequence[np.ndarray]) -> Tuple[np.ndarray, np.ndarray]:
+    """One softmax over the union of disjoint key sets from per-shard
+    results: o = sum_r exp(lse_r - L) o_r, lse = L = log sum_r exp(lse_r)
+    (a shard with no key has lse = -inf and weight 0). fp64."""
+    o = np.stack([np.asarray(x, np.float64) for x in outs])       # [G, H, D]
+    l = np.stack([np.asarray(x, np.float64) for x in lses])       # [G, H]
+    m = l.max(axis=0)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    wts = np.where(np.isfinite(l), np.exp(l - m_safe[None]), 0.0)
+    tot = wts.sum(axis=0)
+    out = np.where(tot[:, None] > 0, (wts[:, :, None] * o).sum(axis=0) / np.where(tot > 0, tot, 1.0)[:, None], 0.0)
+    lse = np.where(tot > 0, m_safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    return out, lse
+
+
 # ---------------------------------------------------------------- attention
 def sparse_attn(q_bits, codes, scales, idx, swa_bits, softmax_scale: float
                 ) -> Tuple[np.ndarray, np.ndarray]:

@@ -28,6 +28,10 @@ What pins each oracle function:
                   layer's own pool under its own scores gives its top-k
   pool_reindex    a pool holding every valid position reduces to the full
   (decode_group)  scan (topk); the pool is the Full layer's top-C
+  merge_topk_candidates  per-shard top-k lists merged = the unsharded top-k
+                  (tie-heavy scores, 2 to 8 shards)
+  lse_merge       attention split over shards and merged = one softmax over
+                  the union; an empty shard contributes nothing
   sparse_attn     top-k covering every entry = dense attention computed with
                   torch's scaled_dot_product_attention in fp64 (library);
                   single key; equal logits; k = 0 (window only); no keys;
@@ -627,3 +631,43 @@ def test_window_only_queries_are_banded_causal_attention():
             np.testing.assert_allclose(o, ro[:, jj].numpy(), rtol=0, atol=1e-12)
             logits = (q64[:, jj] @ kv64[band[jj]].T) * scale
             np.testing.assert_allclose(lse, torch.logsumexp(logits, dim=-1).numpy(), rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------------ context-parallel merges
+def test_sharded_topk_merge_equals_unsharded_topk():
+    """Each of G shards takes the top-k of its own contiguous positions; the
+    merge of their candidate lists equals the top-k of the whole context
+    (heavy ties included, so the tie rule must survive the merge)."""
+    rng = np.random.default_rng(41)
+    for G, n, k in ((2, 3000, 100), (4, 1001, 257), (8, 640, 640), (3, 50, 80)):
+        s = rng.integers(0, 20, n).astype(np.float64)
+        want = oracle.topk(s, n, k)
+        bounds = np.linspace(0, n, G + 1).astype(int)
+        cs, ci = [], []
+        for r in range(G):
+            t0, t1 = bounds[r], bounds[r + 1]
+            loc = oracle.topk(s[t0:t1], t1 - t0, k)
+            loc = loc[loc >= 0]
+            cs.append(s[t0 + loc])
+            ci.append((t0 + loc).astype(np.int32))
+        np.testing.assert_array_equal(oracle.merge_topk_candidates(cs, ci, k), want)
+
+
+def test_sharded_attention_lse_merge_equals_one_softmax():
+    """Attention over the selected entries split between shards (the window
+    on the last shard), merged by LSE, equals one softmax over all of them;
+    a shard with no key contributes nothing."""
+    q, codes, scales, swa = _rand_case(43, n_cache=40, n_swa=7)
+    scale = 1 / math.sqrt(576)
+    qb, wb = oracle.bf16_bits(q), oracle.bf16_bits(swa)
+    idx = np.arange(40, dtype=np.int32)
+    o_all, lse_all = oracle.sparse_attn(qb, codes, scales, idx, wb, scale)
+    no_rows = np.zeros((0, 576), np.uint16)
+    parts = [(idx[:13], no_rows), (np.zeros(0, np.int32), no_rows), (idx[13:], wb)]
+    res = [oracle.sparse_attn(qb, codes, scales, i, rows, scale) for i, rows in parts]
+    assert np.all(np.isneginf(res[1][1]))
+    o, lse = oracle.lse_merge([r[0] for r in res], [r[1] for r in res])
+    np.testing.assert_allclose(o, o_all, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_all, rtol=0, atol=1e-12)
+    o0, l0 = oracle.lse_merge([res[1][0]], [res[1][1]])
+    assert np.all(o0 == 0) and np.all(np.isneginf(l0))
