@@ -11,6 +11,14 @@ indexes, every layer attends (K4 + K5). Default workload: batch 64, context
 Multi-GPU: one process per GPU (torchrun); every rank runs an independent
 replica with its own seed (weak scaling, no collective on the data path);
 time is the max over ranks. Rank 0 prints one JSON line.
+
+Besides the step, the line carries two kernels outside the default step,
+each timed with events around every launch:
+  indexer_fp8_quant   csa2_quant_indexer_fp8 over B x T rows of 64 bf16
+                      channels (more than L2 holds);
+  indexer_pool_topk   csa2_indexer_pool_topk, a Reindex query selecting the
+                      top-k inside the Full layer's top-4k, L2 flushed before
+                      each launch (one GPU only).
 """
 from __future__ import annotations
 
