@@ -56,8 +56,8 @@ def lib():
         L.orc_quant_fp4.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int, _u8p, _u8p]
         L.orc_dequant_fp4.restype = None
         L.orc_dequant_fp4.argtypes = [_u8p, _u8p, ctypes.c_int64, ctypes.c_int, _f64p]
-        L.orc_e4m3_code.restype = ctypes.c_uint8
-        L.orc_e4m3_code.argtypes = [ctypes.c_float]
+        L.orc_e4m3_code_quotient.restype = ctypes.c_uint8
+        L.orc_e4m3_code_quotient.argtypes = [ctypes.c_double, ctypes.c_float]
         L.orc_quant_index_fp8.restype = None
         L.orc_quant_index_fp8.argtypes = [_u16p, ctypes.c_int64, ctypes.c_int, _u8p, _f32p]
         L.orc_indexer_scores.restype = None
@@ -145,9 +145,10 @@ def dequant_fp4(codes, scales) -> np.ndarray:
 
 
 # ---------------------------------------------------------------- indexer FP8 quantiser
-def e4m3_code(r: float) -> int:
-    """E4M3FN code of the binary32 value nearest r (the argument is passed as a C float)."""
-    return int(lib().orc_e4m3_code(float(r)))
+def e4m3_code_quotient(x: float, sigma: float) -> int:
+    """E4M3FN code nearest to the exact quotient x / sigma (x passed as a C
+    double, sigma > 0 as a C float)."""
+    return int(lib().orc_e4m3_code_quotient(float(x), float(sigma)))
 
 
 def quant_index_fp8(x_bf16_bits) -> Tuple[np.ndarray, np.ndarray]:

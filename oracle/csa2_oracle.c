@@ -216,36 +216,43 @@ void orc_dequant_fp4(const uint8_t *codes, const uint8_t *scales, int64_t n,
 /* ------------------------------------------------------------------------ */
 
 /*
- * E4M3FN code of a binary32 value r, round to nearest with ties to the even
- * mantissa, saturating at +-448, canonical +0 when the magnitude rounds to 0.
- * Method as in orc_group_scale: the grid step in the binade [2^E, 2^(E+1))
- * is 2^(E-3) for E >= -6, and the subnormal step 2^-9 continues below 2^-6.
- * r is a binary32 value, exact in fp64, so r / step is exact and nearbyint
- * performs the one rounding.
+ * E4M3FN code of the exact quotient x / sigma, for a finite x and a binary32
+ * sigma > 0: the grid value nearest to x / sigma, ties to the even mantissa,
+ * saturating at +-448 (the largest finite value: anything above it is
+ * nearest to it), canonical +0 when the magnitude rounds to 0.
+ *
+ * The quotient itself is never formed, so nothing is rounded before the one
+ * rounding onto the E4M3 grid. The grid values v_0 = 0 < v_1 < ... < v_126 =
+ * 448 are the non-negative codes 0x00..0x7E in order. The nearest value is
+ * found by comparing |x| with products v_i * sigma and with the midpoints
+ * (v_i + v_(i+1)) / 2 * sigma: a grid value has at most 4 significant bits, a
+ * midpoint at most 5, sigma at most 24, so every product is exact in fp64,
+ * and every comparison below is an exact comparison of real numbers.
  */
-uint8_t orc_e4m3_code(float r)
+uint8_t orc_e4m3_code_quotient(double x, float sigma)
 {
-    double a = fabs((double)r);
-    double mag;
-    if (a >= 448.0) {
-        mag = 448.0;
-    } else if (a == 0.0) {
-        mag = 0.0;
+    double a = fabs(x);
+    double s = (double)sigma;
+    /* i = the largest grid index with v_i * sigma <= |x| (v_0 = 0 always is) */
+    int i = 0;
+    while (i < 126 && orc_e4m3_value((uint8_t)(i + 1)) * s <= a)
+        ++i;
+    int code;
+    if (i == 126) {
+        code = 126;                               /* at or above 448: saturate */
     } else {
-        int e;
-        frexp(a, &e);
-        int E = e - 1;
-        if (E < -6)
-            E = -6;
-        double step = ldexp(1.0, E - 3);
-        mag = nearbyint(a / step) * step;   /* may carry to 2^(E+1): still on the grid */
-        if (mag > 448.0)
-            mag = 448.0;
+        double mid = 0.5 * (orc_e4m3_value((uint8_t)i) + orc_e4m3_value((uint8_t)(i + 1)));
+        double ms = mid * s;
+        if (a < ms)
+            code = i;
+        else if (a > ms)
+            code = i + 1;
+        else
+            code = (i % 2 == 0) ? i : i + 1;      /* exact tie: even mantissa */
     }
-    if (mag == 0.0)
+    if (code == 0)
         return 0;
-    uint8_t code = e4m3_encode_exact(mag);
-    return (r < 0.0f) ? (uint8_t)(code | 0x80) : code;
+    return (x < 0.0) ? (uint8_t)(code | 0x80) : (uint8_t)code;
 }
 
 /*
@@ -253,11 +260,13 @@ uint8_t orc_e4m3_code(float r)
  * among the state a KV owner hands to its consumer layers, and [NEO part 2]
  * has the indexer read FP8 operands; the pages give no rule for the scale.
  * Reading: one binary32 scale per row of `dim` channels,
- *     sigma = amax / 448   (binary32 division; 0 for an all-zero row),
- * and code_c = E4M3FN nearest to x_c / sigma (binary32 division, then one
- * round to nearest even, saturating; all codes 0 when sigma = 0). Both
- * divisions are binary32 so that a kernel dividing in fp32 takes the same
- * integer decisions; the dequantised value is sigma * e4m3(code).
+ *     sigma = the binary32 value nearest to amax / 448 (0 for an all-zero
+ *             row), so that the row's largest magnitude lands on the top
+ *             E4M3 value,
+ * and code_c = the E4M3FN value nearest to the exact quotient x_c / sigma
+ * (orc_e4m3_code_quotient: one rounding, ties to even, saturating, canonical
+ * +0; all codes 0 when sigma = 0). The dequantised value is
+ * sigma * e4m3(code).
  */
 void orc_quant_index_fp8(const uint16_t *x_bf16, int64_t n_rows, int dim,
                          uint8_t *codes, float *sigma)
@@ -270,17 +279,12 @@ void orc_quant_index_fp8(const uint16_t *x_bf16, int64_t n_rows, int dim,
             if (v > amax)
                 amax = v;
         }
-        float sg = (float)amax / 448.0f;      /* amax is a bf16 value: exact in binary32 */
+        /* amax is a bf16 value, exact in binary32; the IEEE binary32 division
+         * rounds the exact quotient amax / 448 to nearest (even). */
+        float sg = (float)amax / 448.0f;
         sigma[t] = sg;
-        for (int c = 0; c < dim; ++c) {
-            if (sg == 0.0f) {
-                codes[t * dim + c] = 0;
-                continue;
-            }
-            float x = (float)orc_bf16_value(row[c]);
-            float r = x / sg;
-            codes[t * dim + c] = orc_e4m3_code(r);
-        }
+        for (int c = 0; c < dim; ++c)
+            codes[t * dim + c] = (sg == 0.0f) ? 0 : orc_e4m3_code_quotient(orc_bf16_value(row[c]), sg);
     }
 }
 

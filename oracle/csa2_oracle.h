@@ -71,13 +71,14 @@ void orc_dequant_fp4(const uint8_t *codes, const uint8_t *scales, int64_t n,
 
 /* ---- indexer FP8 quantiser ([ZUL section 3] "indexer K / scale") ------- */
 
-/* E4M3FN code of a binary32 value: nearest, ties to even mantissa,
- * saturating at +-448, canonical +0. */
-uint8_t orc_e4m3_code(float r);
+/* E4M3FN code of the exact quotient x / sigma (sigma > 0 binary32): nearest
+ * grid value, ties to even mantissa, saturating at +-448, canonical +0. */
+uint8_t orc_e4m3_code_quotient(double x, float sigma);
 
 /* n_rows rows of `dim` bf16 channels -> codes [n_rows][dim] (E4M3FN) and one
- * binary32 scale per row: sigma = amax / 448 and code = e4m3(x / sigma), both
- * divisions in binary32; an all-zero row gives sigma = 0 and zero codes. */
+ * binary32 scale per row: sigma = binary32 nearest to amax / 448 and
+ * code = orc_e4m3_code_quotient(x, sigma); an all-zero row gives sigma = 0
+ * and zero codes. */
 void orc_quant_index_fp8(const uint16_t *x_bf16, int64_t n_rows, int dim,
                          uint8_t *codes, float *sigma);
 

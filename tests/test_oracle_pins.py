@@ -10,13 +10,17 @@ What pins each oracle function:
                   finite E4M3 scale: brute-force argmin of |x - s*m|
   quant_fp4       group/nibble layout against a composition written here from
                   the pinned pieces; error bound; idempotence; bytes per token
-  e4m3_code       torch's RNE float8_e4m3fn cast (library) and a brute-force
-                  nearest search over every finite bf16 value in range and
-                  every E4M3 midpoint with its binary32 neighbours;
-                  saturation; canonical +0
-  quant_index_fp8 sigma against numpy binary32 division (library); codes
-                  against brute force on wide-magnitude rows; idempotence on
-                  E4M3-grid rows; power-of-two equivariance; error bound;
+  e4m3_code_quotient  with sigma = 1: torch's RNE float8_e4m3fn cast
+                  (library) and a brute-force nearest search over every finite
+                  bf16 value in range and every E4M3 midpoint with its
+                  binary32 neighbours; saturation; canonical +0
+  quant_index_fp8 sigma: the binary32 value nearest amax / 448, checked in
+                  exact rationals against its neighbours; codes: an
+                  exact-rational brute force over all 127 grid values on
+                  wide-magnitude rows and on rows where the binary32 quotient
+                  lands on an E4M3 midpoint that the exact quotient misses
+                  (where the two roundings differ); idempotence on E4M3-grid
+                  rows; power-of-two equivariance; half-step error bound;
                   zero rows
   indexer_scores  one-hot head weights reduce to an integer matmul (numpy);
                   linearity in w; ReLU placement with negative sigma; q = 0.
@@ -41,6 +45,7 @@ What pins each oracle function:
                   128 rows per query (golden constant)
 """
 import math
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -139,7 +144,11 @@ def e4m3_nearest_bruteforce(r: np.ndarray) -> np.ndarray:
     return np.where((r < 0) & (pick != 0), pick | 0x80, pick).astype(np.uint8)
 
 
-def test_e4m3_code_against_torch_cast_and_bruteforce():
+def test_e4m3_code_quotient_sigma_one_against_torch_cast_and_bruteforce():
+    """With sigma = 1 the quotient is x itself: every finite bf16 value in
+    range and every E4M3 midpoint with its binary32 neighbours against
+    torch's RNE float8_e4m3fn cast (library) and the brute-force nearest
+    search; saturation; canonical +0."""
     _, vals = all_finite_bf16_bits()
     ev = e4m3_finite_values()[:127]
     mids = ((ev[:-1] + ev[1:]) / 2).astype(np.float32)          # exact: at most 5 significant bits
@@ -147,14 +156,14 @@ def test_e4m3_code_against_torch_cast_and_bruteforce():
     up = np.nextafter(mids, np.float32(np.inf))
     down = np.nextafter(mids, np.float32(0))
     r = np.concatenate([vals[np.abs(vals) <= 448].astype(np.float32), mids, up, down, -mids, -up, -down])
-    got = np.array([oracle.e4m3_code(float(x)) for x in r], np.uint8)
+    got = np.array([oracle.e4m3_code_quotient(float(x), 1.0) for x in r], np.uint8)
     ref = torch.from_numpy(r).to(torch.float8_e4m3fn).view(torch.uint8).numpy().copy()
     ref[(ref & 0x7F) == 0] = 0                                    # canonical +0
     np.testing.assert_array_equal(got, ref)
     np.testing.assert_array_equal(got, e4m3_nearest_bruteforce(r))
     # saturation above the largest finite value, both signs
     for x in (448.5, 464.0, 1e6, 3.0e38):
-        assert oracle.e4m3_code(x) == 0x7E and oracle.e4m3_code(-x) == 0xFE
+        assert oracle.e4m3_code_quotient(x, 1.0) == 0x7E and oracle.e4m3_code_quotient(-x, 1.0) == 0xFE
 
 
 def bf16_rows(x: np.ndarray) -> np.ndarray:
@@ -165,9 +174,83 @@ def bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32)
 
 
-def test_quant_index_fp8_rows_against_bruteforce():
+E4M3_GRID = [Fraction(float(v)) for v in e4m3_finite_values()[:127]]   # codes 0x00 .. 0x7E, ascending
+
+
+def exact_nearest_e4m3(x: float, sigma: float) -> int:
+    """Brute force in exact rationals: the E4M3FN byte whose value is nearest
+    to x / sigma over all 127 non-negative grid values (ties to the even
+    byte, saturating at 448, canonical +0). Independent of the oracle's
+    midpoint comparisons and of any binary32 quotient."""
+    r = abs(Fraction(x) / Fraction(sigma))
+    best_d, best_i = None, 0
+    for i, v in enumerate(E4M3_GRID):
+        d = abs(r - v)
+        if best_d is None or d < best_d or (d == best_d and i % 2 == 0):
+            best_d, best_i = d, i
+    if best_i == 0:
+        return 0
+    return best_i | 0x80 if x < 0 else best_i
+
+
+def binary32_nearest(q: Fraction) -> np.float32:
+    """The binary32 value nearest to a positive rational q (ties to even),
+    found by comparing the candidates around float(q) exactly."""
+    c = np.float32(float(q))
+    cands = [np.nextafter(c, np.float32(0)), c, np.nextafter(c, np.float32(np.inf))]
+    best = min(cands, key=lambda f: (abs(Fraction(float(f)) - q), int(np.array(f).view(np.uint32)) & 1))
+    return np.float32(best)
+
+
+def double_rounding_rows(n_rows: int, seed: int) -> np.ndarray:
+    """bf16 rows (as bits) whose row maximum fixes sigma and whose other
+    channels x make the binary32 quotient RN(x / sigma) land exactly on an
+    E4M3 midpoint while the exact quotient does not: the inputs on which
+    rounding the exact quotient and rounding the binary32 quotient differ.
+    Found by a vectorised search over every positive bf16 value."""
+    ev = e4m3_finite_values()[:127]
+    mids = np.unique(((ev[:-1] + ev[1:]) / 2).astype(np.float32))
+    _, vals = all_finite_bf16_bits()
+    pos = vals[vals > 0].astype(np.float32)
+    rng = np.random.default_rng(seed)
+    rows = []
+    while len(rows) < n_rows:
+        amax = np.float32(rng.choice(pos[(pos > 1e-30) & (pos < 1e30)]))
+        sg = amax / np.float32(448.0)
+        xs = pos[pos < amax]
+        q = xs / sg
+        hit = xs[np.isin(q, mids)]
+        hit = [x for x in hit if Fraction(float(x)) / Fraction(float(sg)) != Fraction(float(x / sg))]
+        if not hit:
+            continue
+        take = np.array(hit[:63], np.float32)
+        row = np.zeros(64, np.float32)
+        row[0] = amax
+        row[1:1 + len(take)] = take * np.where(np.arange(len(take)) % 2 == 0, 1, -1)
+        rows.append(row)
+    return bf16_rows(np.array(rows))
+
+
+def test_quant_index_fp8_sigma_is_the_nearest_binary32():
+    """sigma is the binary32 value nearest to amax / 448, checked in exact
+    rationals against its neighbours (not by repeating the division)."""
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((400, 64)) * np.exp2(rng.integers(-120, 120, (400, 1)))
+    x[0] = 0.0
+    x[1, 3] = 1e-39                                               # a bf16 subnormal maximum
+    bits = bf16_rows(x)
+    _, sigma = oracle.quant_index_fp8(bits)
+    amax = np.abs(bits_to_f32(bits)).max(axis=1)
+    assert sigma[0] == 0.0
+    for a, s in zip(amax[1:], sigma[1:]):
+        assert s == binary32_nearest(Fraction(float(a)) / 448), (a, s)
+
+
+def test_quant_index_fp8_codes_against_exact_bruteforce():
+    """Codes against the exact-rational brute force on wide-magnitude rows,
+    zero / subnormal / near-maximum rows, and the double-rounding rows."""
     rng = np.random.default_rng(11)
-    x = rng.standard_normal((300, 64)) * np.exp2(rng.integers(-60, 60, (300, 1)))
+    x = rng.standard_normal((40, 64)) * np.exp2(rng.integers(-60, 60, (40, 1)))
     x[0] = 0.0
     x[1] = -0.0
     x[2] = 0.0
@@ -175,19 +258,31 @@ def test_quant_index_fp8_rows_against_bruteforce():
     x[3] = rng.standard_normal(64) * 1e-39                        # bf16 subnormals
     x[4, :] = 3.3e38                                              # near the bf16 maximum
     x[4, ::2] *= -1
-    bits = bf16_rows(x)
+    bits = np.concatenate([bf16_rows(x), double_rounding_rows(12, seed=1)])
     codes, sigma = oracle.quant_index_fp8(bits)
     xv = bits_to_f32(bits)
-    amax = np.abs(xv).max(axis=1)
-    np.testing.assert_array_equal(sigma, amax / np.float32(448.0))          # numpy binary32 division
     assert sigma[0] == 0 and sigma[1] == 0 and np.all(codes[:2] == 0)
-    nz = sigma > 0
-    with np.errstate(divide="ignore", invalid="ignore"):
-        r = (xv[nz] / sigma[nz, None]).astype(np.float32)
-    np.testing.assert_array_equal(codes[nz], e4m3_nearest_bruteforce(r.ravel()).reshape(r.shape))
-    # the largest magnitude of a row lands on 448 (up to the rounding of sigma)
-    top = np.abs(xv).argmax(axis=1)
-    assert np.all((codes[nz, top[nz]] & 0x7F) >= 0x7D)
+    for r in range(len(bits)):
+        if sigma[r] == 0:
+            continue
+        want = [exact_nearest_e4m3(float(v), float(sigma[r])) for v in xv[r]]
+        np.testing.assert_array_equal(codes[r], np.array(want, np.uint8), err_msg=f"row {r}")
+
+
+def test_quant_index_fp8_rounds_the_exact_quotient_not_the_binary32_one():
+    """On the double-rounding rows the oracle's codes differ from rounding
+    the binary32 quotient (torch's RNE cast of numpy's binary32 division) in
+    some channels, and agree with the exact brute force in all of them."""
+    bits = double_rounding_rows(20, seed=2)
+    codes, sigma = oracle.quant_index_fp8(bits)
+    xv = bits_to_f32(bits)
+    q32 = xv / sigma[:, None]                                      # numpy binary32 division (library)
+    via32 = torch.from_numpy(np.ascontiguousarray(q32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    via32 = np.where((via32 & 0x7F) == 0, 0, via32)
+    assert np.count_nonzero(via32 != codes) > 0
+    diff = np.argwhere(via32 != codes)
+    for r, c in diff[:200]:
+        assert codes[r, c] == exact_nearest_e4m3(float(xv[r, c]), float(sigma[r]))
 
 
 def test_quant_index_fp8_idempotent_on_grid_rows():
@@ -218,9 +313,9 @@ def test_quant_index_fp8_power_of_two_equivariance_and_error_bound():
     deq = np.where(codes >= 0x80, -ev[codes & 0x7F], ev[codes & 0x7F]) * sigma[:, None].astype(np.float64)
     r = np.abs(xv) / sigma[:, None]
     e = np.floor(np.log2(np.maximum(r, 2.0 ** -6)))
-    half_ulp = np.exp2(e - 4)                                     # half the E4M3 step at r (2^-10 below 2^-6)
-    bound = sigma[:, None] * (half_ulp + r * 2.0 ** -23)          # + the binary32 rounding of the quotient
-    assert np.all(np.abs(xv - deq) <= bound)
+    half_step = np.exp2(e - 4)                                    # half the E4M3 step at r (2^-10 below 2^-6)
+    # one rounding of the exact quotient: within half a grid step (fp64 slack only)
+    assert np.all(np.abs(xv - deq) <= sigma[:, None] * half_step * (1 + 2.0 ** -40))
 
 
 # ------------------------------------------------------------------ codes
