@@ -5,7 +5,9 @@
 // The pool is the Full layer's top-C (ascending token indices, -1 padded, as
 // K3 emits it); the layer scores only those tokens with its own query.
 //
-// One CTA (512 threads) per query row.
+// One CTA (512 threads) per query row. A pool entry after the row's query
+// position (causal bound), past the sequence or with a bad page sets the status
+// word and is skipped.
 //   score   thread i takes pool entries i, i + 512, ...: the token's 64-byte
 //           indexer key (four 16-byte chunks of its page's core-matrix
 //           layout) and sigma; four fp32 dot products with the row's query
@@ -111,10 +113,13 @@ pool_topk_kernel(const PoolArgs A) {
     int T = A.seq_lens[b];
     pdl_wait();                                  // the pool is written by the previous kernel
     pdl_trigger();
-    if (T < 0 || T > A.max_pages * kPage) {
+    if (T < A.Sq || T > A.max_pages * kPage) {
         if (tid == 0) flag_status(kStatusBounds);
-        T = 0;                                   // no valid token
+        T = A.Sq - 1 - row % A.Sq;               // no valid token for any query of the row
     }
+    // Query j of the sequence sits at position T - Sq + j and is causal: a
+    // pool entry after it is out of range.
+    const int lim = T - A.Sq + row % A.Sq + 1;
     __syncthreads();
 
     // ---------------- score every pool entry
@@ -124,7 +129,7 @@ pool_topk_kernel(const PoolArgs A) {
         const int t = prow[i];
         uint32_t key = 0u;
         if (t >= 0) {
-            const int64_t page = t < T ? A.page_table[static_cast<int64_t>(b) * A.max_pages + (t >> 6)] : -1;
+            const int64_t page = t < lim ? A.page_table[static_cast<int64_t>(b) * A.max_pages + (t >> 6)] : -1;
             if (i > 0 && prow[i - 1] >= t) flag_status(kStatusBounds);      // pool must ascend
             if (page >= 0 && page < A.num_pages) {
                 const int r = t & 63;

@@ -100,17 +100,51 @@ inline cudaError_t launch_quant_kv_fp4(const void *x, int64_t n_tok, const int32
 // section 3: the KV owner hands "indexer K / scale" to its consumer layers;
 // page "DeepSeek 首次公开 V4.1-Flash 技术报告…" (neodrop.ai), architecture
 // part 2: the indexer scores with FP8 operands. The pages give no scale rule;
-// the one taken is sigma = amax / 448 and code = RNE-satfinite E4M3 of
-// x / sigma, both divisions IEEE binary32, canonical +0, all codes 0 (and
-// sigma 0) for an all-zero row.
+// the one taken is sigma = binary32 nearest to amax / 448 and code = the E4M3FN
+// value nearest to the exact quotient x / sigma (one rounding, ties to even,
+// saturating, canonical +0), all codes 0 (and sigma 0) for an all-zero row.
 //
-// Eight threads per row, each with one 16-byte load of 8 channels: the row
-// maximum by three shuffles inside the 8-lane group, eight correctly rounded
-// divisions, four paired hardware conversions, one 8-byte store. A warp moves 512 B in
-// and 272 B out per pass, coalesced. HBM-bound: 128 B read + 68 B written per
-// row.
+// Exact rounding without a division per channel: p = RN(|x| * RN(1 / sigma))
+// is within 2 binary32 ulps of the exact quotient, so the hardware RNE
+// conversion of p can differ from the exact decision only when an E4M3
+// midpoint lies within those ulps of p. Such channels (the low 20 bits of p
+// within 3 of a midpoint's pattern, or p in the E4M3 subnormal range) take a
+// fix-up that decides the side by the sign of fma(midpoint, sigma, -|x|): the
+// product is exact in the fma and a single rounding keeps the sign. Rows with
+// sigma < 2^-100 are first scaled by 2^64 (exact), so no product of the
+// fix-up underflows.
+//
+// Eight threads per row, each with 8 channels; a thread runs kIdxQuantRows
+// rows per pass with all their 16-byte loads issued first, so more bytes are
+// in flight per warp. HBM-bound: 128 B read + 68 B written per row.
 constexpr int kIdxQuantThreads = 256;
-constexpr int kIdxQuantRowsPerBlock = kIdxQuantThreads / 8;
+constexpr int kIdxQuantRows = 4;                                   // rows per thread per pass
+constexpr int kIdxQuantRowsPerBlock = kIdxQuantThreads / 8 * kIdxQuantRows;
+
+// E4M3FN magnitude code of the exact quotient a / s (a >= 0, s > 0 binary32,
+// s >= 2^-100), given p = a * RN(1 / s) rounded once.
+__device__ __forceinline__ uint32_t e4m3_quotient_fixup(float a, float s, float p) {
+    if (p >= 448.0f) return 0x7Eu;
+    if (p < 0.015625f) {                                           // E4M3 subnormal range: steps of 2^-9
+        const float n = floorf(p * 512.0f);
+        const float d = __fmaf_rn((n + 0.5f) * 0.001953125f, s, -a);
+        const uint32_t k = static_cast<uint32_t>(n);
+        return d > 0.0f ? k : d < 0.0f ? k + 1u : k + (k & 1u);    // codes 0..8 are k itself
+    }
+    const uint32_t lo = __float_as_uint(p) & ~0xFFFFFu;            // grid value just below the midpoint
+    const float d = __fmaf_rn(__uint_as_float(lo | 0x80000u), s, -a);
+    const uint32_t clo = (((lo >> 23) - 120u) << 3) | ((lo >> 20) & 7u);   // exponent bias 127 -> 7
+    const uint32_t chi = min(clo + 1u, 0x7Eu);
+    return d > 0.0f ? clo : d < 0.0f ? chi : ((clo & 1u) ? chi : clo);
+}
+
+// Whether RNE(p) may differ from the exact decision (see above).
+__device__ __forceinline__ bool e4m3_quotient_near(float p) {
+    const uint32_t b = __float_as_uint(p);
+    const bool mid = ((b - 0x7FFFDu) & 0xFFFFFu) <= 6u;            // within 3 ulps of an E4M3 midpoint
+    const bool sub = b - 0x3A000000u < 0x3C800000u - 0x3A000000u;  // p in [2^-11, 2^-6)
+    return mid || sub;
+}
 
 __global__ void __launch_bounds__(kIdxQuantThreads)
 quant_index_fp8_kernel(const uint4 *__restrict__ x, int64_t n_rows, uint2 *__restrict__ codes,
@@ -119,36 +153,68 @@ quant_index_fp8_kernel(const uint4 *__restrict__ x, int64_t n_rows, uint2 *__res
     pdl_trigger();
     const int lane = threadIdx.x & 31, part = threadIdx.x & 7;
     const unsigned gmask = 0xffu << (lane & 24);        // the 8 lanes of this row
-    for (int64_t row = static_cast<int64_t>(blockIdx.x) * kIdxQuantRowsPerBlock + (threadIdx.x >> 3); row < n_rows;
-         row += static_cast<int64_t>(gridDim.x) * kIdxQuantRowsPerBlock) {
-        const uint4 v = x[row * 8 + part];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        float f[8];
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * kIdxQuantRowsPerBlock;
+    for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * kIdxQuantRowsPerBlock + (threadIdx.x >> 3);
+         row0 < n_rows; row0 += stride) {
+        uint4 v[kIdxQuantRows];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            f[2 * i] = __uint_as_float(w[i] << 16);
-            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        for (int r = 0; r < kIdxQuantRows; ++r) {
+            const int64_t row = row0 + r * (kIdxQuantThreads / 8);
+            v[r] = row < n_rows ? x[row * 8 + part] : make_uint4(0u, 0u, 0u, 0u);
         }
-        float amax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+        for (int r = 0; r < kIdxQuantRows; ++r) {
+            const int64_t row = row0 + r * (kIdxQuantThreads / 8);
+            const uint32_t w[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+            float f[8];
 #pragma unroll
-        for (int off = 1; off < 8; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, off));
-        const float sg = __fdiv_rn(amax, 448.0f);
-        uint32_t packed[2] = {0u, 0u};
-        if (sg != 0.0f) {
+            for (int i = 0; i < 4; ++i) {
+                f[2 * i] = __uint_as_float(w[i] << 16);
+                f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+            }
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+            for (int off = 1; off < 8; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, off));
+            const float sg = __fdiv_rn(amax, 448.0f);
+            // Scaled domain for tiny sigma (exact power-of-two scaling).
+            const float scl = sg < 0x1p-100f ? 0x1p64f : 1.0f;
+            const float s2 = sg * scl;
+            const float inv = __frcp_rn(s2);
+            float a[8], p[8];
+            uint32_t near = 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                a[i] = fabsf(f[i]) * scl;
+                p[i] = a[i] * inv;
+                near |= e4m3_quotient_near(p[i]) ? (1u << i) : 0u;
+            }
+            uint32_t mag[8];
 #pragma unroll
             for (int i = 0; i < 8; i += 2) {
-                // one paired conversion: low byte from channel i, high byte from i + 1
-                uint32_t c2 = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(f[i], sg), __fdiv_rn(f[i + 1], sg)),
-                                                       __NV_SATFINITE, __NV_E4M3);
-                if ((c2 & 0x7fu) == 0u) c2 &= 0xff00u;             // canonical +0
-                if ((c2 & 0x7f00u) == 0u) c2 &= 0x00ffu;
-                packed[i >> 2] |= c2 << (8 * (i & 3));
+                const uint32_t c2 = __nv_cvt_float2_to_fp8x2(make_float2(p[i], p[i + 1]), __NV_SATFINITE, __NV_E4M3);
+                mag[i] = c2 & 0x7Fu;
+                mag[i + 1] = (c2 >> 8) & 0x7Fu;
+            }
+            if (__any_sync(0xffffffffu, near != 0u)) {                 // rare: exact fix-up of close calls
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (near & (1u << i)) mag[i] = e4m3_quotient_fixup(a[i], s2, p[i]);
+            }
+            uint32_t packed[2] = {0u, 0u};
+            if (sg != 0.0f) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t c = mag[i] | ((mag[i] != 0u && f[i] < 0.0f) ? 0x80u : 0u);   // canonical +0
+                    packed[i >> 2] |= c << (8 * (i & 3));
+                }
+            }
+            if (row < n_rows) {
+                codes[row * 8 + part] = make_uint2(packed[0], packed[1]);
+                if (part == 0) sigma[row] = sg;
             }
         }
-        codes[row * 8 + part] = make_uint2(packed[0], packed[1]);
-        if (part == 0) sigma[row] = sg;
     }
 }
 

@@ -200,6 +200,14 @@ def indexer_topk(q_idx: torch.Tensor, w: torch.Tensor, cache: PagedCache, page_t
     return out
 
 
+def indexer_scores_in_workspace(ws: torch.Tensor, B: int, Sq: int, max_pages: int) -> torch.Tensor:
+    """The fp32 scores a completed csa2_indexer_topk call leaves at the start
+    of its workspace, as a view [B, Sq, 64 * max_pages] (csa2.h: entries after
+    a query's position are unspecified)."""
+    n = B * Sq * PAGE * max_pages
+    return ws[:4 * n].view(torch.float32).view(B, Sq, PAGE * max_pages)
+
+
 def indexer_pool_topk(q_idx: torch.Tensor, w: torch.Tensor, cache: PagedCache, page_table: torch.Tensor,
                       seq_lens: torch.Tensor, pool: torch.Tensor, k: int,
                       out: Optional[torch.Tensor] = None) -> torch.Tensor:

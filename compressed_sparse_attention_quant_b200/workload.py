@@ -13,13 +13,14 @@ from .group import LayerGroup
 
 
 class DeviceWorkload:
-    def __init__(self, wl: inputs.Workload, device="cuda"):
+    def __init__(self, wl: inputs.Workload, device="cuda", pool_size=None):
         self.wl = wl
         self.device = device
         B, Sq = wl.batch, wl.q_tokens
         self.page_table = inputs.page_table(wl, device)
         self.seq_lens = inputs.seq_lens(wl, device)
-        self.group = LayerGroup(wl.modes, B, Sq, wl.pages_per_seq, B * wl.pages_per_seq, wl.top_k, device)
+        self.group = LayerGroup(wl.modes, B, Sq, wl.pages_per_seq, B * wl.pages_per_seq, wl.top_k, device,
+                                pool_size=pool_size)
         lens = wl.lens()
         # Bulk build: positions [0, len_b - Sq) of each owner's cache.
         for owner, cache in self.group.caches.items():

@@ -136,9 +136,10 @@ csa2_status csa2_quant_kv_fp4(const void *x_bf16, int64_t n_tok, int dim,
  * the indexer scores with FP8 operands).
  *
  * For each of n_rows rows of 64 bf16 channels:
- *     sigma[r]    = amax_r / 448                 (IEEE binary32 division)
- *     codes[r][c] = E4M3FN(x[r][c] / sigma[r])   (binary32 division, then round
- *                   to nearest even, saturating at +-448, canonical +0)
+ *     sigma[r]    = the binary32 value nearest to amax_r / 448
+ *     codes[r][c] = the E4M3FN value nearest to the exact quotient
+ *                   x[r][c] / sigma[r] (one rounding, ties to even mantissa,
+ *                   saturating at +-448, canonical +0)
  * An all-zero row gives sigma = 0 and zero codes. Inputs must be finite. The
  * pages print no scale rule; this is the plainest one (the row maximum lands
  * on the top E4M3 value). Keys: codes and sigma are the kidx_in and
@@ -180,7 +181,11 @@ csa2_status csa2_quant_indexer_fp8(const void *x_bf16, int64_t n_rows, int dim,
  *   out_idx     device int32 [B][Sq][k]
  *   ws          device workspace of at least csa2_indexer_topk_workspace_bytes()
  *               bytes, 256-byte aligned; contents need no initialisation and
- *               are clobbered.
+ *               are clobbered. When the call's work has completed on the
+ *               stream, its first B * Sq * 64 * max_pages floats hold the
+ *               scores as float [B * Sq][64 * max_pages]: entry (b * Sq + j, t)
+ *               is s_t as computed (fp32) for every t <= pos; other entries
+ *               are unspecified.
  *
  * Limits (else CSA2_ERR_UNSUPPORTED): 4 indexer heads x 64 channels,
  * Sq <= 4, B * Sq <= 65535, 64 * max_pages <= 2^30, cache->num_pages <=
@@ -210,7 +215,8 @@ csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq,
  *
  *   q_idx, w, cache, page_table, seq_lens, max_pages: as csa2_indexer_topk
  *   pool        device int32 [B][Sq][pool_size]: token indices in ascending
- *               order, -1 entries skipped; an entry >= seq_lens[b], a bad
+ *               order, -1 entries skipped; an entry after the query's
+ *               position seq_lens[b] - Sq + j (causal bound), a bad
  *               page-table entry or a descending pair sets
  *               CSA2_ERR_DEVICE_BOUNDS (the entry is skipped)
  *   pool_size   1 <= pool_size <= 32768 (CSA2_ERR_UNSUPPORTED above)

@@ -4,6 +4,7 @@ import pytest
 import torch
 
 import oracle
+from fp8_cases import double_rounding_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -132,7 +133,9 @@ def test_quant_out_of_range_slot_sets_device_status(lib):
 def _index_rows(rng, n):
     """Wide-magnitude rows plus the rows where a rounding decision is close:
     zero rows, bf16 subnormals, near the bf16 maximum, E4M3 midpoints (ties)
-    and their bf16 neighbours under sigma = 1."""
+    and their bf16 neighbours under sigma = 1, and rows whose binary32
+    quotient x / sigma lands exactly on an E4M3 midpoint that the exact
+    quotient misses."""
     x = rng.standard_normal((n, 64)) * np.exp2(rng.integers(-60, 60, (n, 1)))
     x[0] = 0.0
     x[1] = -0.0
@@ -157,7 +160,9 @@ def _index_rows(rng, n):
     up, down = nb.copy(), nb.copy()
     up[:, 1:] += (nb[:, 1:] & 0x7FFF) != 0
     down[:, 1:] -= (nb[:, 1:] & 0x7FFF) != 0
-    return np.concatenate([bits, up, down])
+    special = 5 + len(rows)
+    # the close-call rows first, so that a caller taking the first n rows keeps them
+    return np.concatenate([bits[:special], up, down, double_rounding_rows(40, seed=n), bits[special:]])
 
 
 @pytest.mark.parametrize("n", [1, 37, 75813])

@@ -55,6 +55,7 @@ import torch.nn.functional as F
 import oracle
 from compressed_sparse_attention_quant_b200 import inputs
 from conftest import golden, read_kv_fixture
+from fp8_cases import double_rounding_rows
 
 CONST = read_kv_fixture("pages_constants.txt")
 
@@ -200,35 +201,6 @@ def binary32_nearest(q: Fraction) -> np.float32:
     cands = [np.nextafter(c, np.float32(0)), c, np.nextafter(c, np.float32(np.inf))]
     best = min(cands, key=lambda f: (abs(Fraction(float(f)) - q), int(np.array(f).view(np.uint32)) & 1))
     return np.float32(best)
-
-
-def double_rounding_rows(n_rows: int, seed: int) -> np.ndarray:
-    """bf16 rows (as bits) whose row maximum fixes sigma and whose other
-    channels x make the binary32 quotient RN(x / sigma) land exactly on an
-    E4M3 midpoint while the exact quotient does not: the inputs on which
-    rounding the exact quotient and rounding the binary32 quotient differ.
-    Found by a vectorised search over every positive bf16 value."""
-    ev = e4m3_finite_values()[:127]
-    mids = np.unique(((ev[:-1] + ev[1:]) / 2).astype(np.float32))
-    _, vals = all_finite_bf16_bits()
-    pos = vals[vals > 0].astype(np.float32)
-    rng = np.random.default_rng(seed)
-    rows = []
-    while len(rows) < n_rows:
-        amax = np.float32(rng.choice(pos[(pos > 1e-30) & (pos < 1e30)]))
-        sg = amax / np.float32(448.0)
-        xs = pos[pos < amax]
-        q = xs / sg
-        hit = xs[np.isin(q, mids)]
-        hit = [x for x in hit if Fraction(float(x)) / Fraction(float(sg)) != Fraction(float(x / sg))]
-        if not hit:
-            continue
-        take = np.array(hit[:63], np.float32)
-        row = np.zeros(64, np.float32)
-        row[0] = amax
-        row[1:1 + len(take)] = take * np.where(np.arange(len(take)) % 2 == 0, 1, -1)
-        rows.append(row)
-    return bf16_rows(np.array(rows))
 
 
 def test_quant_index_fp8_sigma_is_the_nearest_binary32():
