@@ -205,14 +205,19 @@ class OracleArm:
                 o_.sparse_attn(q[j], codes, scales, idx, swa[rows], scale)
         return time.perf_counter() - t0
 
-    def describe(self, n_timed: int) -> str:
+    def describe(self, n_timed: int, threads: int) -> str:
         wl = self.wl
         return (f"{n_timed} sequence-steps over sequences {self.seqs} of {wl.batch}: "
                 f"{wl.q_tokens} query token(s) x {len(wl.modes)} layer(s), context {wl.lens()[0]}, "
-                f"top-k {wl.top_k}; single-threaded fp64 oracle; cache quantization untimed")
+                f"top-k {wl.top_k}; fp64 oracle on {threads} host thread(s); cache quantization untimed")
 
 
-def cpu_baseline(wl: inputs.Workload, n_seqs: int, budget_s: float) -> dict:
+def cpu_baseline(wl: inputs.Workload, n_seqs: int, budget_s: float, threads: int) -> dict:
+    """The oracle (its OpenMP build: bit-identical results, independent outer
+    loops on `threads` host cores) on a bounded sample of the workload."""
+    import oracle
+    oracle.use_all_cores(True)
+    oracle.set_threads(threads)
     arm = OracleArm(wl, n_seqs)
     arm.prepare()
     spent, n = 0.0, 0
@@ -220,13 +225,17 @@ def cpu_baseline(wl: inputs.Workload, n_seqs: int, budget_s: float) -> dict:
         spent += arm.step(arm.seqs[n % len(arm.seqs)])
         n += 1
     tok = n * wl.q_tokens
-    return {"value": tok / spent, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": arm.describe(n)}
+    return {"value": tok / spent, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": arm.describe(n, oracle.threads())}
 
 
 def run_reference(args, wl):
     rank = int(os.environ.get("RANK", "0"))
     if not replicas.reports(rank):
         return                      # the oracle arm runs on rank 0 only
+    import oracle
+    oracle.use_all_cores(True)      # the same oracle source, on every host core
+    oracle.set_threads(oracle.host_cores())
     arm = OracleArm(wl, args.ref_seqs)
     arm.prepare()
     times = []
@@ -236,6 +245,7 @@ def run_reference(args, wl):
             times.append(t)
     per_seq = sum(times) / len(times)
     value = wl.q_tokens / per_seq
+    desc = arm.describe(len(times), oracle.threads())
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": per_seq * 1e3, "higher_is_better": True,
@@ -243,8 +253,8 @@ def run_reference(args, wl):
             "config": {"workload": wl.name, "batch": wl.batch, "q_tokens": wl.q_tokens,
                        "context": wl.context, "top_k": wl.top_k, "modes": "".join(wl.modes),
                        "step": "one sequence of the batch per step (bounded sample)"},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": arm.describe(len(times))},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+                             "sample": desc},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -286,6 +296,100 @@ def pool_leg(args, wl, dw, lib, flush, stream, hbm) -> dict:
                 "input": "pool = the Full layer's top-4k; query = the Full query rolled by one channel"}
     except Exception as e:                                  # the leg is optional: report, do not fail
         return {"kernel": "csa2_indexer_pool_topk", "error": f"{type(e).__name__}: {e}"[:300]}
+
+
+def time_steps(dw, args, flush, stream):
+    """Mean device time (ms) of one whole step of a DeviceWorkload: W untimed
+    warm-up steps, then K steps, each preceded by an untimed L2 flush, CUDA
+    events on the launching stream around each step."""
+    for _ in range(args.warmup):
+        flush.zero_()
+        dw.step()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(args.steps):
+        if not args.no_flush:
+            flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        dw.step()
+        e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs) / args.steps
+
+
+def other_workload(args, name, dev, flush, stream, hbm, with_cpu: bool) -> dict:
+    """Step throughput and roofline fractions of another benchmark workload
+    (its own inputs resident in HBM), with the oracle timed on a bounded
+    sample on every host core. Errors are reported, never raised."""
+    from compressed_sparse_attention_quant_b200 import lib, workload
+    try:
+        wl = inputs.WORKLOADS[name]
+        dw = workload.DeviceWorkload(wl, dev)
+        acct = dw.algorithmic_bytes()
+        ms = time_steps(dw, args, flush, stream)
+        gbs = acct["total"] / (ms * 1e-3) / 1e9
+        out = {"value": wl.batch * wl.q_tokens / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+               "config": {"batch": wl.batch, "q_tokens": wl.q_tokens, "context": wl.context, "top_k": wl.top_k,
+                          "modes": "".join(wl.modes)},
+               "algorithmic_bytes_per_step": acct["total"], "step_hbm_gbs": gbs,
+               "step_frac_of_8tbs": gbs / NOMINAL_HBM_GBS, "step_frac_of_measured_copy": gbs / hbm,
+               "attention_tflops_per_step": attention_flops(wl) / 1e12,
+               "device_status": lib.status_string(lib.last_device_error())}
+        del dw
+        torch.cuda.empty_cache()
+        if with_cpu:
+            import oracle
+            out["cpu_baseline"] = cpu_baseline(wl, 1, args.cpu_budget_other, oracle.host_cores())
+        return out
+    except Exception as e:                                  # optional leg: report, do not fail
+        return {"error": f"{type(e).__name__}: {e}"[:300]}
+
+
+def attention_flops(wl) -> float:
+    """Algorithmic attention FLOPs of one step: QK and PV over k + 128 keys,
+    16 heads x 576 channels, per query token and layer."""
+    return 4.0 * 16 * 576 * (wl.top_k + 128) * wl.batch * wl.q_tokens * len(wl.modes)
+
+
+def bulk_quant_leg(args, wl, dw, stream, hbm) -> dict:
+    """csa2_quant_kv_fp4 as a bulk cache build: B x T tokens (the whole
+    context of the workload, with their indexer keys), rewritten into the
+    same slots. Events around each launch; inputs > L2."""
+    from compressed_sparse_attention_quant_b200 import lib
+    try:
+        n = wl.batch * wl.context
+        x = torch.randn(n, lib.DIM, device=stream.device, dtype=torch.bfloat16,
+                        generator=torch.Generator(device=stream.device).manual_seed(7))
+        kid = torch.randint(0, 120, (n, lib.IDX_DIM), device=stream.device, dtype=torch.uint8)
+        ks = torch.ones(n, device=stream.device)
+        pos = torch.arange(wl.context, device=stream.device)
+        slots = torch.cat([lib.slot_mapping(dw.page_table, b, pos) for b in range(wl.batch)])
+        cache = lib.PagedCache(dw.group.num_pages, stream.device)
+        for _ in range(2):
+            lib.quant_kv_fp4(x, slots, cache, kid, ks)
+        torch.cuda.synchronize()
+        evs = []
+        for _ in range(args.steps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            lib.quant_kv_fp4(x, slots, cache, kid, ks)
+            e1.record(stream)
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+        per_tok = 576 * 2 + 4 + 64 + 4 + 288 + 36 + 64 + 4       # bf16 in, slot, key + sigma in; FP4 + scales + key + sigma out
+        ach = n * per_tok / (ms * 1e-3) / 1e9
+        del x, kid, ks, slots, cache
+        torch.cuda.empty_cache()
+        return {"kernel": "csa2_quant_kv_fp4", "tokens": n, "bytes_per_token": per_tok, "ms_per_launch": ms,
+                "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm, "frac_of_8tbs": ach / NOMINAL_HBM_GBS,
+                "input": "B x T tokens of N(0,1) bf16 + indexer keys, rewritten into the workload's slots"}
+    except Exception as e:
+        return {"kernel": "csa2_quant_kv_fp4", "error": f"{type(e).__name__}: {e}"[:300]}
 
 
 def run_gpu(args, wl):
@@ -498,10 +602,19 @@ def run_gpu(args, wl):
     clocks = clk.summary()
     if clocks:
         line["clocks"] = clocks
+    line["attention_tflops_per_step"] = attention_flops(wl) / 1e12
     if world == 1:
         line["indexer_pool_topk"] = pool_leg(args, wl, dw, lib, flush, stream, hbm)
+        line["kv_quant_bulk"] = bulk_quant_leg(args, wl, dw, stream, hbm)
+    if world == 1 and not args.no_other_workloads:
+        del dw, g
+        torch.cuda.empty_cache()
+        line["workloads"] = {name: other_workload(args, name, dev, flush, stream, hbm, not args.no_cpu_baseline)
+                             for name in inputs.WORKLOADS if name != wl.name}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, args.ref_seqs, args.cpu_budget)
+        import oracle
+        line["cpu_baseline"] = cpu_baseline(wl, args.ref_seqs, args.cpu_budget, oracle.host_cores())
+        line["cpu_baseline_1core"] = cpu_baseline(wl, args.ref_seqs, args.cpu_budget / 2, 1)
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -559,6 +672,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work (cpu_baseline)")
     ap.add_argument("--ref-seqs", type=int, default=2, help="sequences the oracle arm prepares")
     ap.add_argument("--dry-run", action="store_true", help="launch path only (process group, max over ranks)")
+    ap.add_argument("--no-other-workloads", action="store_true", help="time only --workload")
+    ap.add_argument("--cpu-budget-other", type=float, default=3.0,
+                    help="seconds of oracle work per other workload")
     args = ap.parse_args()
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
         sys.exit(relaunch_under_torchrun(args))

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cstring>
 #include <algorithm>
+#include <mutex>
 
 #include "attn.cuh"
 #include "common.cuh"
@@ -22,12 +23,16 @@ namespace {
 constexpr int kMaxDevices = 64;
 
 struct DeviceInfo {
-    bool ready = false;
+    std::atomic<bool> ready{false};
     int sm_count = 0;
     int att_ctas_per_sm = 0;
+    int q8_blocks = 0;            // resident blocks of the FP8 quantiser (whole device)
     int tk_max_cluster = 1;       // largest power-of-two top-k cluster the device can co-schedule
 };
 DeviceInfo g_dev[kMaxDevices];
+// Serialises the one-time per-device set-up (attributes, occupancy, scratch
+// address) when several host threads make their first call at once.
+std::mutex g_init_mutex;
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -39,7 +44,12 @@ cudaError_t device_info(DeviceInfo **out) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     DeviceInfo &d = g_dev[dev];
-    if (!d.ready) {
+    if (d.ready.load(std::memory_order_acquire)) {
+        *out = &d;
+        return cudaSuccess;
+    }
+    std::lock_guard<std::mutex> lock(g_init_mutex);
+    if (!d.ready.load(std::memory_order_relaxed)) {
         e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(indexer_score_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -69,7 +79,8 @@ cudaError_t device_info(DeviceInfo **out) {
                                  reinterpret_cast<const void *>(sparse_attn_kernel),
                                  reinterpret_cast<const void *>(attn_merge_kernel),
                                  reinterpret_cast<const void *>(quant_index_fp8_kernel),
-                                 reinterpret_cast<const void *>(pool_topk_kernel)};
+                                 reinterpret_cast<const void *>(pool_topk_kernel),
+                                 reinterpret_cast<const void *>(lse_merge_kernel)};
         for (const void *kf : kernels) {
             e = cudaFuncSetAttribute(kf, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
             if (e != cudaSuccess) return e;
@@ -79,6 +90,10 @@ cudaError_t device_info(DeviceInfo **out) {
                                                           kAttSmemBytes);
         if (e != cudaSuccess) return e;
         if (d.att_ctas_per_sm < 1) d.att_ctas_per_sm = 1;
+        int q8 = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&q8, quant_index_fp8_kernel, kIdxQuantThreads, 0);
+        if (e != cudaSuccess) return e;
+        d.q8_blocks = std::max(1, q8) * d.sm_count;
         // Largest top-k cluster (<= 16 CTAs) that fits on the device at once.
         d.tk_max_cluster = 1;
         for (int cs = kTkMaxCluster; cs > 1; cs /= 2) {
@@ -101,7 +116,7 @@ cudaError_t device_info(DeviceInfo **out) {
             }
             (void)cudaGetLastError();                      // clear a refusal of this size
         }
-        d.ready = true;
+        d.ready.store(true, std::memory_order_release);
     }
     *out = &d;
     return cudaSuccess;
@@ -125,38 +140,29 @@ IdxLayout idx_layout(int B, int Sq, int max_pages, int k) {
     return L;
 }
 
-// ---------------------------------------------------------------- attention splits
-struct AttSplit {
-    int n_splits;
-    int tiles_per_split;
+// ---------------------------------------------------------------- attention work plan
+struct AttPlan {
+    int n_win;           // window steps per query row (8, or 0 without a window)
+    int n_st;            // steps of 16 keys per query row
+    int64_t total;       // steps over all rows
+    int grid;            // CTAs (each a contiguous range of steps)
 };
 
-// Split the (k + 128)-key list of each query row into S contiguous tile runs
-// so that R * S CTAs fill the machine: minimise waves x tiles per CTA, with a
-// small charge per split for writing and merging its partial.
-AttSplit att_split(int R, int k, int slots) {
-    const int n_tiles = (k + kWindow + kAttTile - 1) / kAttTile;
-    const int s_min = (n_tiles + kMaxTilesPerSplit - 1) / kMaxTilesPerSplit;
-    AttSplit best{s_min, (n_tiles + s_min - 1) / s_min};
-    double best_cost = 1e30;
-    for (int s = s_min; s <= n_tiles && s <= s_min + 64; ++s) {
-        const int tps = (n_tiles + s - 1) / s;
-        const int s_eff = (n_tiles + tps - 1) / tps;
-        const int64_t ctas = static_cast<int64_t>(R) * s_eff;
-        const int64_t waves = (ctas + slots - 1) / slots;
-        const double cost = static_cast<double>(waves) * tps + (s_eff > 1 ? 0.25 * s_eff : 0.0);
-        if (cost < best_cost - 1e-9) {
-            best_cost = cost;
-            best = AttSplit{s_eff, tps};
-        }
-    }
-    return best;
+// At most one wave of CTAs, each with at least 4 steps of work.
+AttPlan att_plan(int R, int k, int slots, bool window = true) {
+    AttPlan pl;
+    pl.n_win = window ? kAttWinSteps : 0;
+    pl.n_st = pl.n_win + (k + kAttStepKeys - 1) / kAttStepKeys;
+    pl.total = static_cast<int64_t>(R) * pl.n_st;
+    pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(slots, pl.total / 4)));
+    return pl;
 }
 
-size_t att_ws_bytes(int R, const AttSplit &sp) {
-    if (sp.n_splits <= 1) return 0;
-    const size_t po = round_up(static_cast<size_t>(R) * sp.n_splits * kHeads * kDim * 4, 256);
-    const size_t pm = round_up(static_cast<size_t>(R) * sp.n_splits * kHeads * 8, 256);
+// Partials: two per CTA (the first and the last row segment of its range).
+size_t att_ws_bytes(const AttPlan &pl) {
+    if (pl.grid <= 1) return 0;
+    const size_t po = round_up(static_cast<size_t>(2) * pl.grid * kHeads * kDim * 4, 256);
+    const size_t pm = round_up(static_cast<size_t>(2) * pl.grid * kHeads * 8, 256);
     return po + pm;
 }
 
@@ -200,7 +206,7 @@ csa2_status csa2_quant_indexer_fp8(const void *x_bf16, int64_t n_rows, int dim, 
     if (n_rows > (INT64_C(1) << 40)) return CSA2_ERR_INVALID_ARG;
     DeviceInfo *dev = nullptr;
     if (device_info(&dev) != cudaSuccess) return CSA2_ERR_CUDA;
-    return cuda_status(launch_quant_index_fp8(x_bf16, n_rows, codes_e4m3, sigma, dev->sm_count,
+    return cuda_status(launch_quant_index_fp8(x_bf16, n_rows, codes_e4m3, sigma, dev->q8_blocks,
                                               static_cast<cudaStream_t>(stream)));
 }
 
@@ -209,10 +215,17 @@ size_t csa2_indexer_topk_workspace_bytes(int B, int Sq, int max_pages, int k) {
     return idx_layout(B, Sq, max_pages, k).total;
 }
 
-csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq, int idx_heads, int idx_dim,
+}  // extern "C"
+
+namespace csa2 {
+namespace {
+
+// csa2_indexer_topk, with the selected entries' scores written to out_scores
+// when it is not null.
+csa2_status indexer_topk_impl(const void *q_idx, const float *w, int B, int Sq, int idx_heads, int idx_dim,
                               const csa2_paged_cache *cache, const int32_t *page_table, int max_pages,
-                              const int32_t *seq_lens, int k, int32_t *out_idx, void *ws, size_t ws_bytes,
-                              void *stream) {
+                              const int32_t *seq_lens, int k, int32_t *out_idx, float *out_scores, void *ws,
+                              size_t ws_bytes, void *stream) {
     if (idx_heads != kIdxHeads || idx_dim != kIdxDim) return CSA2_ERR_UNSUPPORTED;
     if (B <= 0 || B > 65535 || Sq <= 0 || max_pages <= 0 || k <= 0 || k > 65536 || !cache_ok(cache))
         return CSA2_ERR_INVALID_ARG;
@@ -223,7 +236,8 @@ csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq, 
     if (!q_idx || !w || !page_table || !seq_lens || !out_idx || !cache->kidx || !cache->kidx_scale)
         return CSA2_ERR_INVALID_ARG;
     if (!aligned(q_idx, 16) || !aligned(w, 16) || !aligned(cache->kidx, 16) || !aligned(cache->kidx_scale, 16) ||
-        !aligned(page_table, 4) || !aligned(seq_lens, 4) || !aligned(out_idx, 4))
+        !aligned(page_table, 4) || !aligned(seq_lens, 4) || !aligned(out_idx, 4) ||
+        (out_scores && !aligned(out_scores, 4)))
         return CSA2_ERR_ALIGNMENT;
     const IdxLayout L = idx_layout(B, Sq, max_pages, k);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return CSA2_ERR_WORKSPACE;
@@ -273,8 +287,30 @@ csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq, 
         C *= 2;
     e = launch_pdl_cluster(topk_cluster_kernel, dim3(static_cast<unsigned>(R * C)), dim3(kTkThreads), sizeof(TkSmem),
                            st, C, static_cast<const float *>(scores), L.t_cap, static_cast<const uint32_t *>(hist),
-                           seq_lens, Sq, max_pages, k, out_idx);
+                           seq_lens, Sq, max_pages, k, out_idx, out_scores);
     return cuda_status(e);
+}
+
+}  // namespace
+}  // namespace csa2
+
+extern "C" {
+
+csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq, int idx_heads, int idx_dim,
+                              const csa2_paged_cache *cache, const int32_t *page_table, int max_pages,
+                              const int32_t *seq_lens, int k, int32_t *out_idx, void *ws, size_t ws_bytes,
+                              void *stream) {
+    return indexer_topk_impl(q_idx, w, B, Sq, idx_heads, idx_dim, cache, page_table, max_pages, seq_lens, k, out_idx,
+                             nullptr, ws, ws_bytes, stream);
+}
+
+csa2_status csa2_indexer_topk_scores(const void *q_idx, const float *w, int B, int Sq, int idx_heads, int idx_dim,
+                                     const csa2_paged_cache *cache, const int32_t *page_table, int max_pages,
+                                     const int32_t *seq_lens, int k, int32_t *out_idx, float *out_scores, void *ws,
+                                     size_t ws_bytes, void *stream) {
+    if (!out_scores) return CSA2_ERR_INVALID_ARG;
+    return indexer_topk_impl(q_idx, w, B, Sq, idx_heads, idx_dim, cache, page_table, max_pages, seq_lens, k, out_idx,
+                             out_scores, ws, ws_bytes, stream);
 }
 
 csa2_status csa2_indexer_pool_topk(const void *q_idx, const float *w, int B, int Sq, int idx_heads, int idx_dim,
@@ -306,17 +342,63 @@ csa2_status csa2_indexer_pool_topk(const void *q_idx, const float *w, int B, int
     A.Sq = Sq;
     A.pool = pool;
     A.C = pool_size;
+    A.seg = pool_size;
+    A.seg_stride = 0;
+    A.row_stride = pool_size;
+    A.given = nullptr;
     A.k = k;
     A.out = out_idx;
+    A.out_local = nullptr;
+    A.lo = 0;
+    A.hi = 0;
     return cuda_status(launch_pool_topk(A, B * Sq, static_cast<cudaStream_t>(stream)));
 }
 
+csa2_status csa2_topk_merge(const float *cand_scores, const int32_t *cand_idx, int n_shards, int R, int k_shard,
+                            int k, int32_t shard_lo, int32_t shard_hi, int32_t *out_idx, int32_t *out_local,
+                            void *stream) {
+    if (!cand_scores || !cand_idx || (!out_idx && !out_local) || n_shards <= 0 || R <= 0 || k_shard <= 0 || k <= 0)
+        return CSA2_ERR_INVALID_ARG;
+    if (R > 65535 || static_cast<int64_t>(n_shards) * k_shard > kPoolMax) return CSA2_ERR_UNSUPPORTED;
+    if (!aligned(cand_scores, 4) || !aligned(cand_idx, 4) || (out_idx && !aligned(out_idx, 4)) ||
+        (out_local && !aligned(out_local, 4)))
+        return CSA2_ERR_ALIGNMENT;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return CSA2_ERR_CUDA;
+    PoolArgs A = {};
+    A.Sq = 1;                                   // no sequence lengths in merge mode
+    A.max_pages = 1;
+    A.pool = cand_idx;
+    A.C = n_shards * k_shard;
+    A.seg = k_shard;
+    A.seg_stride = static_cast<int64_t>(R) * k_shard;
+    A.row_stride = k_shard;
+    A.given = cand_scores;
+    A.k = k;
+    A.out = out_idx;
+    A.out_local = out_local;
+    A.lo = shard_lo;
+    A.hi = shard_hi;
+    return cuda_status(launch_pool_topk(A, R, static_cast<cudaStream_t>(stream)));
+}
+
+csa2_status csa2_lse_merge(const float *o_parts, const float *lse_parts, int n_parts, int R, float *out, float *lse,
+                           void *stream) {
+    if (!o_parts || !lse_parts || !out || !lse || n_parts <= 0 || R <= 0) return CSA2_ERR_INVALID_ARG;
+    if (R > 65535) return CSA2_ERR_UNSUPPORTED;
+    if (!aligned(o_parts, 16) || !aligned(out, 16) || !aligned(lse_parts, 4) || !aligned(lse, 4))
+        return CSA2_ERR_ALIGNMENT;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return CSA2_ERR_CUDA;
+    return cuda_status(launch_pdl(lse_merge_kernel, dim3(R, kHeads / kMergeHeads), dim3(kMergeThreads), 0,
+                                  static_cast<cudaStream_t>(stream), o_parts, lse_parts, n_parts, R, out, lse));
+}
+
 size_t csa2_sparse_attn_workspace_bytes(int B, int Sq, int k) {
-    if (B <= 0 || Sq <= 0 || k < 0) return 0;
+    if (B <= 0 || Sq <= 0 || k < 0 || k > 65536 || static_cast<int64_t>(B) * Sq > 65535) return 0;
     DeviceInfo *dev = nullptr;
     if (device_info(&dev) != cudaSuccess) return 0;
-    const int R = B * Sq;
-    return att_ws_bytes(R, att_split(R, k, dev->sm_count * dev->att_ctas_per_sm));
+    return att_ws_bytes(att_plan(B * Sq, k, dev->sm_count * dev->att_ctas_per_sm));
 }
 
 csa2_status csa2_sparse_attn_decode(const void *q_bf16, int B, int Sq, int H, int D,
@@ -324,23 +406,23 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int B, int Sq, int H, in
                                     const int32_t *seq_lens, const int32_t *topk_idx, int k,
                                     const void *swa_bf16, int W, float softmax_scale, float *out, float *lse,
                                     void *ws, size_t ws_bytes, void *stream) {
-    if (H != kHeads || D != kDim || W != kWindow) return CSA2_ERR_UNSUPPORTED;
+    if (H != kHeads || D != kDim || (W != kWindow && W != 0)) return CSA2_ERR_UNSUPPORTED;
     if (B <= 0 || Sq <= 0 || k < 0 || k > 65536 || max_pages <= 0 || !cache_ok(cache) ||
-        !std::isfinite(softmax_scale))
+        !std::isfinite(softmax_scale) || (W == 0 && k == 0))
         return CSA2_ERR_INVALID_ARG;
     if (static_cast<int64_t>(B) * Sq > 65535) return CSA2_ERR_UNSUPPORTED;
-    if (!q_bf16 || !page_table || !seq_lens || (k > 0 && !topk_idx) || !swa_bf16 || !out || !lse ||
+    if (!q_bf16 || !page_table || !seq_lens || (k > 0 && !topk_idx) || (W > 0 && !swa_bf16) || !out || !lse ||
         !cache->kv_fp4 || !cache->kv_scale)
         return CSA2_ERR_INVALID_ARG;
-    if (!aligned(q_bf16, 16) || !aligned(swa_bf16, 16) || !aligned(cache->kv_fp4, 16) ||
-        !aligned(cache->kv_scale, 4) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(page_table, 4) ||
+    if (!aligned(q_bf16, 16) || (W > 0 && !aligned(swa_bf16, 16)) || !aligned(cache->kv_fp4, 16) ||
+        !aligned(cache->kv_scale, 16) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(page_table, 4) ||
         !aligned(seq_lens, 4) || (topk_idx && !aligned(topk_idx, 4)))
         return CSA2_ERR_ALIGNMENT;
     DeviceInfo *dev = nullptr;
     if (device_info(&dev) != cudaSuccess) return CSA2_ERR_CUDA;
     const int R = B * Sq;
-    const AttSplit sp = att_split(R, k, dev->sm_count * dev->att_ctas_per_sm);
-    const size_t need = att_ws_bytes(R, sp);
+    const AttPlan pl = att_plan(R, k, dev->sm_count * dev->att_ctas_per_sm, W > 0);
+    const size_t need = att_ws_bytes(pl);
     if (need > 0 && (!ws || !aligned(ws, 256) || ws_bytes < need)) return CSA2_ERR_WORKSPACE;
 
     AttParams P;
@@ -358,25 +440,24 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int B, int Sq, int H, in
     P.scale_log2 = softmax_scale * 1.4426950408889634f;
     P.out = out;
     P.lse = lse;
-    P.n_splits = sp.n_splits;
-    P.tiles_per_split = sp.tiles_per_split;
     P.part_o = nullptr;
     P.part_ml = nullptr;
-    if (sp.n_splits > 1) {
+    P.n_win = pl.n_win;
+    P.n_st = pl.n_st;
+    P.total_steps = pl.total;
+    if (need > 0) {
         uint8_t *base = static_cast<uint8_t *>(ws);
         P.part_o = reinterpret_cast<float *>(base);
         P.part_ml = reinterpret_cast<float2 *>(
-            base + round_up(static_cast<size_t>(R) * sp.n_splits * kHeads * kDim * 4, 256));
+            base + round_up(static_cast<size_t>(2) * pl.grid * kHeads * kDim * 4, 256));
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    dim3 grid(sp.n_splits, R);
-    cudaError_t e = launch_pdl(sparse_attn_kernel, grid, dim3(kAttThreads), kAttSmemBytes, st, P);
+    cudaError_t e = launch_pdl(sparse_attn_kernel, dim3(pl.grid), dim3(kAttThreads), kAttSmemBytes, st, P);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
-    if (sp.n_splits > 1) {
-        e = launch_pdl(attn_merge_kernel, dim3(R, kHeads / kMergeHeads), dim3(kMergeThreads),
-                       sp.n_splits * kMergeHeads * sizeof(float2), st,
-                       static_cast<const float *>(P.part_o), static_cast<const float2 *>(P.part_ml), sp.n_splits,
-                       out, lse);
+    if (pl.grid > 1) {
+        e = launch_pdl(attn_merge_kernel, dim3(R, kHeads / kMergeHeads), dim3(kMergeThreads), 0, st,
+                       static_cast<const float *>(P.part_o), static_cast<const float2 *>(P.part_ml), pl.total,
+                       pl.n_st, pl.grid, out, lse);
     }
     return cuda_status(e);
 }
@@ -404,13 +485,20 @@ csa2_status csa2_sparse_attn_decode_noalloc(const void *q_bf16, int B, int Sq, i
                                             int max_pages, const int32_t *seq_lens, const int32_t *topk_idx,
                                             int k, const void *swa_bf16, int W, float softmax_scale, float *out,
                                             float *lse, void *stream) {
-    if (B <= 0 || Sq <= 0 || k < 0) return CSA2_ERR_INVALID_ARG;
+    // The shape and range checks of csa2_sparse_attn_decode come first, so a
+    // bad argument reports its own status rather than a workspace error.
+    if (H != kHeads || D != kDim || (W != kWindow && W != 0)) return CSA2_ERR_UNSUPPORTED;
+    if (B <= 0 || Sq <= 0 || k < 0 || k > 65536) return CSA2_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(B) * Sq > 65535) return CSA2_ERR_UNSUPPORTED;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CSA2_ERR_CUDA;
-    if (g_noalloc_ptr[dev] == nullptr) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return CSA2_ERR_CUDA;
-        g_noalloc_ptr[dev] = p;
+    {
+        std::lock_guard<std::mutex> lock(g_init_mutex);      // first call per device: one thread looks up
+        if (g_noalloc_ptr[dev] == nullptr) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return CSA2_ERR_CUDA;
+            g_noalloc_ptr[dev] = p;
+        }
     }
     const size_t need = csa2_sparse_attn_workspace_bytes(B, Sq, k);
     if (need > CSA2_NOALLOC_SCRATCH_BYTES) return CSA2_ERR_WORKSPACE;

@@ -22,6 +22,13 @@
 //           these are the lowest token indices) are compacted in order.
 // Scores equal the mathematical value whenever every partial sum is exact in
 // fp32 (small-integer E4M3 inputs, sigma = 1, power-of-two weights), like K2.
+//
+// Merge mode (context-parallel decode): the entries are the shards' top-k
+// lists with their scores given, in shard order (each list ascending, the
+// shards owning increasing position ranges, so the concatenation ascends);
+// the same selection gives the top-k of the union, which is the top-k of the
+// whole context, and each shard may take the entries it owns as local
+// positions.
 #pragma once
 
 #include "common.cuh"
@@ -46,7 +53,7 @@ constexpr size_t pool_smem_bytes(int pool_size) {
 }
 
 struct PoolArgs {
-    const uint8_t *q_idx;        // [R][4][64] E4M3
+    const uint8_t *q_idx;        // [R][4][64] E4M3 (scoring mode)
     const float *w;              // [R][4]
     const uint8_t *kidx;         // [pages][4096]
     const float *kidx_scale;     // [pages][64]
@@ -55,10 +62,18 @@ struct PoolArgs {
     int max_pages;
     const int32_t *seq_lens;     // [B]
     int Sq;
-    const int32_t *pool;         // [R][C]
+    // Entry i of row r is at pool[(i / seg) * seg_stride + r * row_stride + i % seg]
+    // (one segment [R][C] for a candidate pool; [shards][R][k_shard] for a merge).
+    const int32_t *pool;
     int C;
+    int seg;
+    int64_t seg_stride;
+    int64_t row_stride;
+    const float *given;          // merge mode: the entries' scores (same addressing), no scoring
     int k;
-    int32_t *out;                // [R][k]
+    int32_t *out;                // [R][k] (may be null in merge mode)
+    int32_t *out_local;          // merge mode: [R][k] entries in [lo, hi) minus lo, else -1 (or null)
+    int32_t lo, hi;
 };
 
 // From a shared 2048-bin histogram, the bin holding the need-th largest key
@@ -102,15 +117,15 @@ pool_topk_kernel(const PoolArgs A) {
     const int b = row / A.Sq;
 
     // Inputs no earlier kernel of the step writes: the query and weights.
-    if (tid < kIdxHeads * kIdxDim / 2) {
+    if (!A.given && tid < kIdxHeads * kIdxDim / 2) {
         const uint8_t *qb = A.q_idx + static_cast<int64_t>(row) * kIdxHeads * kIdxDim + 2 * tid;
         const uint32_t h2 = e4m3x2_to_f16x2(qb[0] | (static_cast<uint32_t>(qb[1]) << 8));
         const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h2));
         (&fs.q[0][0])[2 * tid] = f.x;
         (&fs.q[0][0])[2 * tid + 1] = f.y;
     }
-    if (tid < kIdxHeads) fs.w[tid] = A.w[static_cast<int64_t>(row) * kIdxHeads + tid];
-    int T = A.seq_lens[b];
+    if (!A.given && tid < kIdxHeads) fs.w[tid] = A.w[static_cast<int64_t>(row) * kIdxHeads + tid];
+    int T = A.given ? A.Sq : A.seq_lens[b];
     pdl_wait();                                  // the pool is written by the previous kernel
     pdl_trigger();
     if (T < A.Sq || T > A.max_pages * kPage) {
@@ -123,14 +138,20 @@ pool_topk_kernel(const PoolArgs A) {
     __syncthreads();
 
     // ---------------- score every pool entry
-    const int32_t *prow = A.pool + static_cast<int64_t>(row) * A.C;
+    auto entry = [&](int i) -> int64_t {
+        return static_cast<int64_t>(i / A.seg) * A.seg_stride + static_cast<int64_t>(row) * A.row_stride + i % A.seg;
+    };
     uint32_t n_valid = 0u;
     for (int i = tid; i < A.C; i += kPoolThreads) {
-        const int t = prow[i];
+        const int t = A.pool[entry(i)];
         uint32_t key = 0u;
-        if (t >= 0) {
+        if (t >= 0 && A.given) {
+            if (i > 0 && A.pool[entry(i - 1)] >= t) flag_status(kStatusBounds);      // must ascend
+            key = float_key(__ldg(A.given + entry(i)));
+            ++n_valid;
+        } else if (t >= 0) {
             const int64_t page = t < lim ? A.page_table[static_cast<int64_t>(b) * A.max_pages + (t >> 6)] : -1;
-            if (i > 0 && prow[i - 1] >= t) flag_status(kStatusBounds);      // pool must ascend
+            if (i > 0 && A.pool[entry(i - 1)] >= t) flag_status(kStatusBounds);      // pool must ascend
             if (page >= 0 && page < A.num_pages) {
                 const int r = t & 63;
                 const uint8_t *kb = A.kidx + page * kKidxPageBytes + (r >> 3) * 512 + (r & 7) * 16;
@@ -220,20 +241,25 @@ pool_topk_kernel(const PoolArgs A) {
     // Position of an entry = selected strictly-greater entries before it plus
     // kept ties before it.
     uint32_t gt_before = static_cast<uint32_t>(pre & 0xffffffffu);
-    int32_t *orow = A.out + static_cast<int64_t>(row) * A.k;
+    int32_t *orow = A.out ? A.out + static_cast<int64_t>(row) * A.k : nullptr;
+    int32_t *lrow = A.out_local ? A.out_local + static_cast<int64_t>(row) * A.k : nullptr;
+    auto put = [&](uint32_t pos, int32_t t) {
+        if (orow) orow[pos] = t;
+        if (lrow) lrow[pos] = (t >= A.lo && t < A.hi) ? t - A.lo : -1;
+    };
     for (int i = i0; i < i1; ++i) {
         const uint32_t kk = keys[i];
         if (kk == 0u) continue;
         if (all || kk > thr) {
             const uint32_t pos = gt_before + min(tie_before, ties_keep);
-            if (pos < need) orow[pos] = prow[i];
+            if (pos < need) put(pos, A.pool[entry(i)]);
             ++gt_before;
         } else if (kk == thr) {
-            if (tie_before < ties_keep && gt_before + tie_before < need) orow[gt_before + tie_before] = prow[i];
+            if (tie_before < ties_keep && gt_before + tie_before < need) put(gt_before + tie_before, A.pool[entry(i)]);
             ++tie_before;
         }
     }
-    for (int i = static_cast<int>(need) + tid; i < A.k; i += kPoolThreads) orow[i] = -1;
+    for (int i = static_cast<int>(need) + tid; i < A.k; i += kPoolThreads) put(static_cast<uint32_t>(i), -1);
 }
 
 inline cudaError_t launch_pool_topk(const PoolArgs &A, int rows, cudaStream_t stream) {

@@ -146,7 +146,7 @@ __device__ __forceinline__ bool e4m3_quotient_near(float p) {
     return mid || sub;
 }
 
-__global__ void __launch_bounds__(kIdxQuantThreads)
+__global__ void __launch_bounds__(kIdxQuantThreads, 4)
 quant_index_fp8_kernel(const uint4 *__restrict__ x, int64_t n_rows, uint2 *__restrict__ codes,
                        float *__restrict__ sigma) {
     pdl_wait();
@@ -218,10 +218,12 @@ quant_index_fp8_kernel(const uint4 *__restrict__ x, int64_t n_rows, uint2 *__res
     }
 }
 
-inline cudaError_t launch_quant_index_fp8(const void *x, int64_t n_rows, void *codes, float *sigma, int sm_count,
+// Grid: one wave of resident blocks (grid-stride loop), or fewer when the
+// rows run out.
+inline cudaError_t launch_quant_index_fp8(const void *x, int64_t n_rows, void *codes, float *sigma, int resident,
                                           cudaStream_t stream) {
     const int64_t need = (n_rows + kIdxQuantRowsPerBlock - 1) / kIdxQuantRowsPerBlock;
-    const int64_t blocks = std::min<int64_t>(need, static_cast<int64_t>(sm_count) * 8);
+    const int64_t blocks = std::min<int64_t>(need, resident);
     return launch_pdl(quant_index_fp8_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kIdxQuantThreads), 0, stream,
                       static_cast<const uint4 *>(x), n_rows, static_cast<uint2 *>(codes), sigma);
 }

@@ -229,7 +229,8 @@ __device__ __forceinline__ uint32_t tk_word(uint32_t nib) {
 
 __global__ void __launch_bounds__(kTkThreads, 1)
 topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint32_t *__restrict__ hist,
-                    const int32_t *__restrict__ seq_lens, int Sq, int max_pages, int k, int32_t *__restrict__ out) {
+                    const int32_t *__restrict__ seq_lens, int Sq, int max_pages, int k, int32_t *__restrict__ out,
+                    float *__restrict__ out_scores) {
     namespace cg = cooperative_groups;
     extern __shared__ __align__(128) uint8_t smem_raw[];
     TkSmem &sm = *reinterpret_cast<TkSmem *>(smem_raw);
@@ -242,11 +243,15 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     pdl_trigger();
     const int n_valid = topk_n_valid(seq_lens, row, Sq, max_pages);
     int32_t *orow = out + static_cast<int64_t>(row) * k;
+    float *srow_out = out_scores ? out_scores + static_cast<int64_t>(row) * k : nullptr;
+    const float *srow = scores + static_cast<int64_t>(row) * t_cap;
     if (n_valid <= k) {                                 // every valid position is selected
-        for (int i = rank * kTkThreads + tid; i < k; i += C * kTkThreads) orow[i] = i < n_valid ? i : -1;
+        for (int i = rank * kTkThreads + tid; i < k; i += C * kTkThreads) {
+            orow[i] = i < n_valid ? i : -1;
+            if (srow_out) srow_out[i] = i < n_valid ? __ldcg(srow + i) : -INFINITY;
+        }
         return;                                         // no distributed shared memory was touched
     }
-    const float *srow = scores + static_cast<int64_t>(row) * t_cap;
     const int64_t per = (static_cast<int64_t>(n_valid) + C - 1) / C;
     const int64_t Wn = min(static_cast<int64_t>(kTkWin), (per + 31) / 32 * 32);
     const int rounds = static_cast<int>((n_valid + C * Wn - 1) / (C * Wn));
@@ -532,7 +537,11 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
             while (m) {
                 const int bit = __ffs(m) - 1;
                 m &= m - 1u;
-                if (pos < static_cast<uint32_t>(k)) orow[pos] = static_cast<int32_t>(w0 + i * 32 + bit);
+                if (pos < static_cast<uint32_t>(k)) {
+                    const int64_t t = w0 + static_cast<int64_t>(i) * 32 + bit;
+                    orow[pos] = static_cast<int32_t>(t);
+                    if (srow_out) srow_out[pos] = __ldcg(srow + t);
+                }
                 ++pos;
             }
         }

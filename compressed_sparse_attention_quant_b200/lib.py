@@ -26,7 +26,8 @@ STATUS = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_UNSUPPORTED", 3:
 # Every function include/csa2.h declares (checked by the CPU test suite).
 EXPORTS = ("csa2_quant_kv_fp4", "csa2_quant_indexer_fp8", "csa2_indexer_topk_workspace_bytes",
            "csa2_indexer_topk", "csa2_indexer_pool_topk", "csa2_sparse_attn_workspace_bytes", "csa2_sparse_attn_decode",
-           "csa2_sparse_attn_decode_noalloc", "csa2_plan",
+           "csa2_sparse_attn_decode_noalloc", "csa2_indexer_topk_scores", "csa2_topk_merge", "csa2_lse_merge",
+           "csa2_plan",
            "csa2_last_device_error", "csa2_status_string", "csa2_launch_count")
 
 
@@ -64,6 +65,10 @@ def _load():
                                            _vp, _i32, _f32, _vp, _vp, _vp, _sz, _vp]),
         "csa2_sparse_attn_decode_noalloc": (_i32, [_vp, _i32, _i32, _i32, _i32, _cp, _vp, _i32, _vp, _vp,
                                                    _i32, _vp, _i32, _f32, _vp, _vp, _vp]),
+        "csa2_indexer_topk_scores": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _cp, _vp, _i32, _vp, _i32, _vp,
+                                            _vp, _vp, _sz, _vp]),
+        "csa2_topk_merge": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+        "csa2_lse_merge": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp, _vp]),
         "csa2_plan": (_i32, [_ip, _i32, _ip, _ip]),
         "csa2_last_device_error": (_i32, [_vp]),
         "csa2_status_string": (ctypes.c_char_p, [_i32]),
@@ -200,6 +205,70 @@ def indexer_topk(q_idx: torch.Tensor, w: torch.Tensor, cache: PagedCache, page_t
     return out
 
 
+def indexer_topk_scores(q_idx: torch.Tensor, w: torch.Tensor, cache: PagedCache, page_table: torch.Tensor,
+                        seq_lens: torch.Tensor, k: int, out: Optional[torch.Tensor] = None,
+                        scores: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None
+                        ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """indexer_topk that also returns the selected entries' fp32 scores (-inf for -1)."""
+    B, Sq = q_idx.shape[0], q_idx.shape[1]
+    max_pages = page_table.shape[1]
+    _req(q_idx, torch.uint8, "q_idx", (B, Sq, IDX_HEADS, IDX_DIM))
+    _req(w, torch.float32, "w", (B, Sq, IDX_HEADS))
+    _req(page_table, torch.int32, "page_table", (B, max_pages))
+    _req(seq_lens, torch.int32, "seq_lens", (B,))
+    if out is None:
+        out = torch.empty(B, Sq, k, dtype=torch.int32, device=q_idx.device)
+    if scores is None:
+        scores = torch.empty(B, Sq, k, dtype=torch.float32, device=q_idx.device)
+    _req(out, torch.int32, "out_idx", (B, Sq, k))
+    _req(scores, torch.float32, "out_scores", (B, Sq, k))
+    if ws is None:
+        ws = workspace(indexer_topk_workspace_bytes(B, Sq, max_pages, k), q_idx.device)
+    rc = _L.csa2_indexer_topk_scores(_ptr(q_idx), _ptr(w), B, Sq, IDX_HEADS, IDX_DIM, ctypes.byref(cache.desc),
+                                     _ptr(page_table), max_pages, _ptr(seq_lens), k, _ptr(out), _ptr(scores),
+                                     _ptr(ws), ws.numel() * ws.element_size(), _stream())
+    _check("csa2_indexer_topk_scores", rc)
+    return out, scores
+
+
+def topk_merge(cand_scores: torch.Tensor, cand_idx: torch.Tensor, k: int, shard_lo: int = 0, shard_hi: int = 0,
+               out: Optional[torch.Tensor] = None, out_local: Optional[torch.Tensor] = None,
+               want_global: bool = True, want_local: bool = False):
+    """Global top-k from G shards' candidates [G, R, k_shard] (scores, global
+    positions). Returns (global [R, k] or None, local [R, k] or None)."""
+    G, R, ks = cand_idx.shape
+    _req(cand_scores, torch.float32, "cand_scores", (G, R, ks))
+    _req(cand_idx, torch.int32, "cand_idx", (G, R, ks))
+    if want_global and out is None:
+        out = torch.empty(R, k, dtype=torch.int32, device=cand_idx.device)
+    if want_local and out_local is None:
+        out_local = torch.empty(R, k, dtype=torch.int32, device=cand_idx.device)
+    for t, name in ((out, "out_idx"), (out_local, "out_local")):
+        if t is not None:
+            _req(t, torch.int32, name, (R, k))
+    rc = _L.csa2_topk_merge(_ptr(cand_scores), _ptr(cand_idx), G, R, ks, k, int(shard_lo), int(shard_hi),
+                            _ptr(out), _ptr(out_local), _stream())
+    _check("csa2_topk_merge", rc)
+    return out, out_local
+
+
+def lse_merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: Optional[torch.Tensor] = None,
+              lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One softmax over disjoint key sets: o_parts [P, R, 16, 576], lse_parts [P, R, 16]."""
+    P, R = o_parts.shape[0], o_parts.shape[1]
+    _req(o_parts, torch.float32, "o_parts", (P, R, HEADS, DIM))
+    _req(lse_parts, torch.float32, "lse_parts", (P, R, HEADS))
+    if out is None:
+        out = torch.empty(R, HEADS, DIM, dtype=torch.float32, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty(R, HEADS, dtype=torch.float32, device=o_parts.device)
+    _req(out, torch.float32, "out", (R, HEADS, DIM))
+    _req(lse, torch.float32, "lse", (R, HEADS))
+    rc = _L.csa2_lse_merge(_ptr(o_parts), _ptr(lse_parts), P, R, _ptr(out), _ptr(lse), _stream())
+    _check("csa2_lse_merge", rc)
+    return out, lse
+
+
 def indexer_scores_in_workspace(ws: torch.Tensor, B: int, Sq: int, max_pages: int) -> torch.Tensor:
     """The fp32 scores a completed csa2_indexer_topk call leaves at the start
     of its workspace, as a view [B, Sq, 64 * max_pages] (csa2.h: entries after
@@ -231,10 +300,11 @@ def indexer_pool_topk(q_idx: torch.Tensor, w: torch.Tensor, cache: PagedCache, p
 
 
 def sparse_attn_decode(q: torch.Tensor, cache: PagedCache, page_table: torch.Tensor,
-                       seq_lens: torch.Tensor, topk_idx: Optional[torch.Tensor], swa: torch.Tensor,
+                       seq_lens: torch.Tensor, topk_idx: Optional[torch.Tensor], swa: Optional[torch.Tensor],
                        softmax_scale: float, out: Optional[torch.Tensor] = None,
                        lse: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None
                        ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """swa None: no window rows (W = 0, a context-parallel shard without the newest tokens)."""
     B, Sq = q.shape[0], q.shape[1]
     max_pages = page_table.shape[1]
     _req(q, torch.bfloat16, "q", (B, Sq, HEADS, DIM))
@@ -243,7 +313,8 @@ def sparse_attn_decode(q: torch.Tensor, cache: PagedCache, page_table: torch.Ten
     k = 0 if topk_idx is None else topk_idx.shape[2]
     if topk_idx is not None:
         _req(topk_idx, torch.int32, "topk_idx", (B, Sq, k))
-    _req(swa, torch.bfloat16, "swa", (B, WINDOW + Sq - 1, DIM))
+    if swa is not None:
+        _req(swa, torch.bfloat16, "swa", (B, WINDOW + Sq - 1, DIM))
     if out is None:
         out = torch.empty(B, Sq, HEADS, DIM, dtype=torch.float32, device=q.device)
     if lse is None:
@@ -254,7 +325,8 @@ def sparse_attn_decode(q: torch.Tensor, cache: PagedCache, page_table: torch.Ten
     if ws is None:
         ws = workspace(need, q.device)
     rc = _L.csa2_sparse_attn_decode(_ptr(q), B, Sq, HEADS, DIM, ctypes.byref(cache.desc), _ptr(page_table),
-                                    max_pages, _ptr(seq_lens), _ptr(topk_idx), k, _ptr(swa), WINDOW,
+                                    max_pages, _ptr(seq_lens), _ptr(topk_idx), k, _ptr(swa),
+                                    WINDOW if swa is not None else 0,
                                     float(softmax_scale), _ptr(out), _ptr(lse), _ptr(ws),
                                     ws.numel() * ws.element_size(), _stream())
     _check("csa2_sparse_attn_decode", rc)

@@ -200,6 +200,65 @@ csa2_status csa2_indexer_topk(const void *q_idx, const float *w, int B, int Sq,
                               void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * csa2_indexer_topk_scores -- csa2_indexer_topk that also returns the scores
+ * of the selected entries: out_scores[b][j][i] = s_t (fp32, as computed) of
+ * t = out_idx[b][j][i], -inf where out_idx is -1. The context-parallel split
+ * of one long sequence (scope table, multi-GPU part) exchanges these
+ * (score, index) candidates between the shards that own its positions.
+ *
+ *   out_scores  device float [B][Sq][k]; every other argument, limit and
+ *               status as csa2_indexer_topk
+ */
+csa2_status csa2_indexer_topk_scores(const void *q_idx, const float *w, int B, int Sq,
+                                     int idx_heads, int idx_dim,
+                                     const csa2_paged_cache *cache,
+                                     const int32_t *page_table, int max_pages,
+                                     const int32_t *seq_lens, int k, int32_t *out_idx,
+                                     float *out_scores, void *ws, size_t ws_bytes,
+                                     void *stream);
+
+/*
+ * csa2_topk_merge -- context-parallel decode, the global top-k from the
+ * shards' candidates. G shards own increasing, disjoint position ranges of
+ * the same sequences; shard g's csa2_indexer_topk_scores output for its k_shard
+ * best positions (as global positions, ascending, -1 padded) is candidate
+ * list g. Because a shard's own top-k holds every one of its positions that
+ * belongs to the global top-k, the k best candidates by (score desc, position
+ * asc) are the top-k of the whole context, the same rule as
+ * csa2_indexer_topk.
+ *
+ *   cand_scores device float [G][R][k_shard]   (R = B * Sq query rows)
+ *   cand_idx    device int32 [G][R][k_shard]   global positions, ascending per
+ *               list, shards in position order; a descending pair sets
+ *               CSA2_ERR_DEVICE_BOUNDS
+ *   k           entries to select; 1 <= G * k_shard <= 32768
+ *   out_idx     device int32 [R][k] the global top-k, ascending, -1 padded
+ *               (may be NULL)
+ *   out_local   device int32 [R][k] the same list with the entries in
+ *               [shard_lo, shard_hi) given as local positions (minus
+ *               shard_lo) and every other entry -1: the indices a shard
+ *               attends with over its own cache (may be NULL; not both NULL)
+ * No workspace.
+ */
+csa2_status csa2_topk_merge(const float *cand_scores, const int32_t *cand_idx, int n_shards, int R,
+                            int k_shard, int k, int32_t shard_lo, int32_t shard_hi,
+                            int32_t *out_idx, int32_t *out_local, void *stream);
+
+/*
+ * csa2_lse_merge -- context-parallel decode, one softmax over the union of
+ * the shards' disjoint key sets from their normalised results:
+ *     L = log sum_p exp(lse_p),  out = sum_p exp(lse_p - L) * o_p,  lse = L
+ * A part with lse = -inf (no key) weighs 0; with no key anywhere out = 0 and
+ * lse = -inf. Natural-log lse as csa2_sparse_attn_decode writes it.
+ *
+ *   o_parts     device float [n_parts][R][16][576], 16-byte aligned
+ *   lse_parts   device float [n_parts][R][16]
+ *   out, lse    device float [R][16][576] and [R][16]
+ */
+csa2_status csa2_lse_merge(const float *o_parts, const float *lse_parts, int n_parts, int R,
+                           float *out, float *lse, void *stream);
+
+/*
  * csa2_indexer_pool_topk -- Reindex under the hierarchical sparse indexer
  * ([NEO part 2]: later indexing layers filter only within the candidate pool
  * built by the first Full layer, so their cost does not grow with the
@@ -244,18 +303,26 @@ csa2_status csa2_indexer_pool_topk(const void *q_idx, const float *w, int B, int
  *     out[b][j][h] = sum_i softmax_i(scale * <q, key_i>) * key_i
  *     lse[b][j][h] = log sum_i exp(scale * <q, key_i>)
  * With no key at all out = 0 and lse = -inf. Dequantized FP4 entries are
- * exact in f16; q and the window rows are rounded to f16 (exact for
- * magnitudes in [2^-14, 65504]); probabilities are rounded to f16; all sums
- * accumulate in fp32.
+ * exact in f16. q and the window rows are carried in f16 under a power-of-two
+ * exponent per 144-channel quarter (chosen from the values), so magnitudes
+ * from about 2^-100 to 2^110 keep f16 precision; probabilities are rounded to
+ * f16; all sums accumulate in fp32. Logits must stay within fp32 range.
  *
  *   q_bf16      device bf16 [B][Sq][16][576]
  *   cache       host pointer; reads kv_fp4 and kv_scale of the owner's cache
  *   page_table  device int32 [B][max_pages];   seq_lens device int32 [B]
- *   topk_idx    device int32 [B][Sq][k] (k may be 0: window only)
- *   swa_bf16    device bf16 [B][W + Sq - 1][576], W must be 128
+ *   topk_idx    device int32 [B][Sq][k] (k may be 0: window only); an index
+ *               after its query's position, past the sequence or on a bad
+ *               page sets CSA2_ERR_DEVICE_BOUNDS and is skipped
+ *   swa_bf16    device bf16 [B][W + Sq - 1][576]; W must be 128, or 0 for no
+ *               window rows at all (swa_bf16 may then be NULL; a
+ *               context-parallel shard that does not hold the newest tokens).
+ *               W = 0 with k = 0 is CSA2_ERR_INVALID_ARG.
  *   out         device float [B][Sq][16][576];  lse device float [B][Sq][16]
  *   ws          device workspace of csa2_sparse_attn_workspace_bytes() bytes,
- *               256-byte aligned (split-k partials); clobbered.
+ *               256-byte aligned (partials of rows split over CTAs; at most
+ *               2 x CTAs x 37 KB); clobbered. The size returned for (B, Sq, k)
+ *               also covers W = 0.
  */
 size_t csa2_sparse_attn_workspace_bytes(int B, int Sq, int k);
 csa2_status csa2_sparse_attn_decode(const void *q_bf16, int B, int Sq, int H,

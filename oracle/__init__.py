@@ -24,6 +24,42 @@ import numpy as np
 from . import build as _build
 
 _lib = None
+_openmp = False
+
+
+def use_all_cores(on: bool = True) -> None:
+    """Load the OpenMP build of the same C source (bit-identical results; its
+    independent outer loops run on every host core). For timing the oracle
+    only; must be chosen before the first oracle call of the process."""
+    global _openmp
+    if _lib is not None and on != _openmp:
+        raise RuntimeError("oracle library already loaded")
+    _openmp = on
+
+
+_nthreads = None
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def set_threads(n: int) -> None:
+    """Threads of the OpenMP build's parallel loops (the test build ignores it)."""
+    global _nthreads
+    if _openmp:
+        lib().omp_set_num_threads(int(n))       # libgomp, reached through the library's handle
+        _nthreads = int(n)
+
+
+def threads() -> int:
+    """Threads the loaded oracle runs its parallel loops on (1 for the test build)."""
+    if not _openmp:
+        return 1
+    return _nthreads if _nthreads is not None else host_cores()
 
 _u8p = ctypes.POINTER(ctypes.c_uint8)
 _u16p = ctypes.POINTER(ctypes.c_uint16)
@@ -36,7 +72,7 @@ _intp = ctypes.POINTER(ctypes.c_int)
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
+        path = _build.build(openmp=_openmp)
         L = ctypes.CDLL(path)
         L.orc_bf16_value.restype = ctypes.c_double
         L.orc_bf16_value.argtypes = [ctypes.c_uint16]

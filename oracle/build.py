@@ -13,26 +13,32 @@ SRC = os.path.join(HERE, "csa2_oracle.c")
 HDR = os.path.join(HERE, "csa2_oracle.h")
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(OUT_DIR, "liboracle.so")
+LIB_OMP = os.path.join(OUT_DIR, "liboracle_omp.so")     # same source, OpenMP on (host-core timing only)
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in (SRC, HDR, __file__))
 
 
-def build(force: bool = False) -> str:
-    if force or needs_build():
+def build(force: bool = False, openmp: bool = False) -> str:
+    """Build the test oracle (single-threaded), or with openmp=True the same
+    source with its "omp parallel for" loops active."""
+    lib = LIB_OMP if openmp else LIB
+    if force or needs_build(lib):
         os.makedirs(OUT_DIR, exist_ok=True)
-        tmp = LIB + f".tmp{os.getpid()}"
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = ["gcc", "-std=c99", "-O2", "-fPIC", "-shared",
-               "-ffp-contract=off", "-fno-fast-math", "-Wall", "-Wextra",
-               "-o", tmp, SRC, "-lm"]
+               "-ffp-contract=off", "-fno-fast-math", "-Wall", "-Wextra"]
+        cmd += ["-fopenmp"] if openmp else ["-Wno-unknown-pragmas"]
+        cmd += ["-o", tmp, SRC, "-lm"]
         subprocess.run(cmd, check=True)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv))
+    print(build(force="--force" in sys.argv, openmp=True))

@@ -6,6 +6,12 @@
  * All arithmetic is fp64 or exact integers. Built with -ffp-contract=off and
  * no fast-math so that every fp64 operation is the IEEE operation written.
  *
+ * The "omp parallel for" lines mark outer loops whose iterations are
+ * independent (tokens, rows, heads): each iteration does the same operations
+ * in the same order whichever thread runs it, so the OpenMP build (used only
+ * to time the oracle on every host core) gives bit-identical results. The
+ * test build ignores them.
+ *
  * Parity status of each function (what pins it) is listed in the header of
  * tests/test_oracle_pins.py. The indexer formula itself is not printed on the
  * pages (parity unpinned: it is the DSA-style reading, see below).
@@ -173,6 +179,7 @@ void orc_quant_fp4(const uint16_t *x_bf16, int64_t n, int dim,
                    uint8_t *codes, uint8_t *scales)
 {
     int groups = dim / 16;
+    #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < n; ++t) {
         const uint16_t *row = x_bf16 + t * dim;
         uint8_t *crow = codes + t * (dim / 2);
@@ -271,6 +278,7 @@ uint8_t orc_e4m3_code_quotient(double x, float sigma)
 void orc_quant_index_fp8(const uint16_t *x_bf16, int64_t n_rows, int dim,
                          uint8_t *codes, float *sigma)
 {
+    #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < n_rows; ++t) {
         const uint16_t *row = x_bf16 + t * dim;
         double amax = 0.0;
@@ -308,6 +316,7 @@ void orc_indexer_scores(const uint8_t *q, const float *w, int n_heads,
                         int idim, const uint8_t *k, const float *sigma,
                         int64_t n, int relu, double *s)
 {
+    #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < n; ++t) {
         double score = 0.0;
         for (int h = 0; h < n_heads; ++h) {
@@ -447,7 +456,7 @@ void orc_sparse_attn(const uint16_t *q, int n_heads, int dim,
         for (int c = 0; c < dim; ++c)
             keys[(int64_t)r * dim + c] = orc_bf16_value(swa[(int64_t)i * dim + c]);
 
-    double *logit = (double *)malloc((size_t)(n_keys > 0 ? n_keys : 1) * sizeof(double));
+    #pragma omp parallel for schedule(static)
     for (int h = 0; h < n_heads; ++h) {
         double *oh = o + (int64_t)h * dim;
         if (n_keys == 0) {
@@ -456,6 +465,7 @@ void orc_sparse_attn(const uint16_t *q, int n_heads, int dim,
             lse[h] = -INFINITY;
             continue;
         }
+        double *logit = (double *)malloc((size_t)n_keys * sizeof(double));
         double m = -INFINITY;
         for (int i = 0; i < n_keys; ++i) {
             double dot = 0.0;
@@ -477,8 +487,8 @@ void orc_sparse_attn(const uint16_t *q, int n_heads, int dim,
         for (int c = 0; c < dim; ++c)
             oh[c] /= l;
         lse[h] = m + log(l);
+        free(logit);
     }
-    free(logit);
     free(keys);
 }
 

@@ -233,3 +233,65 @@ def test_argument_errors_are_reported_before_launch(mods):
         lib.indexer_topk(qi, w, cache, pt, sl, 4)
     assert e.value.status == 2                             # CSA2_ERR_UNSUPPORTED (Sq > 4)
     assert lib.launch_count() == before
+
+
+def _assert_scaled_close(o_gpu, lse_gpu, o_ref, lse_ref, what):
+    """The attention bar for inputs far from unit scale: relative L2 1e-3, and
+    max-abs 2e-3 times the output's magnitude (an absolute 2e-3 is below the
+    fp32 resolution of outputs near 1e5); lse to 2e-3 relative to its size."""
+    mag = max(1.0, float(np.abs(o_ref).max()))
+    err = np.abs(o_gpu.astype(np.float64) - o_ref)
+    rel = float(np.linalg.norm(o_gpu - o_ref)) / max(float(np.linalg.norm(o_ref)), 1e-300)
+    assert float(err.max()) <= 2e-3 * mag, f"{what}: max-abs {err.max():.3e} (scale {mag:.3e})"
+    assert rel <= 1e-3, f"{what}: rel-L2 {rel:.3e}"
+    fin = np.isfinite(lse_ref)
+    np.testing.assert_array_equal(np.isfinite(lse_gpu), fin, err_msg=what)
+    if fin.any():
+        tol = 2e-3 * np.maximum(1.0, np.abs(lse_ref[fin]))
+        assert np.all(np.abs(lse_gpu[fin] - lse_ref[fin]) <= tol), f"{what}: lse"
+
+
+@pytest.mark.parametrize("q_gain,w_gain", [(1e5, 1.0), (1.0, 1e5), (1e-6, 1.0), (1.0, 1e-6), (1e-6, 1e-6),
+                                           (3e4, 3e4)],
+                         ids=["q1e5", "win1e5", "q1e-6", "win1e-6", "both1e-6", "both3e4"])
+def test_attention_inputs_outside_the_f16_range(mods, q_gain, w_gain):
+    """Queries and window rows far outside f16's exact range (|x| > 65504 or
+    < 2^-14) against the oracle: the kernel carries power-of-two exponents
+    for them instead of narrowing to f16 directly."""
+    lib, workload = mods
+    wl = inputs.small_workload(f"range{q_gain}_{w_gain}", 2, 2, [900, 400], 64, modes=("F",), seed=9)
+    dw = workload.DeviceWorkload(wl)
+    dw.step()
+    g = dw.group
+    q = (dw.q[0].float() * q_gain).to(torch.bfloat16)
+    swa = (dw.swa[0].float() * w_gain).to(torch.bfloat16)
+    o, l = lib.sparse_attn_decode(q, g.cache(0), dw.page_table, dw.seq_lens, g.index(0), swa, SCALE)
+    assert lib.last_device_error() == 0
+    idx = g.index(0).cpu().numpy()
+    for b in range(2):
+        qb, sb = oracle.bf16_bits(q[b]), oracle.bf16_bits(swa[b])
+        for j in range(2):
+            ro, rl = attend(dw, 0, b, j, qb[j], sb, idx[b, j])
+            _assert_scaled_close(o[b, j].cpu().numpy(), l[b, j].cpu().numpy(), ro, rl, f"b {b} j {j}")
+
+
+def test_attention_index_after_the_query_is_flagged(mods):
+    """Query j sits at position T - Sq + j; a selected index after it (a
+    future draft token) is out of range: flagged and skipped."""
+    lib, workload = mods
+    wl = inputs.small_workload("causal", 1, 4, [600], 32, modes=("F",), seed=5)
+    dw = workload.DeviceWorkload(wl)
+    dw.step()
+    g = dw.group
+    idx = g.index(0).clone()
+    T = wl.lens()[0]
+    idx[0, 0, 0] = T - 1                                   # query 0 is at T - 4
+    idx[0, 0] = torch.sort(idx[0, 0]).values
+    o, l = lib.sparse_attn_decode(dw.q[0], g.cache(0), dw.page_table, dw.seq_lens, idx, dw.swa[0], SCALE)
+    assert lib.last_device_error() == 6                    # CSA2_ERR_DEVICE_BOUNDS
+    q = oracle.bf16_bits(dw.q[0][0])
+    swa = oracle.bf16_bits(dw.swa[0][0])
+    keep = idx[0, 0].cpu().numpy().copy()
+    keep[keep > T - 4] = -1                                # the kernel skips the future entry
+    ro, rl = attend(dw, 0, 0, 0, q[0], swa, keep)
+    assert_attn_close(o[0, 0].cpu().numpy(), l[0, 0].cpu().numpy(), ro, rl, "query 0")

@@ -153,11 +153,12 @@ def test_layer_group_with_candidate_pool_matches_oracle(lib):
         owner_cache[o] = {}
         for b in range(wl.batch):
             T = wl.lens()[b]
-            kv = torch.cat([r for _, r in inputs.kv_chunks(wl, o, b, "cpu")])
+            # the inputs are drawn on the device the workload was built on
+            kv = torch.cat([r for _, r in inputs.kv_chunks(wl, o, b, dw.device)])
             codes, scales = oracle.quant_fp4(oracle.bf16_bits(kv[:T]))
             owner_cache[o][b] = {"codes": codes, "scales": scales,
-                                 "kidx": inputs.kidx_rows(wl, o, b, 0, T, "cpu").numpy(),
-                                 "ksig": inputs.kidx_scale_rows(wl, o, b, 0, T, "cpu").numpy()}
+                                 "kidx": inputs.kidx_rows(wl, o, b, 0, T, dw.device).cpu().numpy(),
+                                 "ksig": inputs.kidx_scale_rows(wl, o, b, 0, T, dw.device).cpu().numpy()}
     for li, m in enumerate(wl.modes):
         layer_in[li] = {}
         for b in range(wl.batch):
@@ -196,8 +197,8 @@ def test_pool_with_four_query_tokens_is_causal_per_query(lib):
     ph, oh = pool.cpu().numpy(), out.cpu().numpy()
     for b in range(2):
         T = wl.lens()[b]
-        kid = inputs.kidx_rows(wl, 0, b, 0, T, "cpu").numpy()
-        ks = inputs.kidx_scale_rows(wl, 0, b, 0, T, "cpu").numpy()
+        kid = inputs.kidx_rows(wl, 0, b, 0, T, dw.device).cpu().numpy()
+        ks = inputs.kidx_scale_rows(wl, 0, b, 0, T, dw.device).cpu().numpy()
         for j in range(4):
             assert ph[b, j].max() <= T - 4 + j
             want = oracle.pool_reindex(dw.q_idx[1][b, j].cpu().numpy(), dw.w[1][b, j].cpu().numpy(), kid, ks,
