@@ -13,6 +13,7 @@
 #include "quant.cuh"
 #include "topk.cuh"
 #include "pool.cuh"
+#include "replay.cuh"
 
 namespace csa2 {
 
@@ -69,6 +70,9 @@ cudaError_t device_info(DeviceInfo **out) {
         e = cudaFuncSetAttribute(pool_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(pool_smem_bytes(kPoolMax)));
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(swa_replay_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kRpSmemBytes));
+        if (e != cudaSuccess) return e;
         // One shared-memory carveout for every kernel of the path, so that
         // consecutive launches do not reconfigure the SMs' L1 / shared split.
         const void *kernels[] = {reinterpret_cast<const void *>(quant_kv_fp4_kernel),
@@ -80,7 +84,8 @@ cudaError_t device_info(DeviceInfo **out) {
                                  reinterpret_cast<const void *>(attn_merge_kernel),
                                  reinterpret_cast<const void *>(quant_index_fp8_kernel),
                                  reinterpret_cast<const void *>(pool_topk_kernel),
-                                 reinterpret_cast<const void *>(lse_merge_kernel)};
+                                 reinterpret_cast<const void *>(lse_merge_kernel),
+                                 reinterpret_cast<const void *>(swa_replay_kernel)};
         for (const void *kf : kernels) {
             e = cudaFuncSetAttribute(kf, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
             if (e != cudaSuccess) return e;
@@ -380,6 +385,30 @@ csa2_status csa2_topk_merge(const float *cand_scores, const int32_t *cand_idx, i
     A.lo = shard_lo;
     A.hi = shard_hi;
     return cuda_status(launch_pool_topk(A, R, static_cast<cudaStream_t>(stream)));
+}
+
+csa2_status csa2_swa_replay_attn(const void *q_bf16, int B, int L, int H, int D, const void *swa_bf16, int W,
+                                 const int32_t *seq_lens, float softmax_scale, float *out, float *lse, void *stream) {
+    if (H != kHeads || D != kDim || W != kWindow) return CSA2_ERR_UNSUPPORTED;
+    if (B <= 0 || L <= 0 || !std::isfinite(softmax_scale)) return CSA2_ERR_INVALID_ARG;
+    if (B > 65535 || L > (1 << 24)) return CSA2_ERR_UNSUPPORTED;
+    if (!q_bf16 || !swa_bf16 || !seq_lens || !out || !lse) return CSA2_ERR_INVALID_ARG;
+    if (!aligned(q_bf16, 16) || !aligned(swa_bf16, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
+        !aligned(seq_lens, 4))
+        return CSA2_ERR_ALIGNMENT;
+    DeviceInfo *dev = nullptr;
+    if (device_info(&dev) != cudaSuccess) return CSA2_ERR_CUDA;
+    RpParams P;
+    P.q = static_cast<const __nv_bfloat16 *>(q_bf16);
+    P.swa = static_cast<const __nv_bfloat16 *>(swa_bf16);
+    P.seq_lens = seq_lens;
+    P.L = L;
+    P.scale_log2 = softmax_scale * 1.4426950408889634f;
+    P.out = out;
+    P.lse = lse;
+    const dim3 grid(static_cast<unsigned>((L + kRpQueries - 1) / kRpQueries), static_cast<unsigned>(B));
+    return cuda_status(launch_pdl(swa_replay_kernel, grid, dim3(kRpThreads), kRpSmemBytes,
+                                  static_cast<cudaStream_t>(stream), P));
 }
 
 csa2_status csa2_lse_merge(const float *o_parts, const float *lse_parts, int n_parts, int R, float *out, float *lse,

@@ -10,7 +10,8 @@
 // 11 + 11 + 10 bits, run by one thread-block cluster of C CTAs per query row
 // (C = 1..16). CTA r of the cluster owns the position windows
 // [(i*C + r)*W, +W) for rounds i = 0, 1, ... (a single round unless the row
-// exceeds C * 2^17 positions).
+// exceeds C * 2^17 positions); inside a window each thread owns a contiguous
+// run of positions and the bitmap words over them.
 //   level 1  the indexer already built the row's histogram of the top 11 key
 //            bits: every CTA finds the bin b1 holding the k-th largest key.
 //   pass A   one read of the CTA's scores (L2-resident): keys in bins above
@@ -127,39 +128,53 @@ __device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t *wbuf
     return res;
 }
 
-// From the row's 2048-bin histogram (global), the bin holding the need-th
-// largest key, and how many keys lie in higher bins. Every thread of the
-// block gets the answer.
-template <int NT>
-__device__ __forceinline__ void find_threshold_bin(const uint32_t *__restrict__ gh, uint32_t need,
-                                                   uint32_t *wbuf, int *s_bin, uint32_t *s_above,
-                                                   int *bin_out, uint32_t *above_out) {
-    constexpr int PER = kTopkBins / NT;
-    const int top = kTopkBins - 1 - threadIdx.x * PER;   // this thread's bins: top, top-1, ...
-    uint32_t c[PER];
+// Warp-level pick over a histogram of nbins (<= 2048, a multiple of 64) bins
+// in shared or global memory: the bin holding the need-th largest element
+// (bins scanned from the top) and the count in higher bins. Lane l owns the 64
+// bins 2047 - 64 l - 63 .. 2047 - 64 l: their sum, a warp scan, then the one
+// lane holding the crossing rescans its bins. Every lane of the warp gets the
+// answer; when the counts fall short of need (corrupt input) it is (0, 0).
+template <bool kGlobal>
+__device__ __forceinline__ uint4 pick_ld4(const uint32_t *p) {
+    return kGlobal ? __ldcg(reinterpret_cast<const uint4 *>(p)) : *reinterpret_cast<const uint4 *>(p);
+}
+
+template <bool kGlobal>
+__device__ __forceinline__ void warp_pick(const uint32_t *h, int nbins, uint32_t need, uint32_t &bin,
+                                          uint32_t &above) {
+    const int lane = threadIdx.x & 31;
+    const int lo = kTopkBins - 64 * (lane + 1);                // this lane's bins: lo .. lo + 63
     uint32_t local = 0u;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        c[i] = __ldcg(&gh[top - i]);
-        local += c[i];
-    }
-    if (threadIdx.x == 0) {                 // stays if the counts fall short of need (corrupt input)
-        *s_bin = 0;
-        *s_above = 0u;
-    }
-    uint32_t tot;
-    uint32_t run = block_excl_scan<NT>(local, wbuf, &tot);
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        if (run < need && run + c[i] >= need) {
-            *s_bin = top - i;
-            *s_above = run;
+    if (lo < nbins) {
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+            const uint4 v = pick_ld4<kGlobal>(h + lo + 4 * i);
+            local += v.x + v.y + v.z + v.w;
         }
-        run += c[i];
     }
-    __syncthreads();
-    *bin_out = *s_bin;
-    *above_out = *s_above;
+    const uint32_t incl = warp_incl_scan(local);
+    const uint32_t run0 = incl - local;                         // elements in bins above this lane's
+    const bool mine = run0 < need && incl >= need;
+    const uint32_t who = __ballot_sync(0xffffffffu, mine);
+    uint32_t b_out = 0u, a_out = 0u;
+    if (mine) {
+        uint32_t run = run0;
+        for (int i = 15; i >= 0; --i) {                         // from the top bin down
+            const uint4 v = pick_ld4<kGlobal>(h + lo + 4 * i);
+            const uint32_t c[4] = {v.w, v.z, v.y, v.x};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (run < need && run + c[e] >= need) {
+                    b_out = static_cast<uint32_t>(lo + 4 * i + 3 - e);
+                    a_out = run;
+                }
+                run += c[e];
+            }
+        }
+    }
+    const int src = who ? __ffs(who) - 1 : 0;
+    bin = who ? __shfl_sync(0xffffffffu, b_out, src) : 0u;
+    above = who ? __shfl_sync(0xffffffffu, a_out, src) : 0u;
 }
 
 struct TkSmem {
@@ -169,64 +184,30 @@ struct TkSmem {
     int32_t cpos[kTkCandCap];           // 48 KB: candidate positions
     uint32_t hloc[2][kTopkBins];        // this CTA's level-2 / level-3 histograms (read by peers)
     uint32_t hsum[kTopkBins];           // cluster-wide sum of the current level
-    uint32_t wbuf[kTkThreads / 32 + 1];
-    uint64_t wbuf64[kTkThreads / 32 + 1];
+    uint32_t wsel[kTkThreads / 32];     // per-warp counts of the emission
+    uint32_t wtie[kTkThreads / 32];
     uint32_t xchg[2][2];                // per round parity: (selected before ties, ties), read by peers
     uint32_t n_cand;
-    int s_bin;
-    uint32_t s_above;
-    uint32_t s_digit;
-    uint32_t s_cum;
+    uint32_t s_pick[2];                 // (bin / digit, count above) of the current level
     uint32_t s_flag;
-    uint32_t s_base[4];
 };
 
-// Digit of the need-th largest element of a histogram of nbins (<= 2048)
-// bins, and the count of elements in higher bins.
-__device__ __forceinline__ void tk_pick(TkSmem &sm, const uint32_t *h, int nbins, uint32_t need, uint32_t &digit,
-                                        uint32_t &above) {
-    const int top = kTopkBins - 1 - static_cast<int>(threadIdx.x) * 2;
-    if (threadIdx.x == 0) {                 // stays if the counts fall short of need (corrupt input)
-        sm.s_digit = 0u;
-        sm.s_cum = 0u;
-    }
-    const uint32_t c0 = top < nbins ? h[top] : 0u;
-    const uint32_t c1 = top - 1 < nbins ? h[top - 1] : 0u;
-    uint32_t tot;
-    const uint32_t run = block_excl_scan<kTkThreads>(c0 + c1, sm.wbuf, &tot);
-    if (run < need && run + c0 >= need) {
-        sm.s_digit = static_cast<uint32_t>(top);
-        sm.s_cum = run;
-    } else if (run + c0 < need && run + c0 + c1 >= need) {
-        sm.s_digit = static_cast<uint32_t>(top - 1);
-        sm.s_cum = run + c0;
-    }
-    __syncthreads();
-    digit = sm.s_digit;
-    above = sm.s_cum;
-    __syncthreads();
-}
-
 // Guarded float4 of scores at positions p .. p+3 (< w1 only).
-__device__ __forceinline__ float4 tk_load(const float *srow, int64_t p, int64_t w1, bool live) {
-    if (live && p + 4 <= w1) return __ldcg(reinterpret_cast<const float4 *>(srow + p));
+__device__ __forceinline__ float4 tk_load(const float *srow, int64_t p, int64_t w1) {
+    if (p + 4 <= w1) return __ldcg(reinterpret_cast<const float4 *>(srow + p));
     float t[4] = {0.f, 0.f, 0.f, 0.f};
-    if (live)
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (p + u < w1) t[u] = __ldcg(srow + p + u);
+    for (int u = 0; u < 4; ++u)
+        if (p + u < w1) t[u] = __ldcg(srow + p + u);
     return make_float4(t[0], t[1], t[2], t[3]);
 }
 
-// OR of a 4-bit group over the 8 lanes sharing one 32-position bitmap word.
-__device__ __forceinline__ uint32_t tk_word(uint32_t nib) {
-    uint32_t w = nib << ((threadIdx.x & 7) * 4);
-    w |= __shfl_xor_sync(0xffffffffu, w, 1);
-    w |= __shfl_xor_sync(0xffffffffu, w, 2);
-    w |= __shfl_xor_sync(0xffffffffu, w, 4);
-    return w;
-}
-
+// Work layout: in each round the CTA's window of Wn positions is split into
+// contiguous runs of P = Wn / 1024 positions (a multiple of 32), one per
+// thread, so a thread's bitmap words hold only its own positions and need no
+// exchange between lanes. Warp-level scans replace block-wide ones: every
+// level and the emission take one CTA barrier plus, for the cluster-wide
+// counts, one cluster barrier.
 __global__ void __launch_bounds__(kTkThreads, 1)
 topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint32_t *__restrict__ hist,
                     const int32_t *__restrict__ seq_lens, int Sq, int max_pages, int k, int32_t *__restrict__ out,
@@ -238,7 +219,7 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     const int C = static_cast<int>(cluster.num_blocks());
     const int rank = static_cast<int>(cluster.block_rank());
     const int row = blockIdx.x / C;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_wait();                                         // scores and histograms are complete
     pdl_trigger();
     const int n_valid = topk_n_valid(seq_lens, row, Sq, max_pages);
@@ -253,114 +234,95 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
         return;                                         // no distributed shared memory was touched
     }
     const int64_t per = (static_cast<int64_t>(n_valid) + C - 1) / C;
-    const int64_t Wn = min(static_cast<int64_t>(kTkWin), (per + 31) / 32 * 32);
+    const int64_t Wn = min(static_cast<int64_t>(kTkWin), (per + 32 * kTkThreads - 1) / (32 * kTkThreads) * (32 * kTkThreads));
+    const int P = static_cast<int>(Wn / kTkThreads);   // positions per thread: 32 .. 128
+    const int NW = P / 32;                              // bitmap words per thread
     const int rounds = static_cast<int>((n_valid + C * Wn - 1) / (C * Wn));
     const bool fast = rounds == 1;
-    auto win = [&](int r, int64_t &w0, int64_t &w1, int &n_it) {
+    auto win = [&](int r, int64_t &w0, int64_t &w1) {
         w0 = (static_cast<int64_t>(r) * C + rank) * Wn;
         w1 = min(w0 + Wn, static_cast<int64_t>(n_valid));
-        n_it = w1 > w0 ? static_cast<int>((w1 - w0 + 4 * kTkThreads - 1) / (4 * kTkThreads)) : 0;
     };
 
     for (int i = tid; i < 2 * kTopkBins; i += kTkThreads) (&sm.hloc[0][0])[i] = 0u;
     if (tid == 0) sm.n_cand = 0u;
-    // ---- level 1: from the indexer's histogram
-    int b1;
-    uint32_t above1;
-    find_threshold_bin<kTkThreads>(hist + static_cast<int64_t>(row) * kTopkBins, static_cast<uint32_t>(k), sm.wbuf,
-                                   &sm.s_bin, &sm.s_above, &b1, &above1);
-    uint32_t need = static_cast<uint32_t>(k) - above1;
+    // ---- level 1: one warp scans the indexer's histogram of the row
+    if (warp == 0) {
+        uint32_t b1w, a1w;
+        warp_pick<true>(hist + static_cast<int64_t>(row) * kTopkBins, kTopkBins, static_cast<uint32_t>(k), b1w, a1w);
+        if (lane == 0) {
+            sm.s_pick[0] = b1w;
+            sm.s_pick[1] = a1w;
+        }
+    }
+    __syncthreads();
+    const int b1 = static_cast<int>(sm.s_pick[0]);
+    uint32_t need = static_cast<uint32_t>(k) - sm.s_pick[1];
 
     // ---- pass A: sure bits, level-2 histogram, candidate list
     // With a positive threshold bin (1024 < b1 < 2047) a score is above b1,
     // or in b1, exactly when its IEEE bits as a signed integer are at least
     // hi_bits, or in [lo_bits, hi_bits): negative scores and -0 fall below
-    // both. That skips the key transform for all but the candidates.
+    // both. Otherwise the order-preserving key decides.
     const bool pos = b1 > 1024 && b1 < kTopkBins - 1;
     const int32_t lo_bits = (b1 - 1024) << kTopkDigitShift;
     const int32_t hi_bits = (b1 - 1023) << kTopkDigitShift;
+    auto classify = [&](float f, int64_t p, int64_t w1, bool &sure, bool &cand, uint32_t &key) {
+        key = float_key(f);
+        if (p >= w1) {
+            sure = cand = false;
+        } else if (pos) {
+            const int32_t bits = __float_as_int(f);
+            sure = bits >= hi_bits;
+            cand = !sure && bits >= lo_bits;
+        } else {
+            const int bin = static_cast<int>(key >> kTopkDigitShift);
+            sure = bin > b1;
+            cand = bin == b1;
+        }
+    };
     for (int r = 0; r < rounds; ++r) {
         int64_t w0, w1;
-        int n_it;
-        win(r, w0, w1, n_it);
-        for (int i0 = 0; i0 < n_it; i0 += kTkUnroll) {
-            float4 f[kTkUnroll];
+        win(r, w0, w1);
+        const int64_t t0 = w0 + static_cast<int64_t>(tid) * P;
+        for (int wi = 0; wi < NW; ++wi) {
+            const int64_t pw = t0 + 32 * wi;                 // this word's first position
+            float4 f[8];
 #pragma unroll
-            for (int u = 0; u < kTkUnroll; ++u)
-                f[u] = tk_load(srow, w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) + tid * 4, w1,
-                               i0 + u < n_it);
-            uint32_t cmask = 0u;                         // 4 bits per unrolled load
+            for (int u = 0; u < 8; ++u) f[u] = tk_load(srow, pw + 4 * u, w1);
+            uint32_t sure_w = 0u, cand_w = 0u;
 #pragma unroll
-            for (int u = 0; u < kTkUnroll; ++u) {
-                const int64_t p = w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) + tid * 4;
+            for (int u = 0; u < 8; ++u) {
                 const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
-                uint32_t s4 = 0u;
-                // one bounds check per float4; per element only on the ragged tail
-                const bool full4 = i0 + u < n_it && p + 4 <= w1;
-                if (pos && full4) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int32_t bits = __float_as_int(fv[e]);
-                        if (bits >= lo_bits) {
-                            if (bits >= hi_bits) {
-                                s4 |= 1u << e;
-                            } else {
-                                cmask |= 1u << (4 * u + e);
-                                atomicAdd(&sm.hloc[0][(static_cast<uint32_t>(bits) >> 10) & (kTopkBins - 1)], 1u);
-                            }
-                        }
+                for (int e = 0; e < 4; ++e) {
+                    bool su, ca;
+                    uint32_t key;
+                    classify(fv[e], pw + 4 * u + e, w1, su, ca, key);
+                    sure_w |= (su ? 1u : 0u) << (4 * u + e);
+                    if (ca) {
+                        cand_w |= 1u << (4 * u + e);
+                        atomicAdd(&sm.hloc[0][(key >> 10) & (kTopkBins - 1)], 1u);
                     }
-                } else if (pos) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int32_t bits = __float_as_int(fv[e]);
-                        if (i0 + u < n_it && p + e < w1 && bits >= lo_bits) {
-                            if (bits >= hi_bits) {
-                                s4 |= 1u << e;
-                            } else {
-                                cmask |= 1u << (4 * u + e);
-                                atomicAdd(&sm.hloc[0][(static_cast<uint32_t>(bits) >> 10) & (kTopkBins - 1)], 1u);
-                            }
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t key = float_key(fv[e]);
-                        const int bin = static_cast<int>(key >> kTopkDigitShift);
-                        if (i0 + u < n_it && p + e < w1) {
-                            if (bin > b1) s4 |= 1u << e;
-                            if (bin == b1) {
-                                cmask |= 1u << (4 * u + e);
-                                atomicAdd(&sm.hloc[0][(key >> 10) & (kTopkBins - 1)], 1u);
-                            }
-                        }
-                    }
-                }
-                if (fast) {
-                    const uint32_t w = tk_word(s4);
-                    if ((tid & 7) == 0 && i0 + u < n_it) sm.sel[(i0 + u) * (kTkThreads / 8) + (tid >> 3)] = w;
                 }
             }
-            if (fast && __any_sync(0xffffffffu, cmask != 0u)) {
-                const uint32_t cnt = __popc(cmask);
+            if (fast) sm.sel[tid * NW + wi] = sure_w;
+            // candidates of this word -> the shared list (warp-aggregated
+            // slots); their scores are read again (L1 / L2 hits), so the
+            // loaded vectors do not stay live.
+            const uint32_t cnt = __popc(cand_w);
+            if (fast && __any_sync(0xffffffffu, cnt != 0u)) {
                 const uint32_t incl = warp_incl_scan(cnt);
                 uint32_t base = 0u;
-                if ((tid & 31) == 31) base = atomicAdd(&sm.n_cand, incl);
+                if (lane == 31) base = atomicAdd(&sm.n_cand, incl);
                 base = __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
-                while (cmask) {
-                    const int bit = __ffs(cmask) - 1;
-                    cmask &= cmask - 1u;
-                    const int u = bit >> 2, e = bit & 3;
-                    float4 fu = f[0];
-#pragma unroll
-                    for (int uu = 1; uu < kTkUnroll; ++uu)
-                        if (u == uu) fu = f[uu];                 // register select, no local array
-                    const float v = e == 0 ? fu.x : e == 1 ? fu.y : e == 2 ? fu.z : fu.w;
+                uint32_t m = cand_w;
+                while (m) {
+                    const int bit = __ffs(m) - 1;
+                    m &= m - 1u;
                     if (base < static_cast<uint32_t>(kTkCandCap)) {
-                        sm.ckey[base] = float_key(v);
-                        sm.cpos[base] = static_cast<int32_t>(w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) +
-                                                             tid * 4 + e);
+                        sm.ckey[base] = float_key(__ldcg(srow + pw + bit));
+                        sm.cpos[base] = static_cast<int32_t>(pw + bit);
                     }
                     ++base;
                 }
@@ -383,7 +345,7 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     __syncthreads();
     const bool use_list = fast && sm.s_flag == 0u;
     uint32_t d2, above2;
-    tk_pick(sm, sm.hsum, kTopkBins, need, d2, above2);
+    warp_pick<false>(sm.hsum, kTopkBins, need, d2, above2);   // every warp, same answer
     const uint32_t cnt2 = sm.hsum[d2];
     need -= above2;
     uint32_t prefix = (static_cast<uint32_t>(b1) << 11) | d2;
@@ -399,16 +361,15 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
         } else {
             for (int r = 0; r < rounds; ++r) {
                 int64_t w0, w1;
-                int n_it;
-                win(r, w0, w1, n_it);
-                for (int i = 0; i < n_it; ++i) {
-                    const int64_t p = w0 + static_cast<int64_t>(i) * (4 * kTkThreads) + tid * 4;
-                    const float4 f = tk_load(srow, p, w1, true);
+                win(r, w0, w1);
+                const int64_t t0 = w0 + static_cast<int64_t>(tid) * P;
+                for (int i = 0; i < P; i += 4) {
+                    const float4 f = tk_load(srow, t0 + i, w1);
                     const float fv[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const uint32_t key = float_key(fv[e]);
-                        if (p + e < w1 && (key >> 10) == prefix) atomicAdd(&sm.hloc[1][key & 1023u], 1u);
+                        if (t0 + i + e < w1 && (key >> 10) == prefix) atomicAdd(&sm.hloc[1][key & 1023u], 1u);
                     }
                 }
             }
@@ -421,7 +382,7 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
         }
         __syncthreads();
         uint32_t d3, above3;
-        tk_pick(sm, sm.hsum, 1024, need, d3, above3);
+        warp_pick<false>(sm.hsum, 1024, need, d3, above3);
         need -= above3;
         prefix = (prefix << 10) | d3;
         bits = 32;
@@ -433,13 +394,11 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     uint32_t out_base = 0u, tie_base = 0u;
     for (int r = 0; r < rounds; ++r) {
         int64_t w0, w1;
-        int n_it;
-        win(r, w0, w1, n_it);
-        const int nw = w1 > w0 ? static_cast<int>((w1 - w0 + 31) / 32) : 0;
-        __syncthreads();                                // the previous round's bitmaps are consumed
+        win(r, w0, w1);
+        const int64_t t0 = w0 + static_cast<int64_t>(tid) * P;
         if (use_list) {
-            for (int i = tid; i < nw; i += kTkThreads) sm.tie[i] = 0u;
-            __syncthreads();
+            for (int wi = 0; wi < NW; ++wi) sm.tie[tid * NW + wi] = 0u;
+            __syncthreads();                            // tie words zero before any candidate lands
             const uint32_t nc = sm.n_cand;
             for (uint32_t i = tid; i < nc; i += kTkThreads) {
                 const uint32_t key = sm.ckey[i];
@@ -449,104 +408,123 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
                 else if (top == prefix) atomicOr(&sm.tie[rel >> 5], 1u << (rel & 31));
             }
         } else {
-            for (int i = 0; i < n_it; ++i) {
-                const int64_t p = w0 + static_cast<int64_t>(i) * (4 * kTkThreads) + tid * 4;
-                const float4 f = tk_load(srow, p, w1, true);
-                const float fv[4] = {f.x, f.y, f.z, f.w};
+            for (int wi = 0; wi < NW; ++wi) {
                 uint32_t s4 = 0u, t4 = 0u;
+                for (int i = 0; i < 32; i += 4) {
+                    const int64_t p = t0 + 32 * wi + i;
+                    const float4 f = tk_load(srow, p, w1);
+                    const float fv[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const uint32_t key = float_key(fv[e]);
-                    const uint32_t top = bits == 32 ? key : key >> 10;
-                    if (p + e < w1) {
-                        if (top > prefix) s4 |= 1u << e;
-                        else if (top == prefix) t4 |= 1u << e;
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t key = float_key(fv[e]);
+                        const uint32_t top = bits == 32 ? key : key >> 10;
+                        if (p + e < w1) {
+                            if (top > prefix) s4 |= 1u << (i + e);
+                            else if (top == prefix) t4 |= 1u << (i + e);
+                        }
                     }
                 }
-                const uint32_t ws = tk_word(s4), wt = tk_word(t4);
-                if ((tid & 7) == 0) {
-                    sm.sel[i * (kTkThreads / 8) + (tid >> 3)] = ws;
-                    sm.tie[i * (kTkThreads / 8) + (tid >> 3)] = wt;
-                }
+                sm.sel[tid * NW + wi] = s4;
+                sm.tie[tid * NW + wi] = t4;
             }
         }
         __syncthreads();
-        // thread t owns the contiguous words [wb, we)
-        const int wper = (nw + kTkThreads - 1) / kTkThreads;
-        const int wb = min(tid * wper, nw), we = min(wb + wper, nw);
-        uint32_t n_tie = 0u, n_sel = 0u;
-        for (int i = wb; i < we; ++i) {
-            n_tie += __popc(sm.tie[i]);
-            n_sel += __popc(sm.sel[i]);
+        // counts of this thread's words, then of its warp (warp-level scans)
+        uint32_t n_sel = 0u, n_tie = 0u;
+        for (int wi = 0; wi < NW; ++wi) {
+            n_sel += __popc(sm.sel[tid * NW + wi]);
+            n_tie += __popc(sm.tie[tid * NW + wi]);
         }
-        uint64_t tot2;                                   // (ties, selected) in one scan
-        const uint32_t tie_off = static_cast<uint32_t>(
-            block_excl_scan64<kTkThreads>((static_cast<uint64_t>(n_tie) << 32) | n_sel, sm.wbuf64, &tot2) >> 32);
-        const uint32_t cta_ties = static_cast<uint32_t>(tot2 >> 32), cta_sel = static_cast<uint32_t>(tot2);
+        const uint32_t is_ = warp_incl_scan(n_sel), it_ = warp_incl_scan(n_tie);
+        if (lane == 31) {
+            sm.wsel[warp] = is_;
+            sm.wtie[warp] = it_;
+        }
+        __syncthreads();
+        uint32_t cta_sel = 0u, cta_tie = 0u, wsel_before = 0u, wtie_before = 0u;
+        for (int w = 0; w < kTkThreads / 32; ++w) {
+            const uint32_t a = sm.wsel[w], t = sm.wtie[w];
+            if (w < warp) {
+                wsel_before += a;
+                wtie_before += t;
+            }
+            cta_sel += a;
+            cta_tie += t;
+        }
         if (tid == 0) {
             sm.xchg[r & 1][0] = cta_sel;
-            sm.xchg[r & 1][1] = cta_ties;
+            sm.xchg[r & 1][1] = cta_tie;
         }
         cluster.sync();
-        if (tid == 0) {
-            // Walk the cluster in position order: ranks, each with its ties
-            // taken while the global tie rank is below `need`.
-            uint32_t op = out_base, tp = tie_base;
-            for (int q = 0; q < C; ++q) {
-                const uint32_t *x = cluster.map_shared_rank(&sm.xchg[r & 1][0], q);
-                const uint32_t s = x[0], t = x[1];
-                if (q == rank) {
-                    sm.s_base[0] = op;
-                    sm.s_base[1] = tp;
-                }
-                const uint32_t taken = need > tp ? min(t, need - tp) : 0u;
-                op += s + taken;
-                tp += t;
+        // Walk the cluster in position order: ranks, each with its ties
+        // taken while the global tie rank is below `need` (every thread
+        // computes the same bases).
+        uint32_t op = out_base, tp = tie_base, my_op = 0u, my_tp = 0u;
+        for (int q = 0; q < C; ++q) {
+            const uint32_t *x = cluster.map_shared_rank(&sm.xchg[r & 1][0], q);
+            const uint32_t sq = x[0], tq = x[1];
+            if (q == rank) {
+                my_op = op;
+                my_tp = tp;
             }
-            sm.s_base[2] = op;
-            sm.s_base[3] = tp;
+            const uint32_t taken = need > tp ? min(tq, need - tp) : 0u;
+            op += sq + taken;
+            tp += tq;
         }
-        __syncthreads();
-        uint32_t tie_rank = sm.s_base[1] + tie_off;
-        uint32_t n_out = 0u;
-        for (int i = wb; i < we; ++i) {
-            uint32_t m = sm.sel[i];
-            uint32_t tm = sm.tie[i];
-            if (tm) {
+        uint32_t tie_rank = my_tp + wtie_before + it_ - n_tie;
+        // this thread's outputs: its selected positions plus its kept ties
+        uint32_t kept = 0u;
+        {
+            uint32_t tr = tie_rank;
+            for (int wi = 0; wi < NW; ++wi) {
+                uint32_t tm = sm.tie[tid * NW + wi];
                 const uint32_t c = __popc(tm);
-                if (tie_rank + c <= need) {
-                    m |= tm;
+                if (tr + c <= need) {
+                    kept += c;
                 } else {
-                    uint32_t tr = tie_rank;
                     while (tm) {
                         const uint32_t bit = tm & (0u - tm);
                         tm ^= bit;
-                        if (tr < need) m |= bit;
+                        if (tr < need) ++kept;
                         ++tr;
                     }
+                    tr -= c;
                 }
-                tie_rank += c;
-                sm.sel[i] = m;
+                tr += c;
             }
-            n_out += __popc(m);
         }
-        uint32_t cta_out;
-        uint32_t pos = sm.s_base[0] + block_excl_scan<kTkThreads>(n_out, sm.wbuf, &cta_out);
-        for (int i = wb; i < we; ++i) {
-            uint32_t m = sm.sel[i];
+        // output offset: selected and kept ties before this thread, in position order
+        const uint32_t mine = n_sel + kept;
+        const uint32_t incl = warp_incl_scan(mine);
+        __syncthreads();                                // the warp totals of the counts above are read
+        if (lane == 31) sm.wsel[warp] = incl;
+        __syncthreads();
+        uint32_t wout_before = 0u;
+        for (int w = 0; w < warp; ++w) wout_before += sm.wsel[w];
+        uint32_t pos_out = my_op + wout_before + incl - mine;
+        for (int wi = 0; wi < NW; ++wi) {
+            uint32_t m = sm.sel[tid * NW + wi];
+            uint32_t tm = sm.tie[tid * NW + wi];
+            while (tm) {                                // keep ties while the global tie rank allows
+                const uint32_t bit = tm & (0u - tm);
+                tm ^= bit;
+                if (tie_rank < need) m |= bit;
+                ++tie_rank;
+            }
             while (m) {
                 const int bit = __ffs(m) - 1;
                 m &= m - 1u;
-                if (pos < static_cast<uint32_t>(k)) {
-                    const int64_t t = w0 + static_cast<int64_t>(i) * 32 + bit;
-                    orow[pos] = static_cast<int32_t>(t);
-                    if (srow_out) srow_out[pos] = __ldcg(srow + t);
+                if (pos_out < static_cast<uint32_t>(k)) {
+                    const int64_t t = t0 + 32 * wi + bit;
+                    orow[pos_out] = static_cast<int32_t>(t);
+                    if (srow_out) srow_out[pos_out] = __ldcg(srow + t);
                 }
-                ++pos;
+                ++pos_out;
             }
         }
-        out_base = sm.s_base[2];
-        tie_base = sm.s_base[3];
+        out_base = op;
+        tie_base = tp;
+        __syncthreads();                                // the next round rewrites the bitmaps
     }
     cluster.sync();                                     // no CTA leaves while a peer may read its counts
 }

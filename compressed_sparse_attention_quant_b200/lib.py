@@ -27,6 +27,7 @@ STATUS = {0: "CSA2_OK", 1: "CSA2_ERR_INVALID_ARG", 2: "CSA2_ERR_UNSUPPORTED", 3:
 EXPORTS = ("csa2_quant_kv_fp4", "csa2_quant_indexer_fp8", "csa2_indexer_topk_workspace_bytes",
            "csa2_indexer_topk", "csa2_indexer_pool_topk", "csa2_sparse_attn_workspace_bytes", "csa2_sparse_attn_decode",
            "csa2_sparse_attn_decode_noalloc", "csa2_indexer_topk_scores", "csa2_topk_merge", "csa2_lse_merge",
+           "csa2_swa_replay_attn",
            "csa2_plan",
            "csa2_last_device_error", "csa2_status_string", "csa2_launch_count")
 
@@ -69,6 +70,7 @@ def _load():
                                             _vp, _vp, _sz, _vp]),
         "csa2_topk_merge": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
         "csa2_lse_merge": (_i32, [_vp, _vp, _i32, _i32, _vp, _vp, _vp]),
+        "csa2_swa_replay_attn": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _i32, _vp, _f32, _vp, _vp, _vp]),
         "csa2_plan": (_i32, [_ip, _i32, _ip, _ip]),
         "csa2_last_device_error": (_i32, [_vp]),
         "csa2_status_string": (ctypes.c_char_p, [_i32]),
@@ -266,6 +268,27 @@ def lse_merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, out: Optional[torc
     _req(lse, torch.float32, "lse", (R, HEADS))
     rc = _L.csa2_lse_merge(_ptr(o_parts), _ptr(lse_parts), P, R, _ptr(out), _ptr(lse), _stream())
     _check("csa2_lse_merge", rc)
+    return out, lse
+
+
+def swa_replay_attn(q: torch.Tensor, swa: torch.Tensor, seq_lens: torch.Tensor, softmax_scale: float,
+                    out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None
+                    ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Window attention of L consecutive queries per sequence: q [B, L, 16, 576]
+    bf16, swa [B, 128 + L - 1, 576] bf16 -> (out [B, L, 16, 576], lse [B, L, 16])."""
+    B, L = q.shape[0], q.shape[1]
+    _req(q, torch.bfloat16, "q", (B, L, HEADS, DIM))
+    _req(swa, torch.bfloat16, "swa", (B, WINDOW + L - 1, DIM))
+    _req(seq_lens, torch.int32, "seq_lens", (B,))
+    if out is None:
+        out = torch.empty(B, L, HEADS, DIM, dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty(B, L, HEADS, dtype=torch.float32, device=q.device)
+    _req(out, torch.float32, "out", (B, L, HEADS, DIM))
+    _req(lse, torch.float32, "lse", (B, L, HEADS))
+    rc = _L.csa2_swa_replay_attn(_ptr(q), B, L, HEADS, DIM, _ptr(swa), WINDOW, _ptr(seq_lens),
+                                 float(softmax_scale), _ptr(out), _ptr(lse), _stream())
+    _check("csa2_swa_replay_attn", rc)
     return out, lse
 
 

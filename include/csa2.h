@@ -371,6 +371,32 @@ csa2_status csa2_sparse_attn_decode_noalloc(const void *q_bf16, int B, int Sq,
                                             float *lse, void *stream);
 
 /*
+ * csa2_swa_replay_attn -- window attention of L consecutive query tokens:
+ * the SWA bounded replay ([ZUL section 5], [INF section 2]: the last 128
+ * tokens are recomputed instead of persisted) and the window part of a
+ * Full-mode prefill. Query j of sequence b sits at position
+ * seq_lens[b] - L + j and attends to the window rows j .. j + 127 of swa[b]
+ * (row r holds position seq_lens[b] - (W + L - 1) + r; rows at negative
+ * positions are skipped), one softmax per (query, head):
+ *     out[b][j][h] = sum_r softmax_r(scale * <q, row_r>) * row_r
+ * This is csa2_sparse_attn_decode with k = 0 and Sq = L, computed with the
+ * queries tiled 8 at a time over one staged copy of their window band. The
+ * scores use the exact bf16 inputs (fp32 accumulation); the window rows
+ * enter the value product in f16 under a power-of-two exponent per tile and
+ * the probabilities are rounded to f16.
+ *
+ *   q_bf16      device bf16 [B][L][16][576]
+ *   swa_bf16    device bf16 [B][W + L - 1][576], W must be 128
+ *   seq_lens    device int32 [B]; seq_lens[b] >= L (else CSA2_ERR_DEVICE_BOUNDS
+ *               and that sequence's outputs are left unwritten)
+ *   out         device float [B][L][16][576];  lse device float [B][L][16]
+ * No workspace. Limits: B <= 65535, L <= 2^24.
+ */
+csa2_status csa2_swa_replay_attn(const void *q_bf16, int B, int L, int H, int D,
+                                 const void *swa_bf16, int W, const int32_t *seq_lens,
+                                 float softmax_scale, float *out, float *lse, void *stream);
+
+/*
  * csa2_plan -- ownership bookkeeping for a group of layers ([ZUL section 3]:
  * KV owner layer -> consumer layers; [NEO part 2]: KV, indexer keys and top-K
  * indices shared across layers). Host-only, no device work.
