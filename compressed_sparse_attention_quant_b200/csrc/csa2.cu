@@ -356,7 +356,7 @@ csa2_status csa2_indexer_pool_topk(const void *q_idx, const float *w, int B, int
     A.out_local = nullptr;
     A.lo = 0;
     A.hi = 0;
-    return cuda_status(launch_pool_topk(A, B * Sq, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_pool_topk(A, B * Sq, dev->sm_count, static_cast<cudaStream_t>(stream)));
 }
 
 csa2_status csa2_topk_merge(const float *cand_scores, const int32_t *cand_idx, int n_shards, int R, int k_shard,
@@ -384,7 +384,7 @@ csa2_status csa2_topk_merge(const float *cand_scores, const int32_t *cand_idx, i
     A.out_local = out_local;
     A.lo = shard_lo;
     A.hi = shard_hi;
-    return cuda_status(launch_pool_topk(A, R, static_cast<cudaStream_t>(stream)));
+    return cuda_status(launch_pool_topk(A, R, dev->sm_count, static_cast<cudaStream_t>(stream)));
 }
 
 csa2_status csa2_swa_replay_attn(const void *q_bf16, int B, int L, int H, int D, const void *swa_bf16, int W,

@@ -5,23 +5,30 @@
 // The pool is the Full layer's top-C (ascending token indices, -1 padded, as
 // K3 emits it); the layer scores only those tokens with its own query.
 //
-// One CTA (512 threads) per query row. A pool entry after the row's query
-// position (causal bound), past the sequence or with a bad page sets the status
-// word and is skipped.
-//   score   thread i takes pool entries i, i + 512, ...: the token's 64-byte
-//           indexer key (four 16-byte chunks of its page's core-matrix
-//           layout) and sigma; four fp32 dot products with the row's query
-//           (converted from E4M3 once into shared memory), ReLU, head
-//           weights; the score's order-preserving 32-bit key goes to shared
-//           memory (0 marks an empty or invalid entry: no finite score maps
-//           there).
-//   select  radix select on the keys, 11 + 11 + 10 bits, each level a shared
-//           histogram and a block scan from the top, gives the k-th largest
-//           key T and the number of ties to keep. The entries above T and the
-//           first ties in pool order (pool order is ascending token order, so
-//           these are the lowest token indices) are compacted in order.
-// Scores equal the mathematical value whenever every partial sum is exact in
-// fp32 (small-integer E4M3 inputs, sigma = 1, power-of-two weights), like K2.
+// One thread-block cluster of S CTAs (512 threads each) per query row; CTA q
+// owns the q-th contiguous slice of the pool, so the slices are in pool order.
+//   score   warps take 16 pool entries at a time. The entries' page-table
+//           entries, scales and 64-byte indexer keys are gathered in phases
+//           (indices, then pages, then keys) so the loads of many entries are
+//           in flight together; the keys are the A operand (16 entries x 32
+//           channels per k-step) of FP8 mma.sync m16n8k32 against the row's
+//           query (4 heads as B columns), fp32 accumulation. ReLU, sigma and
+//           the head weights follow; the score's order-preserving 32-bit key
+//           goes to shared memory (0 marks an empty or invalid entry: no
+//           finite score maps there).
+//   select  radix select on the keys, 11 + 11 + 10 bits: each level a shared
+//           histogram per CTA, summed over the cluster through distributed
+//           shared memory, and a warp-level pick; it gives the k-th largest
+//           key T and the number of ties to keep.
+//   emit    entries above T and the first ties in pool order (pool order is
+//           ascending token order, so these are the lowest token indices),
+//           compacted in order: per-thread runs, warp scans, one exchange of
+//           counts across the cluster.
+// A pool entry after the row's query position (causal bound), past the
+// sequence or with a bad page sets the status word and is skipped. Scores
+// equal the mathematical value whenever every partial sum is exact in fp32
+// (small-integer E4M3 inputs, sigma = 1 or a power of two, power-of-two
+// weights), like K2.
 //
 // Merge mode (context-parallel decode): the entries are the shards' top-k
 // lists with their scores given, in shard order (each list ascending, the
@@ -32,24 +39,30 @@
 #pragma once
 
 #include "common.cuh"
+#include "topk.cuh"
+
+#include <cooperative_groups.h>
 
 namespace csa2 {
 
 constexpr int kPoolThreads = 512;
+constexpr int kPoolWarps = kPoolThreads / 32;
 constexpr int kPoolBins = 2048;
-constexpr int kPoolMax = 32768;                  // largest pool per row (128 KB of keys)
+constexpr int kPoolMax = 32768;                  // largest pool per row
+constexpr int kPoolMaxCluster = 8;
+constexpr int kPoolMaxIt = 8;                    // 16-entry groups per warp held in flight
 
 struct PoolSmemFixed {
-    float q[kIdxHeads][kIdxDim];                 // the row's query, fp32
+    uint32_t qb[kIdxHeads * kIdxDim / 4];        // the row's query, E4M3 bytes (4 per word)
     float w[kIdxHeads];
-    uint32_t hist[kPoolBins];
-    uint64_t wbuf64[kPoolThreads / 32 + 1];
-    uint32_t wbuf[kPoolThreads / 32 + 1];
-    uint32_t s_bin, s_above;
+    uint32_t hloc[kPoolBins];                    // this CTA's histogram of the current level (read by peers)
+    uint32_t hsum[kPoolBins];                    // cluster-wide sum
+    uint32_t wcnt[2][kPoolWarps];
+    uint32_t xchg[3];                            // (valid entries, selected, ties) of this CTA, read by peers
 };
 
-constexpr size_t pool_smem_bytes(int pool_size) {
-    return sizeof(PoolSmemFixed) + static_cast<size_t>(pool_size) * sizeof(uint32_t);
+constexpr size_t pool_smem_bytes(int slice) {
+    return sizeof(PoolSmemFixed) + static_cast<size_t>(slice) * sizeof(uint32_t);
 }
 
 struct PoolArgs {
@@ -74,147 +87,188 @@ struct PoolArgs {
     int32_t *out;                // [R][k] (may be null in merge mode)
     int32_t *out_local;          // merge mode: [R][k] entries in [lo, hi) minus lo, else -1 (or null)
     int32_t lo, hi;
+    int slice;                   // entries per CTA of the cluster (a multiple of 16)
 };
 
-// From a shared 2048-bin histogram, the bin holding the need-th largest key
-// and the count of keys in higher bins (each thread owns 4 bins from the top).
-__device__ __forceinline__ void pool_pick(PoolSmemFixed &fs, uint32_t need, uint32_t &bin, uint32_t &above) {
-    constexpr int PER = kPoolBins / kPoolThreads;
-    const int top = kPoolBins - 1 - static_cast<int>(threadIdx.x) * PER;
-    uint32_t c[PER];
-    uint32_t local = 0u;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        c[i] = fs.hist[top - i];
-        local += c[i];
-    }
-    if (threadIdx.x == 0) {                      // stays if the counts fall short of need
-        fs.s_bin = 0u;
-        fs.s_above = 0u;
-    }
-    uint32_t tot;
-    uint32_t run = block_excl_scan<kPoolThreads>(local, fs.wbuf, &tot);
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        if (run < need && run + c[i] >= need) {
-            fs.s_bin = static_cast<uint32_t>(top - i);
-            fs.s_above = run;
-        }
-        run += c[i];
-    }
-    __syncthreads();
-    bin = fs.s_bin;
-    above = fs.s_above;
-    __syncthreads();
+__device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __global__ void __launch_bounds__(kPoolThreads)
 pool_topk_kernel(const PoolArgs A) {
+    namespace cg = cooperative_groups;
     extern __shared__ __align__(128) uint8_t smem_raw[];
     PoolSmemFixed &fs = *reinterpret_cast<PoolSmemFixed *>(smem_raw);
     uint32_t *keys = reinterpret_cast<uint32_t *>(smem_raw + sizeof(PoolSmemFixed));
-    const int row = blockIdx.x, tid = threadIdx.x;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int S = static_cast<int>(cluster.num_blocks());
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int row = blockIdx.x / S, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, tig = lane & 3;
     const int b = row / A.Sq;
+    const int e0 = rank * A.slice;                              // this CTA's entries [e0, e1)
+    const int e1 = min(e0 + A.slice, A.C);
 
     // Inputs no earlier kernel of the step writes: the query and weights.
-    if (!A.given && tid < kIdxHeads * kIdxDim / 2) {
-        const uint8_t *qb = A.q_idx + static_cast<int64_t>(row) * kIdxHeads * kIdxDim + 2 * tid;
-        const uint32_t h2 = e4m3x2_to_f16x2(qb[0] | (static_cast<uint32_t>(qb[1]) << 8));
-        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h2));
-        (&fs.q[0][0])[2 * tid] = f.x;
-        (&fs.q[0][0])[2 * tid + 1] = f.y;
+    if (!A.given) {
+        if (tid < kIdxHeads * kIdxDim / 4)
+            fs.qb[tid] = __ldg(reinterpret_cast<const uint32_t *>(A.q_idx + static_cast<int64_t>(row) * kIdxHeads * kIdxDim) + tid);
+        if (tid < kIdxHeads) fs.w[tid] = A.w[static_cast<int64_t>(row) * kIdxHeads + tid];
     }
-    if (!A.given && tid < kIdxHeads) fs.w[tid] = A.w[static_cast<int64_t>(row) * kIdxHeads + tid];
     int T = A.given ? A.Sq : A.seq_lens[b];
-    pdl_wait();                                  // the pool is written by the previous kernel
+    pdl_wait();                                                 // the pool is written by the previous kernel
     pdl_trigger();
     if (T < A.Sq || T > A.max_pages * kPage) {
-        if (tid == 0) flag_status(kStatusBounds);
-        T = A.Sq - 1 - row % A.Sq;               // no valid token for any query of the row
+        if (tid == 0 && rank == 0) flag_status(kStatusBounds);
+        T = A.Sq - 1 - row % A.Sq;                              // no valid token for any query of the row
     }
     // Query j of the sequence sits at position T - Sq + j and is causal: a
     // pool entry after it is out of range.
     const int lim = T - A.Sq + row % A.Sq + 1;
-    __syncthreads();
-
-    // ---------------- score every pool entry
+    for (int i = tid; i < kPoolBins; i += kPoolThreads) fs.hloc[i] = 0u;
+    __syncthreads();                                            // query, weights in; histogram zero
     auto entry = [&](int i) -> int64_t {
         return static_cast<int64_t>(i / A.seg) * A.seg_stride + static_cast<int64_t>(row) * A.row_stride + i % A.seg;
     };
+
+    // ---------------- keys of this CTA's entries
     uint32_t n_valid = 0u;
-    for (int i = tid; i < A.C; i += kPoolThreads) {
-        const int t = A.pool[entry(i)];
-        uint32_t key = 0u;
-        if (t >= 0 && A.given) {
-            if (i > 0 && A.pool[entry(i - 1)] >= t) flag_status(kStatusBounds);      // must ascend
-            key = float_key(__ldg(A.given + entry(i)));
-            ++n_valid;
-        } else if (t >= 0) {
-            const int64_t page = t < lim ? A.page_table[static_cast<int64_t>(b) * A.max_pages + (t >> 6)] : -1;
-            if (i > 0 && A.pool[entry(i - 1)] >= t) flag_status(kStatusBounds);      // pool must ascend
-            if (page >= 0 && page < A.num_pages) {
-                const int r = t & 63;
-                const uint8_t *kb = A.kidx + page * kKidxPageBytes + (r >> 3) * 512 + (r & 7) * 16;
-                const float sg = A.kidx_scale[page * kPage + r];
-                float dot[kIdxHeads] = {0.f, 0.f, 0.f, 0.f};
+    if (A.given) {
+        for (int i = e0 + tid; i < e1; i += kPoolThreads) {
+            const int t = A.pool[entry(i)];
+            uint32_t key = 0u;
+            if (t >= 0) {
+                if (i > 0 && A.pool[entry(i - 1)] >= t) flag_status(kStatusBounds);   // must ascend
+                key = float_key(__ldg(A.given + entry(i)));
+                ++n_valid;
+            }
+            keys[i - e0] = key;
+        }
+    } else {
+        // query B fragments: head g (< 4) channels 4 tig .. +3 and 16 + 4 tig .. +3 of each k-step
+        uint32_t qf[2][2];
 #pragma unroll
-                for (int c16 = 0; c16 < 4; ++c16) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(kb + c16 * 128);
-                    const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+        for (int ks = 0; ks < 2; ++ks) {
+            qf[ks][0] = g < kIdxHeads ? fs.qb[(g * kIdxDim + ks * 32 + 4 * tig) / 4] : 0u;
+            qf[ks][1] = g < kIdxHeads ? fs.qb[(g * kIdxDim + ks * 32 + 16 + 4 * tig) / 4] : 0u;
+        }
+        const float wlo = fs.w[2 * (tig & 1)], whi = fs.w[2 * (tig & 1) + 1];
+        // groups of 16 entries: warp w takes groups w, w + 16, ... of the slice
+        const int n_groups = (e1 - e0 + 15) / 16;
+        for (int gb = warp; gb < n_groups; gb += kPoolWarps * kPoolMaxIt) {
+            int tok[kPoolMaxIt][2];
+            int64_t pg[kPoolMaxIt][2];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint32_t lo = e4m3x2_to_f16x2(wd[j] & 0xffffu);
-                        const uint32_t hi = e4m3x2_to_f16x2(wd[j] >> 16);
-                        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&lo));
-                        const float2 c = __half22float2(*reinterpret_cast<const __half2 *>(&hi));
-                        const int ch = c16 * 16 + j * 4;
+            for (int it = 0; it < kPoolMaxIt; ++it)              // phase 1: pool indices
 #pragma unroll
-                        for (int h = 0; h < kIdxHeads; ++h) {
-                            const float4 qv = *reinterpret_cast<const float4 *>(&fs.q[h][ch]);
-                            dot[h] = fmaf(qv.x, a.x, dot[h]);
-                            dot[h] = fmaf(qv.y, a.y, dot[h]);
-                            dot[h] = fmaf(qv.z, c.x, dot[h]);
-                            dot[h] = fmaf(qv.w, c.y, dot[h]);
+                for (int h = 0; h < 2; ++h) {
+                    const int grp = gb + it * kPoolWarps;
+                    const int i = e0 + grp * 16 + g + 8 * h;
+                    tok[it][h] = (grp < n_groups && i < e1) ? A.pool[entry(i)] : -1;
+                }
+#pragma unroll
+            for (int it = 0; it < kPoolMaxIt; ++it)              // phase 2: pages
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int t = tok[it][h];
+                    pg[it][h] = (t >= 0 && t < lim) ? A.page_table[static_cast<int64_t>(b) * A.max_pages + (t >> 6)] : -1;
+                }
+#pragma unroll
+            for (int it = 0; it < kPoolMaxIt; ++it) {           // phase 3: keys, MMA, scores
+                const int grp = gb + it * kPoolWarps;
+                if (grp >= n_groups) break;                      // warp-uniform
+                uint32_t a[2][4];
+                float sg[2];
+                bool ok[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int t = tok[it][h];
+                    const int64_t p = pg[it][h];
+                    ok[h] = t >= 0 && t < lim && p >= 0 && p < A.num_pages;
+                    const int r = t & 63;
+                    const uint8_t *kb = A.kidx + (ok[h] ? p * kKidxPageBytes + (r >> 3) * 512 + (r & 7) * 16 + 4 * tig : 0);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)                 // 16-byte chunk c = channels 16c .. 16c + 15
+                        a[c >> 1][(c & 1) * 2 + h] = ok[h] ? __ldg(reinterpret_cast<const uint32_t *>(kb + c * 128)) : 0u;
+                    sg[h] = ok[h] ? __ldg(A.kidx_scale + p * kPage + r) : 0.0f;
+                }
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks)
+                    mma_e4m3_16832(acc, a[ks][0], a[ks][1], a[ks][2], a[ks][3], qf[ks][0], qf[ks][1]);
+                // lanes with tig 0 / 1 hold heads 0, 1 / 2, 3 of entries g and g + 8
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float part = wlo * fmaxf(0.0f, sg[h] * acc[2 * h]) + whi * fmaxf(0.0f, sg[h] * acc[2 * h + 1]);
+                    part += __shfl_xor_sync(0xffffffffu, part, 1);   // heads 0..3
+                    const int i = e0 + grp * 16 + g + 8 * h;
+                    const int t = tok[it][h];
+                    if (tig == 0 && i < e1) {
+                        uint32_t key = 0u;
+                        if (ok[h]) {
+                            if (i > 0 && A.pool[entry(i - 1)] >= t) flag_status(kStatusBounds);   // pool must ascend
+                            key = float_key(part);
+                            ++n_valid;
+                        } else if (t >= 0) {
+                            flag_status(kStatusBounds);
                         }
+                        keys[i - e0] = key;
                     }
                 }
-                float score = 0.0f;
-#pragma unroll
-                for (int h = 0; h < kIdxHeads; ++h) score += fs.w[h] * fmaxf(sg * dot[h], 0.0f);
-                key = float_key(score);
-                ++n_valid;
-            } else {
-                flag_status(kStatusBounds);
             }
         }
-        keys[i] = key;
     }
+    // valid entries of the whole row (cluster)
     {
-        uint32_t tot;
-        block_excl_scan<kPoolThreads>(n_valid, fs.wbuf, &tot);
-        n_valid = tot;                           // every thread: valid entries of the row
+        const uint32_t wv = warp_incl_scan(n_valid);
+        if (lane == 31) fs.wcnt[0][warp] = wv;
+        __syncthreads();
+        if (tid == 0) {
+            uint32_t t = 0u;
+            for (int w = 0; w < kPoolWarps; ++w) t += fs.wcnt[0][w];
+            fs.xchg[0] = t;
+        }
+        cluster.sync();
     }
-    const uint32_t need = min(static_cast<uint32_t>(A.k), n_valid);
+    uint32_t row_valid = 0u;
+    for (int q = 0; q < S; ++q) row_valid += *cluster.map_shared_rank(&fs.xchg[0], q);
+    const uint32_t need = min(static_cast<uint32_t>(A.k), row_valid);
+    const int n_mine = max(e1 - e0, 0);
 
-    // ---------------- threshold key T: the need-th largest key
+    // ---------------- threshold key T: the need-th largest key over the cluster
     uint32_t thr = 0u, n_gt = 0u;                // select keys > thr, then (need - n_gt) ties == thr
-    if (need > 0u && need < n_valid) {
+    const bool all = need == row_valid;          // every valid entry is kept (also when there is none)
+    if (!all) {
         uint32_t prefix = 0u, above = 0u;
 #pragma unroll 1
         for (int lvl = 0; lvl < 3; ++lvl) {
             const int wdt = lvl < 2 ? 11 : 10;               // key bits 31..21, 20..10, 9..0
             const int shift = lvl == 0 ? 21 : (lvl == 1 ? 10 : 0);
-            for (int i = tid; i < kPoolBins; i += kPoolThreads) fs.hist[i] = 0u;
-            __syncthreads();
-            for (int i = tid; i < A.C; i += kPoolThreads) {
+            if (lvl > 0) {
+                cluster.sync();                              // every peer has read this CTA's previous level
+                for (int i = tid; i < kPoolBins; i += kPoolThreads) fs.hloc[i] = 0u;
+                __syncthreads();
+            }
+            for (int i = tid; i < n_mine; i += kPoolThreads) {
                 const uint32_t kk = keys[i];
                 if (kk == 0u) continue;
                 if (lvl > 0 && (kk >> (shift + wdt)) != prefix) continue;
-                atomicAdd(&fs.hist[(kk >> shift) & ((1u << wdt) - 1u)], 1u);
+                atomicAdd(&fs.hloc[(kk >> shift) & ((1u << wdt) - 1u)], 1u);
+            }
+            cluster.sync();
+            for (int i = tid; i < kPoolBins; i += kPoolThreads) {
+                uint32_t v = 0u;
+                for (int q = 0; q < S; ++q) v += cluster.map_shared_rank(&fs.hloc[0], q)[i];
+                fs.hsum[i] = v;
             }
             __syncthreads();
             uint32_t bin, ab;
-            pool_pick(fs, need - above, bin, ab);
+            warp_pick<false>(fs.hsum, 1 << wdt, need - above, bin, ab);
             above += ab;
             prefix = (prefix << wdt) | bin;
         }
@@ -223,9 +277,8 @@ pool_topk_kernel(const PoolArgs A) {
     }
 
     // ---------------- emit, in pool order: keys > thr, then the first ties
-    const bool all = need == n_valid;           // every valid entry is kept (also when there is none)
-    const int seg = (A.C + kPoolThreads - 1) / kPoolThreads;
-    const int i0 = min(tid * seg, A.C), i1 = min(i0 + seg, A.C);
+    const int seg = (n_mine + kPoolThreads - 1) / kPoolThreads;
+    const int i0 = min(tid * seg, n_mine), i1 = min(i0 + seg, n_mine);
     uint32_t n_sel = 0u, n_tie = 0u;
     for (int i = i0; i < i1; ++i) {
         const uint32_t kk = keys[i];
@@ -233,14 +286,37 @@ pool_topk_kernel(const PoolArgs A) {
         if (all || kk > thr) ++n_sel;
         else if (kk == thr) ++n_tie;
     }
-    uint64_t tot64;
-    const uint64_t pre = block_excl_scan64<kPoolThreads>((static_cast<uint64_t>(n_tie) << 32) | n_sel, fs.wbuf64,
-                                                        &tot64);
-    uint32_t tie_before = static_cast<uint32_t>(pre >> 32);
+    const uint32_t is_ = warp_incl_scan(n_sel), it_ = warp_incl_scan(n_tie);
+    __syncthreads();                                            // wcnt[0] of the count above is read
+    if (lane == 31) {
+        fs.wcnt[0][warp] = is_;
+        fs.wcnt[1][warp] = it_;
+    }
+    __syncthreads();
+    uint32_t cta_sel = 0u, cta_tie = 0u, sel_before = is_ - n_sel, tie_before = it_ - n_tie;
+    for (int w = 0; w < kPoolWarps; ++w) {
+        if (w < warp) {
+            sel_before += fs.wcnt[0][w];
+            tie_before += fs.wcnt[1][w];
+        }
+        cta_sel += fs.wcnt[0][w];
+        cta_tie += fs.wcnt[1][w];
+    }
+    if (tid == 0) {
+        fs.xchg[1] = cta_sel;
+        fs.xchg[2] = cta_tie;
+    }
+    cluster.sync();
     const uint32_t ties_keep = need - n_gt;
+    uint32_t sel_base = 0u, tie_base = 0u;
+    for (int q = 0; q < rank; ++q) {
+        sel_base += cluster.map_shared_rank(&fs.xchg[0], q)[1];
+        tie_base += cluster.map_shared_rank(&fs.xchg[0], q)[2];
+    }
     // Position of an entry = selected strictly-greater entries before it plus
-    // kept ties before it.
-    uint32_t gt_before = static_cast<uint32_t>(pre & 0xffffffffu);
+    // kept ties before it (both over the whole cluster, in pool order).
+    uint32_t gt_before = sel_base + sel_before;
+    uint32_t tb = tie_base + tie_before;
     int32_t *orow = A.out ? A.out + static_cast<int64_t>(row) * A.k : nullptr;
     int32_t *lrow = A.out_local ? A.out_local + static_cast<int64_t>(row) * A.k : nullptr;
     auto put = [&](uint32_t pos, int32_t t) {
@@ -251,20 +327,29 @@ pool_topk_kernel(const PoolArgs A) {
         const uint32_t kk = keys[i];
         if (kk == 0u) continue;
         if (all || kk > thr) {
-            const uint32_t pos = gt_before + min(tie_before, ties_keep);
-            if (pos < need) put(pos, A.pool[entry(i)]);
+            const uint32_t pos = gt_before + min(tb, ties_keep);
+            if (pos < need) put(pos, A.pool[entry(e0 + i)]);
             ++gt_before;
         } else if (kk == thr) {
-            if (tie_before < ties_keep && gt_before + tie_before < need) put(gt_before + tie_before, A.pool[entry(i)]);
-            ++tie_before;
+            if (tb < ties_keep && gt_before + tb < need) put(gt_before + tb, A.pool[entry(e0 + i)]);
+            ++tb;
         }
     }
-    for (int i = static_cast<int>(need) + tid; i < A.k; i += kPoolThreads) put(static_cast<uint32_t>(i), -1);
+    for (int i = static_cast<int>(need) + rank * kPoolThreads + tid; i < A.k; i += S * kPoolThreads)
+        put(static_cast<uint32_t>(i), -1);
+    cluster.sync();                                             // no CTA leaves while a peer may read its counts
 }
 
-inline cudaError_t launch_pool_topk(const PoolArgs &A, int rows, cudaStream_t stream) {
-    return launch_pdl(pool_topk_kernel, dim3(static_cast<unsigned>(rows)), dim3(kPoolThreads), pool_smem_bytes(A.C),
-                      stream, A);
+// Cluster size: the largest power of two (<= 8) with every CTA holding at
+// least 1024 entries and all clusters within one wave of two CTAs per SM.
+inline cudaError_t launch_pool_topk(PoolArgs A, int rows, int sm_count, cudaStream_t stream) {
+    int S = 1;
+    while (S * 2 <= kPoolMaxCluster && static_cast<int64_t>(rows) * S * 2 <= 2 * sm_count && A.C / (S * 2) >= 1024)
+        S *= 2;
+    A.slice = (A.C + S - 1) / S;
+    A.slice = (A.slice + 15) / 16 * 16;
+    return launch_pdl_cluster(pool_topk_kernel, dim3(static_cast<unsigned>(rows * S)), dim3(kPoolThreads),
+                              pool_smem_bytes(A.slice), stream, S, A);
 }
 
 }  // namespace csa2
