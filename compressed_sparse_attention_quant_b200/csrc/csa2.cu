@@ -159,7 +159,7 @@ AttPlan att_plan(int R, int k, int slots, bool window = true) {
     pl.n_win = window ? kAttWinSteps : 0;
     pl.n_st = pl.n_win + (k + kAttStepKeys - 1) / kAttStepKeys;
     pl.total = static_cast<int64_t>(R) * pl.n_st;
-    pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(slots, pl.total / 4)));
+    pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(std::min(slots, kMergeMaxParts), pl.total / 4)));
     return pl;
 }
 

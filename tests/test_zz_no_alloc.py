@@ -49,3 +49,28 @@ def test_noalloc_attention_matches_workspace_entry_point_twice():
             for j in range(Sq):
                 assert_attn_close(o[b, j], l[b, j], ref_o[b, j].astype(np.float64),
                                   ref_lse[b, j].astype(np.float64), f"call {call} b {b} j {j}")
+
+
+def test_noalloc_scratch_bound_and_argument_checks():
+    """The partials of any shape fit the library-owned array on this GPU
+    (at most two per CTA of one wave), and argument errors are reported as
+    themselves, before the scratch size is considered; nothing is launched."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import ctypes
+    from compressed_sparse_attention_quant_b200 import lib
+    assert 0 < lib.sparse_attn_workspace_bytes(65535, 1, 65536) <= lib.NOALLOC_SCRATCH_BYTES
+    assert lib.sparse_attn_workspace_bytes(65536, 1, 1) == 0            # B * Sq > 65535: unsupported shape
+    assert lib.sparse_attn_workspace_bytes(1, 1, 65537) == 0            # k > 65536
+    L = lib._L
+    cache = lib._Cache(16, 16, 16, 16, 4)                              # host-side checks only: never launched
+    before = lib.launch_count()
+
+    def call(B, Sq, H, k):
+        return L.csa2_sparse_attn_decode_noalloc(16, B, Sq, H, 576, ctypes.byref(cache), 16, 1, 16, 16, k, 16,
+                                                 128, 0.1, 16, 16, None)
+    assert call(1, 1, 8, 4) == 2                                         # CSA2_ERR_UNSUPPORTED: 8 heads
+    assert call(70000, 1, 16, 4) == 2                                    # B * Sq > 65535
+    assert call(1, 1, 16, -1) == 1                                       # CSA2_ERR_INVALID_ARG
+    assert call(1, 1, 16, 70000) == 1                                    # k > 65536
+    assert lib.launch_count() == before
