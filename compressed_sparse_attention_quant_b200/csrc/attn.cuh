@@ -154,7 +154,7 @@ __device__ __forceinline__ AttRow att_row(const AttParams &P, int row) {
     return r;
 }
 
-__global__ void __maxnreg__(112)
+__global__ void __maxnreg__(104)
 sparse_attn_kernel(const AttParams P) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
     AttSmem &sm = *reinterpret_cast<AttSmem *>(smem_raw);

@@ -285,10 +285,10 @@ csa2_status indexer_topk_impl(const void *q_idx, const float *w, int B, int Sq, 
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
     // Top-k: one cluster of C CTAs per query row, C a power of two chosen so
     // that the R * C CTAs stay within one wave and every CTA keeps at least
-    // 8192 positions.
+    // 32768 positions (32 per thread: one bitmap word each).
     int C = 1;
     while (C * 2 <= dev->tk_max_cluster && static_cast<int64_t>(R) * C * 2 <= dev->sm_count &&
-           L.t_cap / (C * 2) >= 8192)
+           L.t_cap / (C * 2) >= 32768)
         C *= 2;
     e = launch_pdl_cluster(topk_cluster_kernel, dim3(static_cast<unsigned>(R * C)), dim3(kTkThreads), sizeof(TkSmem),
                            st, C, static_cast<const float *>(scores), L.t_cap, static_cast<const uint32_t *>(hist),

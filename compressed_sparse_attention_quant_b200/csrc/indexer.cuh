@@ -36,7 +36,8 @@
 //        weights, stores the scores (128-byte coalesced, L2 evict-last: the
 //        selection re-reads them) and adds each valid score's top 11 key
 //        bits to a shared-memory histogram per query row (rows past the
-//        shared slots go straight to the global histogram).
+//        shared slots go straight to the global histogram); lanes of a warp
+//        with the same bin add their count with one atomic.
 // Every wait is a bounded mbarrier wait that sleeps between probes; a
 // timeout sets the status word, stops the pipeline and the producer waits
 // (bounded) for its copies before the CTA exits.
@@ -411,11 +412,16 @@ indexer_score_kernel(const IdxArgs A) {
 #pragma unroll
                         for (int h = 0; h < 4; ++h) score += wq[qq][h] * fmaxf(0.0f, sig[hf] * acc[qq * 4 + h]);
                         st_policy(srow + qq * A.t_cap, score, pol_keep);
-                        if (t <= cur_T - Sq + qq) {
-                            const uint32_t bin = float_key(score) >> kTopkDigitShift;
+                        // Scores crowd into few bins: lanes with the same bin add
+                        // their count with one atomic (the lowest such lane).
+                        const bool live = t <= cur_T - Sq + qq;
+                        const uint32_t bin = live ? float_key(score) >> kTopkDigitShift : 0xFFFFFFFFu;
+                        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+                        if (live && __ffs(peers) - 1 == lane) {
                             const int hr = hrow0 + qq;
-                            if (hr < kRows) atomicAdd(&sm.hist[hr * kTopkBins + bin], 1u);
-                            else atomicAdd(&A.hist[(static_cast<int64_t>(cur_b) * Sq + qq) * kTopkBins + bin], 1u);
+                            const uint32_t n = __popc(peers);
+                            if (hr < kRows) atomicAdd(&sm.hist[hr * kTopkBins + bin], n);
+                            else atomicAdd(&A.hist[(static_cast<int64_t>(cur_b) * Sq + qq) * kTopkBins + bin], n);
                         }
                     }
                 }

@@ -28,16 +28,19 @@ quant_kv_fp4_kernel(const uint4 *__restrict__ x, int64_t n_tok, const int32_t *_
     const int64_t tok = gid / kGroups;
     const int g = static_cast<int>(gid - tok * kGroups);
     if (tok >= n_tok) return;
+    // 16 bf16 channels = two 16-byte vectors, loaded together with the slot
+    // id (the input rows exist for every token, padding included).
+    const uint4 v0 = x[(tok * kGroups + g) * 2 + 0];
+    const uint4 v1 = x[(tok * kGroups + g) * 2 + 1];
+    const bool key_part = kidx_in != nullptr && g < 4;          // threads 0..3 of a token move its indexer key
+    const uint4 kin = key_part ? kidx_in[tok * 4 + g] : make_uint4(0u, 0u, 0u, 0u);
+    const float ksig = (key_part && g == 0) ? ksig_in[tok] : 0.0f;
     const int32_t slot = slots[tok];
     if (slot < 0) return;                       // padding token: nothing to append
     if (static_cast<int64_t>(slot) >= n_slots) {
         if (g == 0) flag_status(kStatusBounds);
         return;
     }
-
-    // 16 bf16 channels = two 16-byte vectors.
-    const uint4 v0 = x[(tok * kGroups + g) * 2 + 0];
-    const uint4 v1 = x[(tok * kGroups + g) * 2 + 1];
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
     float f[16];
 #pragma unroll
@@ -75,12 +78,12 @@ quant_kv_fp4_kernel(const uint4 *__restrict__ x, int64_t n_tok, const int32_t *_
     kv_scale[sl * kScaleBytes + g] = sb;
 
     // Indexer key and scale of the token, in the page's core-matrix order.
-    if (kidx_in != nullptr && g < 4) {
+    if (key_part) {
         const int64_t page = sl / kPage;
         const int r = static_cast<int>(sl % kPage);
         uint8_t *dst = kidx + page * kKidxPageBytes + (r >> 3) * 512 + g * 128 + (r & 7) * 16;
-        *reinterpret_cast<uint4 *>(dst) = kidx_in[tok * 4 + g];
-        if (g == 0) kidx_scale[sl] = ksig_in[tok];
+        *reinterpret_cast<uint4 *>(dst) = kin;
+        if (g == 0) kidx_scale[sl] = ksig;
     }
 }
 

@@ -134,9 +134,22 @@ __device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t *wbuf
 // bins 2047 - 64 l - 63 .. 2047 - 64 l: their sum, a warp scan, then the one
 // lane holding the crossing rescans its bins. Every lane of the warp gets the
 // answer; when the counts fall short of need (corrupt input) it is (0, 0).
+// Histograms read by a warp-level pick are stored with one padding word per
+// 64 bins (bin b at b + b / 64), so that the 32 lanes of the pick, 64 bins
+// apart, fall in 32 different banks.
+__device__ __forceinline__ int hpad(int b) { return b + (b >> 6); }
+constexpr int kTopkBinsPadded = kTopkBins + kTopkBins / 64;
+
+// Warp-level pick over a histogram of nbins (<= 2048, a multiple of 64) bins:
+// the bin holding the need-th largest element (bins scanned from the top) and
+// the count in higher bins. Lane l owns the 64 bins 2047 - 64 l - 63 ..
+// 2047 - 64 l: their sum, a warp scan, then the one lane holding the crossing
+// rescans its bins. kGlobal: a plain [2048] histogram in global memory; else a
+// padded one (hpad) in shared memory. Every lane of the warp gets the answer;
+// when the counts fall short of need (corrupt input) it is (0, 0).
 template <bool kGlobal>
-__device__ __forceinline__ uint4 pick_ld4(const uint32_t *p) {
-    return kGlobal ? __ldcg(reinterpret_cast<const uint4 *>(p)) : *reinterpret_cast<const uint4 *>(p);
+__device__ __forceinline__ uint32_t pick_ld(const uint32_t *h, int b) {
+    return kGlobal ? __ldcg(h + b) : h[hpad(b)];
 }
 
 template <bool kGlobal>
@@ -146,10 +159,15 @@ __device__ __forceinline__ void warp_pick(const uint32_t *h, int nbins, uint32_t
     const int lo = kTopkBins - 64 * (lane + 1);                // this lane's bins: lo .. lo + 63
     uint32_t local = 0u;
     if (lo < nbins) {
+        if (kGlobal) {
 #pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-            const uint4 v = pick_ld4<kGlobal>(h + lo + 4 * i);
-            local += v.x + v.y + v.z + v.w;
+            for (int i = 0; i < 16; ++i) {
+                const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(h + lo) + i);
+                local += v.x + v.y + v.z + v.w;
+            }
+        } else {
+#pragma unroll 8
+            for (int i = 0; i < 64; ++i) local += h[hpad(lo) + i];   // one padded run of 64
         }
     }
     const uint32_t incl = warp_incl_scan(local);
@@ -159,17 +177,13 @@ __device__ __forceinline__ void warp_pick(const uint32_t *h, int nbins, uint32_t
     uint32_t b_out = 0u, a_out = 0u;
     if (mine) {
         uint32_t run = run0;
-        for (int i = 15; i >= 0; --i) {                         // from the top bin down
-            const uint4 v = pick_ld4<kGlobal>(h + lo + 4 * i);
-            const uint32_t c[4] = {v.w, v.z, v.y, v.x};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                if (run < need && run + c[e] >= need) {
-                    b_out = static_cast<uint32_t>(lo + 4 * i + 3 - e);
-                    a_out = run;
-                }
-                run += c[e];
+        for (int i = 63; i >= 0; --i) {                         // from the top bin down
+            const uint32_t c = pick_ld<kGlobal>(h, lo + i);
+            if (run < need && run + c >= need) {
+                b_out = static_cast<uint32_t>(lo + i);
+                a_out = run;
             }
+            run += c;
         }
     }
     const int src = who ? __ffs(who) - 1 : 0;
@@ -183,7 +197,7 @@ struct TkSmem {
     uint32_t ckey[kTkCandCap];          // 48 KB: candidate keys (bin b1)
     int32_t cpos[kTkCandCap];           // 48 KB: candidate positions
     uint32_t hloc[2][kTopkBins];        // this CTA's level-2 / level-3 histograms (read by peers)
-    uint32_t hsum[kTopkBins];           // cluster-wide sum of the current level
+    uint32_t hsum[kTopkBinsPadded];     // cluster-wide sum of the current level (padded, hpad)
     uint32_t wsel[kTkThreads / 32];     // per-warp counts of the emission
     uint32_t wtie[kTkThreads / 32];
     uint32_t xchg[2][2];                // per round parity: (selected before ties, ties), read by peers
@@ -234,9 +248,9 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
         return;                                         // no distributed shared memory was touched
     }
     const int64_t per = (static_cast<int64_t>(n_valid) + C - 1) / C;
-    const int64_t Wn = min(static_cast<int64_t>(kTkWin), (per + 32 * kTkThreads - 1) / (32 * kTkThreads) * (32 * kTkThreads));
-    const int P = static_cast<int>(Wn / kTkThreads);   // positions per thread: 32 .. 128
-    const int NW = P / 32;                              // bitmap words per thread
+    const int64_t Wn = min(static_cast<int64_t>(kTkWin), (per + 31) / 32 * 32);
+    const int NW = static_cast<int>((Wn / 32 + kTkThreads - 1) / kTkThreads);   // bitmap words per thread: 1 .. 4
+    const int P = 32 * NW;                              // positions per thread (threads past Wn have none)
     const int rounds = static_cast<int>((n_valid + C * Wn - 1) / (C * Wn));
     const bool fast = rounds == 1;
     auto win = [&](int r, int64_t &w0, int64_t &w1) {
@@ -335,7 +349,7 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     for (int i = tid; i < kTopkBins; i += kTkThreads) {
         uint32_t v = 0u;
         for (int q = 0; q < C; ++q) v += cluster.map_shared_rank(&sm.hloc[0][0], q)[i];
-        sm.hsum[i] = v;
+        sm.hsum[hpad(i)] = v;
     }
     if (tid == 0) {
         uint32_t of = 0u;
@@ -344,9 +358,17 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     }
     __syncthreads();
     const bool use_list = fast && sm.s_flag == 0u;
-    uint32_t d2, above2;
-    warp_pick<false>(sm.hsum, kTopkBins, need, d2, above2);   // every warp, same answer
-    const uint32_t cnt2 = sm.hsum[d2];
+    if (warp == 0) {
+        uint32_t d, a;
+        warp_pick<false>(sm.hsum, kTopkBins, need, d, a);
+        if (lane == 0) {
+            sm.s_pick[0] = d;
+            sm.s_pick[1] = a;
+        }
+    }
+    __syncthreads();
+    const uint32_t d2 = sm.s_pick[0], above2 = sm.s_pick[1];
+    const uint32_t cnt2 = sm.hsum[hpad(static_cast<int>(d2))];
     need -= above2;
     uint32_t prefix = (static_cast<uint32_t>(b1) << 11) | d2;
     int bits = 22;
@@ -378,11 +400,19 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
         for (int i = tid; i < 1024; i += kTkThreads) {
             uint32_t v = 0u;
             for (int q = 0; q < C; ++q) v += cluster.map_shared_rank(&sm.hloc[1][0], q)[i];
-            sm.hsum[i] = v;
+            sm.hsum[hpad(i)] = v;
         }
         __syncthreads();
-        uint32_t d3, above3;
-        warp_pick<false>(sm.hsum, 1024, need, d3, above3);
+        if (warp == 0) {
+            uint32_t d, a;
+            warp_pick<false>(sm.hsum, 1024, need, d, a);
+            if (lane == 0) {
+                sm.s_pick[0] = d;
+                sm.s_pick[1] = a;
+            }
+        }
+        __syncthreads();
+        const uint32_t d3 = sm.s_pick[0], above3 = sm.s_pick[1];
         need -= above3;
         prefix = (prefix << 10) | d3;
         bits = 32;
