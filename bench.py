@@ -61,6 +61,15 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def tensor_peak():
+    """Burst bf16 dense TFLOP/s (measured cuBLAS), else the fallback 1590."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
@@ -392,6 +401,57 @@ def bulk_quant_leg(args, wl, dw, stream, hbm) -> dict:
         return {"kernel": "csa2_quant_kv_fp4", "error": f"{type(e).__name__}: {e}"[:300]}
 
 
+def replay_leg(args, wl, stream, hbm) -> dict:
+    """csa2_swa_replay_attn (SWA bounded replay): every sequence of the
+    workload recomputes its last 128 window positions, L = 128 queries over a
+    255-row bf16 band. Reports queries/s and both rooflines: HBM (q in, o and
+    lse out, band in) and tensor (QK + PV flops). Events around each launch;
+    an L2 flush before each."""
+    from compressed_sparse_attention_quant_b200 import lib
+    try:
+        B, L = wl.batch, lib.WINDOW
+        g = torch.Generator(device=stream.device).manual_seed(11)
+        q = torch.randn(B, L, lib.HEADS, lib.DIM, device=stream.device, dtype=torch.bfloat16, generator=g)
+        swa = torch.randn(B, lib.WINDOW + L - 1, lib.DIM, device=stream.device, dtype=torch.bfloat16,
+                          generator=g)
+        lens = torch.full((B,), wl.context, dtype=torch.int32, device=stream.device)
+        out = torch.empty(B, L, lib.HEADS, lib.DIM, dtype=torch.float32, device=stream.device)
+        lse = torch.empty(B, L, lib.HEADS, dtype=torch.float32, device=stream.device)
+        scale = 1.0 / lib.DIM ** 0.5
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=stream.device)
+        for _ in range(2):
+            lib.swa_replay_attn(q, swa, lens, scale, out=out, lse=lse)
+        torch.cuda.synchronize()
+        evs = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            lib.swa_replay_attn(q, swa, lens, scale, out=out, lse=lse)
+            e1.record(stream)
+            evs.append((e0, e1))
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+        n_q = B * L
+        nbytes = n_q * lib.HEADS * (lib.DIM * 2 + lib.DIM * 4 + 4) + B * (lib.WINDOW + L - 1) * lib.DIM * 2
+        flops = 4.0 * lib.HEADS * lib.DIM * lib.WINDOW * n_q
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        tfs = flops / (ms * 1e-3) / 1e12
+        bf16_peak, bf16_kind = tensor_peak()
+        del q, swa, out, lse, flush
+        torch.cuda.empty_cache()
+        return {"kernel": "csa2_swa_replay_attn", "sequences": B, "queries_per_sequence": L,
+                "value": n_q / (ms * 1e-3), "unit": "queries/s", "ms_per_launch": ms,
+                "bytes_per_launch": nbytes, "hbm_gbs": gbs, "hbm_frac": gbs / hbm,
+                "flops_per_launch": flops, "tflops": tfs, "tensor_peak_tflops": bf16_peak,
+                "tensor_frac": tfs / bf16_peak,
+                "tensor_peak_kind": bf16_kind, "device_status": lib.status_string(lib.last_device_error()),
+                "input": "N(0,1) bf16 queries and band, every row inside the sequence"}
+    except Exception as e:
+        return {"kernel": "csa2_swa_replay_attn", "error": f"{type(e).__name__}: {e}"[:300]}
+
+
 def run_gpu(args, wl):
     from compressed_sparse_attention_quant_b200 import lib, workload
 
@@ -606,6 +666,7 @@ def run_gpu(args, wl):
     if world == 1:
         line["indexer_pool_topk"] = pool_leg(args, wl, dw, lib, flush, stream, hbm)
         line["kv_quant_bulk"] = bulk_quant_leg(args, wl, dw, stream, hbm)
+        line["swa_replay"] = replay_leg(args, wl, stream, hbm)
     if world == 1 and not args.no_other_workloads:
         del dw, g
         torch.cuda.empty_cache()

@@ -17,8 +17,8 @@
 // K4, one CTA = 9 warps; warp w owns the 64-channel unit [64 w, 64 w + 64)
 // (scale groups 4w .. 4w + 3) of every key, query head and output:
 //   staging  cp.async copies of the packed FP4 records and scales (or the bf16
-//            window rows) of step i + 3 into a 4-stage ring, zero-filled for
-//            empty keys. Physical slots (top-k index -> page table) are
+//            window rows) of step i + 4 into the stage step i has just
+//            released (4-stage ring), zero-filled for empty keys. Physical slots (top-k index -> page table) are
 //            resolved a chunk of 8 steps ahead, each load issued two steps
 //            before its value is used.
 //   QK       lane (g, tig) converts keys g and g + 8 of the step straight into
@@ -42,8 +42,8 @@
 //            with a per-warp power-of-two exponent.
 // Warp-level mma.sync is used deliberately: with 16 heads the MMA N extent is
 // 16, and at that width the warp MMAs issue faster than tcgen05 single-thread
-// MMAs. Three barriers per step: the staged data, the partial scores and the
-// probabilities are complete.
+// MMAs. Two barriers per step: the partial scores are complete (and the step's
+// stage is free), and the probabilities together with the next step's stage.
 #pragma once
 
 #include "common.cuh"
@@ -58,7 +58,6 @@ constexpr int kAttStageBytes = kAttStepKeys * kDim * 2;       // 18,432: 16 wind
 constexpr int kAttRecBytes = kAttStepKeys * kFp4Bytes;        // 4,608: 16 packed FP4 records
 constexpr int kAttScaleWin = 48;                              // 16-byte aligned window holding 36 scale bytes
 constexpr int kAttStages = 4;
-constexpr int kAttAhead = kAttStages - 1;                     // steps staged ahead of the one computed
 constexpr int kAttChunkSteps = 8;                             // steps per slot-resolution chunk
 constexpr int kAttChunkKeys = kAttChunkSteps * kAttStepKeys;  // 128 (threads 0..127 resolve one key each)
 constexpr int kAttUnit = 64;                                  // channels per warp
@@ -353,12 +352,14 @@ sparse_attn_kernel(const AttParams P) {
         if (tid < kAttChunkKeys) sm.slot[0][tid] = slot;
     }
     __syncthreads();
-    // the issue pointer (row, step) runs kAttAhead steps ahead of the compute pointer
+    // the issue pointer (row, step) runs kAttStages steps ahead of the compute pointer
     int irow = row, is = s;
-    for (int i = 0; i < kAttAhead; ++i) {
+    for (int i = 0; i < kAttStages; ++i) {
         issue(i, irow, is);
         if (++is == n_st) { is = 0; ++irow; }
     }
+    cp_async_wait<kAttStages - 1>();                    // step 0 has landed (this thread's copies)
+    __syncthreads();                                    // ... everyone's
 
     AttRow cur = att_row(P, row);
     if (cur.T < 0 && tid == 0) flag_status(kStatusBounds);
@@ -389,11 +390,7 @@ sparse_attn_kernel(const AttParams P) {
             }
             sm.slot[(ch + 1) & 1][tid] = slot;
         }
-        issue(i + kAttAhead, irow, is);
-        if (++is == n_st) { is = 0; ++irow; }
-        cp_async_wait<kAttAhead>();                     // step i has landed (this thread's copies)
-        __syncthreads();                                // ... everyone's; slot stores visible
-
+        // step i's stage is complete and visible (barrier at the end of the previous step)
         const int st = i % kAttStages;
         const uint8_t *stg = sm.stage[st];
         const uint32_t vm = sm.vmask[st];
@@ -473,7 +470,10 @@ sparse_attn_kernel(const AttParams P) {
                 vb[ks][h][0] = movmatrix_t(kb[0][ks][h]);
                 vb[ks][h][1] = movmatrix_t(kb[1][ks][h]);
             }
-        __syncthreads();                                // all partial scores are in shared memory
+        __syncthreads();                                // all partial scores are in; step i's stage is free
+        // stage the copies of step i + 4 into the stage step i no longer reads
+        issue(i + kAttStages, irow, is);
+        if (++is == n_st) { is = 0; ++irow; }
 
         // ---- softmax of heads 2 warp, 2 warp + 1 (warps 0..7), one key per lane
         if (warp < kHeads / 2) {
@@ -500,7 +500,8 @@ sparse_attn_kernel(const AttParams P) {
             *reinterpret_cast<__half *>(sm.p16 + sh * 32 + ((((sk >> 3) ^ ((sh >> 2) & 1))) << 4) + (sk & 7) * 2) = ph16;
             if (sk == 0) sm.alpha[sh] = alpha;
         }
-        __syncthreads();                                // probabilities and rescale factors are in
+        cp_async_wait<kAttStages - 1>();                // step i + 1 has landed (this thread's copies)
+        __syncthreads();                                // probabilities, rescale factors, step i + 1's stage are in
 
         // ---- O = alpha O + P V, keeping O in units of 2^k_exp for this step
         {

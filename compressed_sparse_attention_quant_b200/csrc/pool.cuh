@@ -48,6 +48,7 @@ namespace csa2 {
 constexpr int kPoolThreads = 512;
 constexpr int kPoolWarps = kPoolThreads / 32;
 constexpr int kPoolBins = 2048;
+static_assert(kPoolBins == kTopkBins, "the pool shares warp_pick and its padded histogram with K3");
 constexpr int kPoolMax = 32768;                  // largest pool per row
 constexpr int kPoolMaxCluster = 8;
 constexpr int kPoolMaxIt = 8;                    // 16-entry groups per warp held in flight
@@ -56,7 +57,7 @@ struct PoolSmemFixed {
     uint32_t qb[kIdxHeads * kIdxDim / 4];        // the row's query, E4M3 bytes (4 per word)
     float w[kIdxHeads];
     uint32_t hloc[kPoolBins];                    // this CTA's histogram of the current level (read by peers)
-    uint32_t hsum[kPoolBins];                    // cluster-wide sum
+    uint32_t hsum[kTopkBinsPadded];              // cluster-wide sum, padded (hpad) as warp_pick reads it
     uint32_t wcnt[2][kPoolWarps];
     uint32_t xchg[3];                            // (valid entries, selected, ties) of this CTA, read by peers
 };
@@ -264,7 +265,7 @@ pool_topk_kernel(const PoolArgs A) {
             for (int i = tid; i < kPoolBins; i += kPoolThreads) {
                 uint32_t v = 0u;
                 for (int q = 0; q < S; ++q) v += cluster.map_shared_rank(&fs.hloc[0], q)[i];
-                fs.hsum[i] = v;
+                fs.hsum[hpad(i)] = v;
             }
             __syncthreads();
             uint32_t bin, ab;

@@ -45,7 +45,6 @@ constexpr int kTkWin = 1 << 17;                  // positions per CTA window
 constexpr int kTkWinWords = kTkWin / 32;
 constexpr int kTkCandCap = 12288;                // candidates kept in shared memory per CTA
 constexpr int kTkMaxCluster = 16;
-constexpr int kTkUnroll = 4;                     // float4 loads in flight per thread
 
 // Zeroes the per-row level-1 histograms before the indexer accumulates them.
 __global__ void __launch_bounds__(256) topk_zero_kernel(uint4 *__restrict__ p, int64_t n16) {
@@ -295,50 +294,60 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
             cand = bin == b1;
         }
     };
+    // Loads are coalesced: lane L of warp w reads positions wb + 128 j + 4 L
+    // .. + 3 (wb = the warp's first position); the eight lanes 8q .. 8q + 7
+    // of iteration j cover one 32-position bitmap word, which three
+    // shuffles assemble from their 4-bit pieces. The words are the same ones
+    // the owning threads read later.
     for (int r = 0; r < rounds; ++r) {
         int64_t w0, w1;
         win(r, w0, w1);
-        const int64_t t0 = w0 + static_cast<int64_t>(tid) * P;
-        for (int wi = 0; wi < NW; ++wi) {
-            const int64_t pw = t0 + 32 * wi;                 // this word's first position
-            float4 f[8];
+        const int64_t wb = w0 + static_cast<int64_t>(warp) * 32 * P;
+        const int n_it = P / 4;                          // 8 * NW iterations of 128 positions
+        for (int j0 = 0; j0 < n_it; j0 += 4) {
+            float4 f[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) f[u] = tk_load(srow, pw + 4 * u, w1);
-            uint32_t sure_w = 0u, cand_w = 0u;
+            for (int u = 0; u < 4; ++u) f[u] = tk_load(srow, wb + 128 * (j0 + u) + 4 * lane, w1);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
+            for (int u = 0; u < 4; ++u) {
+                const int64_t p = wb + 128 * (j0 + u) + 4 * lane;
                 const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
+                uint32_t sn = 0u, cn = 0u;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     bool su, ca;
                     uint32_t key;
-                    classify(fv[e], pw + 4 * u + e, w1, su, ca, key);
-                    sure_w |= (su ? 1u : 0u) << (4 * u + e);
+                    classify(fv[e], p + e, w1, su, ca, key);
+                    sn |= (su ? 1u : 0u) << e;
                     if (ca) {
-                        cand_w |= 1u << (4 * u + e);
+                        cn |= 1u << e;
                         atomicAdd(&sm.hloc[0][(key >> 10) & (kTopkBins - 1)], 1u);
                     }
                 }
-            }
-            if (fast) sm.sel[tid * NW + wi] = sure_w;
-            // candidates of this word -> the shared list (warp-aggregated
-            // slots); their scores are read again (L1 / L2 hits), so the
-            // loaded vectors do not stay live.
-            const uint32_t cnt = __popc(cand_w);
-            if (fast && __any_sync(0xffffffffu, cnt != 0u)) {
-                const uint32_t incl = warp_incl_scan(cnt);
-                uint32_t base = 0u;
-                if (lane == 31) base = atomicAdd(&sm.n_cand, incl);
-                base = __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
-                uint32_t m = cand_w;
-                while (m) {
-                    const int bit = __ffs(m) - 1;
-                    m &= m - 1u;
-                    if (base < static_cast<uint32_t>(kTkCandCap)) {
-                        sm.ckey[base] = float_key(__ldcg(srow + pw + bit));
-                        sm.cpos[base] = static_cast<int32_t>(pw + bit);
+                if (fast) {
+                    uint32_t sw = sn << (4 * (lane & 7));
+                    sw |= __shfl_xor_sync(0xffffffffu, sw, 1);
+                    sw |= __shfl_xor_sync(0xffffffffu, sw, 2);
+                    sw |= __shfl_xor_sync(0xffffffffu, sw, 4);
+                    if ((lane & 7) == 0) sm.sel[(p - w0) >> 5] = sw;
+                }
+                // candidates of this piece -> the shared list (warp-aggregated slots)
+                const uint32_t cnt = __popc(cn);
+                if (fast && __any_sync(0xffffffffu, cnt != 0u)) {
+                    const uint32_t incl = warp_incl_scan(cnt);
+                    uint32_t base = 0u;
+                    if (lane == 31) base = atomicAdd(&sm.n_cand, incl);
+                    base = __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        if ((cn >> e) & 1u) {
+                            if (base < static_cast<uint32_t>(kTkCandCap)) {
+                                sm.ckey[base] = float_key(fv[e]);
+                                sm.cpos[base] = static_cast<int32_t>(p + e);
+                            }
+                            ++base;
+                        }
                     }
-                    ++base;
                 }
             }
         }
