@@ -7,74 +7,95 @@
 // beside the global compressed state).
 //
 // Work: the key list of a query row is its 128 window rows (none when the
-// caller passes no window) followed by its k selected entries (padded to a
-// multiple of 16), cut into steps of 16 keys.
-// The steps of all rows form one flat sequence that is split into equal
-// contiguous ranges, one per CTA (persistent: about two CTAs per SM). A CTA
-// writes a row's result directly when its range covers the whole row, else an
-// unnormalised partial (m, l, O) of its first or last row; K5 merges those.
+// caller passes no window) followed by its k selected entries, cut into
+// blocks of 128 keys. The blocks of all rows form one flat sequence that is
+// split into equal contiguous ranges, one per CTA (persistent, one CTA per
+// SM). A CTA writes a row's result directly when its range covers the whole
+// row, else an unnormalised partial (m, l, O) of its first or last row; K5
+// merges those.
 //
-// K4, one CTA = 9 warps; warp w owns the 64-channel unit [64 w, 64 w + 64)
-// (scale groups 4w .. 4w + 3) of every key, query head and output:
-//   staging  cp.async copies of the packed FP4 records and scales (or the bf16
-//            window rows) of step i + 4 into the stage step i has just
-//            released (4-stage ring), zero-filled for empty keys. Physical slots (top-k index -> page table) are
-//            resolved a chunk of 8 steps ahead, each load issued two steps
-//            before its value is used.
-//   QK       lane (g, tig) converts keys g and g + 8 of the step straight into
-//            m16n8k16 B fragments: in k-step s it takes channels
-//            16 tig + 4 s .. + 3 of the unit, so its four k-steps are one
-//            8-byte load and one scale; the query fragments (held in
-//            registers for the row) use the same order, so each product
-//            q_c k_c is summed once. FP4 -> f16 is the hardware E2M1x2
-//            conversion times the E4M3 scale (exact in f16); the window's
-//            bf16 -> f16 goes through a per-warp power-of-two exponent that
-//            keeps it in range.
-//   softmax  the nine warps' partial scores meet in shared memory; warp w < 8
-//            sums them for heads 2w, 2w + 1 (one key per lane) and runs the
-//            online softmax of those heads (exp2 domain, exact running
-//            maximum, probabilities rounded to f16, the same values feed the
-//            sum), writing the f16 probabilities and the rescale factors.
-//   PV       movmatrix transposes the key fragments of QK into the value
-//            fragments (keys = values), so the value tile never goes to
-//            shared memory; the probabilities are the A operand (ldmatrix).
-//            The O accumulator (16 heads x 64 channels) stays in registers
-//            with a per-warp power-of-two exponent.
-// Warp-level mma.sync is used deliberately: with 16 heads the MMA N extent is
-// 16, and at that width the warp MMAs issue faster than tcgen05 single-thread
-// MMAs. Two barriers per step: the partial scores are complete (and the step's
-// stage is free), and the probabilities together with the next step's stage.
+// K4 runs both products on the tensor cores (tcgen05, accumulators in tensor
+// memory), with the keys as the MMA's M side so that the 16 heads are its N:
+//   S^T [128 keys x 16 heads] = K [keys x 576] . Q^T        (36 MMAs, K = 16)
+//   O^T [576 x 16] += V^T [576 x keys] . P^T [keys x 16]    (5 x 8 MMAs)
+// Keys are values, so one f16 tile of the block serves both: it is stored as
+// 72 slabs of 128 keys x 8 channels (16 bytes per key), which is the K-major
+// operand layout of the QK product and the MN-major one of the PV product.
+// The fifth 128-channel tile of O reads 64 channels past the end of the slab
+// tile; those rows of its accumulator are never read.
+//   producers (warps 4..7, one key each): gather the block's packed FP4
+//            records by bulk copy into a staging buffer one block ahead,
+//            convert E2M1 x E4M3 scale to f16 (exact in f16) into the slab
+//            tile, group by group of 128 channels as the previous block's PV
+//            releases each group; window rows are bf16 and are copied into
+//            the tile unchanged (cp.async, zero-filled before position 0).
+//            At a row's first block they stage its query twice: bf16 as is
+//            (for the window block) and f16 under a power-of-two exponent
+//            that keeps it in range (for the FP4 blocks).
+//   MMA      (warp 8, one thread): QK of the block as its groups arrive, one
+//            commit; after the probabilities, PV tile by tile, one commit per
+//            tile (each releases that channel group to the producers).
+//   softmax  (warps 0..3, one key per thread, the block's S row from tensor
+//            memory): exp2 domain, exact running maximum per head (a block
+//            whose maximum rises rescales O in tensor memory first),
+//            probabilities rounded to f16 (FP4 blocks) or split into two bf16
+//            terms hi + lo (the window block, bf16 operands), and the sum of
+//            exactly the values the MMA uses. At the end of a row segment
+//            they read O from tensor memory and write the result or partial.
+// Every wait is an mbarrier wait with a time limit.
 #pragma once
 
 #include "common.cuh"
 
 namespace csa2 {
 
-constexpr int kAttWarps = 9;                                   // one 64-channel unit each
-constexpr int kAttThreads = kAttWarps * 32;                    // 288
-constexpr int kAttStepKeys = 16;
-constexpr int kAttWinSteps = kWindow / kAttStepKeys;          // 8
-constexpr int kAttStageBytes = kAttStepKeys * kDim * 2;       // 18,432: 16 window rows of bf16
-constexpr int kAttRecBytes = kAttStepKeys * kFp4Bytes;        // 4,608: 16 packed FP4 records
-constexpr int kAttScaleWin = 48;                              // 16-byte aligned window holding 36 scale bytes
-constexpr int kAttStages = 4;
-constexpr int kAttChunkSteps = 8;                             // steps per slot-resolution chunk
-constexpr int kAttChunkKeys = kAttChunkSteps * kAttStepKeys;  // 128 (threads 0..127 resolve one key each)
-constexpr int kAttUnit = 64;                                  // channels per warp
-static_assert(kAttWarps * kAttUnit == kDim, "nine 64-channel units");
+constexpr int kAttBlk = 128;                                   // keys per block (MMA M)
+constexpr int kAttSoftWarps = 4;                               // warps 0..3
+constexpr int kAttProdWarps = 4;                               // warps 4..7
+constexpr int kAttMmaWarp = 8;
+constexpr int kAttThreads = 9 * 32;                            // 288
+constexpr int kAttGroups = 5;                                  // channel groups of 128 (the last holds 64)
+constexpr int kAttSlab = kAttBlk * 16;                         // 2,048: 128 keys x 8 channels of 16 bits
+constexpr int kAttTileBytes = (kDim / 8) * kAttSlab;           // 147,456
+constexpr int kAttQBytes = kHeads * kDim * 2;                  // 18,432
+constexpr int kAttPBytes = kAttBlk * kHeads * 2;               // 4,096
+constexpr int kAttRawStride = 304;                             // 288-byte record + 16 (conflict-free 16-byte reads)
+constexpr int kAttRawBytes = kAttBlk * kAttRawStride;          // 38,912
+constexpr int kAttTmemCols = 128;
+constexpr int kAttSCol = 0;                                    // S^T: 16 columns
+constexpr int kAttOCol = 16;                                   // O^T: 5 tiles x 16 columns
+constexpr uint32_t kIdescBf16 = (1u << 7) | (1u << 10);        // A and B format BF16 (kind::f16)
+// Operand strides (bytes between adjacent 8 x 16-byte core matrices).
+// K-major: LBO = along K, SBO = along M/N.
+constexpr uint32_t kTileLboK = kAttSlab, kTileSboK = 128;      // A of QK: channel groups / key groups
+constexpr uint32_t kQLbo = 256, kQSbo = 128;                   // B of QK: channel groups / head groups
+// MN-major: LBO = along K, SBO = along M/N.
+constexpr uint32_t kTileLboMN = 128, kTileSboMN = kAttSlab;    // A of PV: key groups / channel groups
+constexpr uint32_t kPLbo = 256, kPSbo = 128;                   // B of PV: key groups / head groups
 
 struct AttSmem {
-    alignas(128) uint8_t stage[kAttStages][kAttStageBytes];   // 73,728
-    float4 spart[2][kAttWarps][2][32];                        // 18,432: partial scores per warp
-    alignas(16) uint8_t p16[kHeads * kAttStepKeys * 2];       // 512: f16 probabilities [head][key], chunks swizzled
-    float alpha[kHeads];                                      // rescale of O for this step, per head
-    float l_fin[kHeads];                                      // running sum, m_fin: running max (segment end)
-    float m_fin[kHeads];
-    int slot[2][kAttChunkKeys];                               // physical slots of two chunks
-    uint8_t soff[kAttStages][kAttStepKeys];                   // scale offset inside the 48-byte window
-    uint32_t vmask[kAttStages];                               // valid keys of a staged step
+    alignas(128) uint8_t tile[kAttTileBytes];                 // f16 (FP4 block) or bf16 (window) keys
+    alignas(16) uint8_t qf[kAttQBytes];                        // must follow the tile (read past its end)
+    alignas(16) uint8_t qb[kAttQBytes];
+    alignas(16) uint8_t p_hi[kAttPBytes];
+    alignas(16) uint8_t p_lo[kAttPBytes];
+    alignas(16) uint8_t raw[kAttRawBytes];                     // packed FP4 records of the next block
+    uint64_t deq_done[kAttGroups];                             // producers -> MMA (group t of the tile is in)
+    uint64_t pv_done[kAttGroups];                              // MMA -> producers, softmax (PV tile t done)
+    uint64_t s_full;                                           // MMA -> softmax (S of the block)
+    uint64_t p_ready;                                          // softmax -> MMA (P, rescaled O)
+    uint64_t raw_full;                                         // bulk copies -> producers
+    uint64_t drain;
+    uint32_t tmem_base;
+    uint32_t mask[2][4];                                       // valid keys of a block, by block parity
+    int eq[2];                                                 // query exponent of a block
+    float qmax[2][kAttProdWarps];
+    float red_m[kAttSoftWarps][kHeads];
+    float red_l[kAttSoftWarps][kHeads];
 };
 constexpr size_t kAttSmemBytes = sizeof(AttSmem);
+static_assert(offsetof(AttSmem, qf) == kAttTileBytes, "the PV tail tile reads on into qf");
+static_assert(kAttSmemBytes <= 232448, "one CTA per SM");
 
 struct AttParams {
     const __nv_bfloat16 *q;        // [R][16][576]
@@ -93,28 +114,22 @@ struct AttParams {
     float *lse;                    // [R][16]
     float *part_o;                 // [2 * grid][16][576]
     float2 *part_ml;               // [2 * grid][16]: (m in the log2 domain, l)
-    int n_win;                     // window steps per row: 8 (128 rows), or 0 without a window
-    int n_st;                      // steps per row: n_win + ceil(k / 16)
+    int n_win;                     // window blocks per row: 1, or 0 without a window
+    int n_st;                      // blocks per row: n_win + ceil(k / 128)
     int64_t total_steps;           // R * n_st
 };
 
-// First step of CTA c's range (the same formula on host and device).
+// First block of CTA c's range (the same formula on host and device).
 __host__ __device__ __forceinline__ int64_t att_range_start(int64_t total, int c, int grid) {
     return total * c / grid;
 }
 
-// CTA whose range holds step s.
+// CTA whose range holds block s.
 __host__ __device__ __forceinline__ int att_cta_of(int64_t total, int64_t s, int grid) {
     int c = static_cast<int>(s * grid / total);
     while (c + 1 < grid && att_range_start(total, c + 1, grid) <= s) ++c;
     while (c > 0 && att_range_start(total, c, grid) > s) --c;
     return c;
-}
-
-__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
-    uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-    return y;
 }
 
 // bf16x2 -> f32 pair (exact).
@@ -137,7 +152,7 @@ __device__ __forceinline__ int f16_exponent(float m) {
     return max(-100, min(100, e));
 }
 
-// Row state of a query row resolved once per segment.
+// Row state of a query row.
 struct AttRow {
     int row, b, j, T, pos;   // T < 0: no valid key at all
 };
@@ -153,399 +168,518 @@ __device__ __forceinline__ AttRow att_row(const AttParams &P, int row) {
     return r;
 }
 
-__global__ void __maxnreg__(104)
-sparse_attn_kernel(const AttParams P) {
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    AttSmem &sm = *reinterpret_cast<AttSmem *>(smem_raw);
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, tig = lane & 3;
-    const int grid = static_cast<int>(gridDim.x);
-    const int64_t st0 = att_range_start(P.total_steps, blockIdx.x, grid);
-    const int n_my = static_cast<int>(att_range_start(P.total_steps, blockIdx.x + 1, grid) - st0);
-    const int n_st = P.n_st;
-    const int n_rows_swa = kWindow + P.Sq - 1;
-    const int cbase = warp * kAttUnit;                 // this warp's first channel
+// Block i of a CTA's range.
+struct AttBlk {
+    int row, j;        // query row, block of the row
+    bool win;          // the window block
+    int e0, n;         // first selected entry, keys in the block
+    bool first, last;  // first / last block of a row segment of this CTA
+};
 
-    // ------------------------------------------------ staging helpers
-    // (row, step-in-row) of CTA step i, by division (used once per chunk).
-    auto step_of = [&](int i, int &row, int &s) {
-        const int64_t gs = st0 + i;
-        row = static_cast<int>(gs / n_st);
-        s = static_cast<int>(gs - static_cast<int64_t>(row) * n_st);
-    };
-    // Top-k index of key t (< 128) of chunk ch, or -1 (window step, padding, past the range).
-    auto load_idx = [&](int ch, int t, int &row_out) -> int {
-        row_out = -1;
-        const int i = ch * kAttChunkSteps + t / kAttStepKeys;
-        if (t >= kAttChunkKeys || i >= n_my) return -1;
-        int row, s;
-        step_of(i, row, s);
-        if (s < P.n_win) return -1;
-        const int e = (s - P.n_win) * kAttStepKeys + (t % kAttStepKeys);
-        if (e >= P.k) return -1;
-        row_out = row;
-        return P.topk_idx[static_cast<int64_t>(row) * P.k + e];
-    };
-    // Issue the copies of CTA step i (its row and step given) into its stage (one commit group).
-    auto issue = [&](int i, int row, int s) {
-        if (i < n_my) {
-            const int st = i % kAttStages;
-            uint8_t *dst = sm.stage[st];
-            if (s < P.n_win) {
-                // 16 window rows: 16 x 72 chunks of 16 bytes, chunk c of key e
-                // at position c ^ (e & 7) (conflict-free reads).
-                const AttRow r = att_row(P, row);
-                const int first = r.pos - (kWindow - 1) + s * kAttStepKeys;   // position of key 0
-                const __nv_bfloat16 *src0 =
-                    P.swa + (static_cast<int64_t>(r.b) * n_rows_swa + r.j + s * kAttStepKeys) * kDim;
-                for (int c = tid; c < kAttStepKeys * (kDim / 8); c += kAttThreads) {
-                    const int e = c / (kDim / 8), ch = c - e * (kDim / 8);
-                    const bool ok = r.T >= 0 && first + e >= 0;
-                    const uint8_t *src = reinterpret_cast<const uint8_t *>(ok ? src0 + e * kDim + ch * 8 : P.swa);
-                    cp_async16(dst + e * (kDim * 2) + ((ch ^ (e & 7)) << 4), src, ok ? 16u : 0u);
-                }
-                if (warp == 0) {
-                    const bool v = lane < kAttStepKeys && r.T >= 0 && first + lane >= 0;
-                    const uint32_t m = __ballot_sync(0xffffffffu, v);
-                    if (lane == 0) sm.vmask[st] = m;
-                }
-            } else {
-                // 16 FP4 records (18 chunks each) + 16 scale windows (3 chunks).
-                const int *sl = sm.slot[(i / kAttChunkSteps) & 1] + (i % kAttChunkSteps) * kAttStepKeys;
-                for (int c = tid; c < kAttStepKeys * 21; c += kAttThreads) {
-                    const int e = c / 21, part = c - e * 21;
-                    const int slot = sl[e];
-                    if (part < 18) {
-                        const uint8_t *src = slot >= 0 ? P.kv_fp4 + static_cast<int64_t>(slot) * kFp4Bytes + part * 16
-                                                       : P.kv_fp4;
-                        cp_async16(dst + e * kFp4Bytes + part * 16, src, slot >= 0 ? 16u : 0u);
-                    } else {
-                        const int64_t sb = static_cast<int64_t>(slot) * kScaleBytes;
-                        const uint8_t *src = slot >= 0 ? P.kv_scale + (sb & ~static_cast<int64_t>(15)) + (part - 18) * 16
-                                                       : P.kv_scale;
-                        cp_async16(dst + kAttRecBytes + e * kAttScaleWin + (part - 18) * 16, src, slot >= 0 ? 16u : 0u);
-                        if (part == 18) sm.soff[st][e] = static_cast<uint8_t>(slot >= 0 ? (sb & 15) : 0);
-                    }
-                }
-                if (warp == 0) {
-                    const uint32_t m = __ballot_sync(0xffffffffu, lane < kAttStepKeys && sl[lane & 15] >= 0);
-                    if (lane == 0) sm.vmask[st] = m;
-                }
-            }
-        }
-        cp_async_commit();
-    };
+__device__ __forceinline__ AttBlk att_blk(const AttParams &P, int64_t b0, int nblk, int i) {
+    AttBlk k;
+    const int64_t gb = b0 + i;
+    k.row = static_cast<int>(gb / P.n_st);
+    k.j = static_cast<int>(gb - static_cast<int64_t>(k.row) * P.n_st);
+    k.win = k.j < P.n_win;
+    k.e0 = k.win ? 0 : (k.j - P.n_win) * kAttBlk;
+    k.n = k.win ? kAttBlk : min(kAttBlk, P.k - k.e0);
+    k.first = i == 0 || k.j == 0;
+    k.last = i == nblk - 1 || k.j == P.n_st - 1;
+    return k;
+}
 
-    // ------------------------------------------------ per-row (segment) state
-    uint32_t qa[4][4];          // query fragments (heads g, g + 8) of this warp's unit
-    float q_mul = 1.0f;         // 2^eq: query exponent of this warp
-    float o[8][4];              // O accumulator (heads g, g + 8 x the unit), units of 2^o_exp
-    int o_exp = 0;
-    float m_run = -INFINITY, l_run = 0.0f;   // softmax lanes: head 2 warp + (lane >> 4)
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
 
-    auto load_query = [&](int row) {
-        const __nv_bfloat16 *qr = P.q + static_cast<int64_t>(row) * kHeads * kDim;
-        uint4 v[2][2];
-        float mx = 0.0f;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            const uint4 *hp = reinterpret_cast<const uint4 *>(qr + (g + 8 * hh) * kDim + cbase + 16 * tig);
-            v[hh][0] = __ldg(hp);
-            v[hh][1] = __ldg(hp + 1);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float2 f = bf16x2_f32((&v[hh][0].x)[i]);
-                mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        const int eq = f16_exponent(mx);
-        const float sdown = exp2f(static_cast<float>(-eq));
-        q_mul = exp2f(static_cast<float>(eq));
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            // k-step s takes channels 16 tig + 4 s .. + 3 (words 2s, 2s + 1 of the lane's 16 channels)
-#pragma unroll
-            for (int st = 0; st < 4; ++st) {
-                const float2 a = bf16x2_f32((&v[hh][0].x)[2 * st]), c = bf16x2_f32((&v[hh][0].x)[2 * st + 1]);
-                qa[st][hh] = f32x2_f16x2(a.x * sdown, a.y * sdown);        // a0 / a1
-                qa[st][2 + hh] = f32x2_f16x2(c.x * sdown, c.y * sdown);    // a2 / a3
-            }
-        }
-    };
-    auto reset_row = [&]() {
-#pragma unroll
-        for (int n = 0; n < 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.0f;
-        o_exp = 0;
-        m_run = -INFINITY;
-        l_run = 0.0f;
-    };
-    // Result of the segment [s_first, s_last] of row r (all threads).
-    auto finish_row = [&](const AttRow &r, int s_first, int s_last, int part_slot) {
-        if (warp < kHeads / 2 && (lane & 15) == 0) {
-            const int h = 2 * warp + (lane >> 4);
-            sm.l_fin[h] = l_run;
-            sm.m_fin[h] = m_run;
-        }
-        __syncthreads();
-        const float l0 = sm.l_fin[g], l1 = sm.l_fin[g + 8];
-        const float omul = exp2f(static_cast<float>(o_exp));
-        const bool whole = s_first == 0 && s_last == n_st - 1;
-        float *dst;
-        float mul[2];
-        if (whole) {
-            dst = P.out + static_cast<int64_t>(r.row) * kHeads * kDim;
-            mul[0] = l0 > 0.0f ? omul / l0 : 0.0f;
-            mul[1] = l1 > 0.0f ? omul / l1 : 0.0f;
-        } else {
-            dst = P.part_o + static_cast<int64_t>(part_slot) * kHeads * kDim;
-            mul[0] = mul[1] = omul;
-        }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float *hrow = dst + (g + 8 * hh) * kDim + cbase + 16 * tig;
-#pragma unroll
-            for (int st = 0; st < 4; ++st) {
-                const int n = 2 * st;
-                *reinterpret_cast<float4 *>(hrow + 4 * st) =
-                    make_float4(o[n][2 * hh] * mul[hh], o[n][2 * hh + 1] * mul[hh], o[n + 1][2 * hh] * mul[hh],
-                                o[n + 1][2 * hh + 1] * mul[hh]);
-            }
-        }
-        if (tid < kHeads) {
-            const float l = sm.l_fin[tid], m = sm.m_fin[tid];
-            if (whole)
-                P.lse[static_cast<int64_t>(r.row) * kHeads + tid] =
-                    l > 0.0f ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
-            else
-                P.part_ml[static_cast<int64_t>(part_slot) * kHeads + tid] = make_float2(m, l);
-        }
-    };
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+          "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-    if (n_my <= 0) return;                              // no work (uniform)
+__device__ __forceinline__ void named_bar(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
-    // ------------------------------------------------ prologue
-    // The query, window rows, lengths and page table are inputs no earlier
-    // kernel of the step writes: the first row's query fragments load before
-    // the wait for the selection.
-    int row, s;
-    step_of(0, row, s);
-    load_query(row);
-    reset_row();
-    pdl_wait();                                         // the top-k indices are ready
-    pdl_trigger();
+// Bulk global -> shared copy completing on an mbarrier (default L2 policy).
+__device__ __forceinline__ void bulk_g2s_plain(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+// Reduction of 16 per-lane values over the warp's 32 lanes, one head per
+// lane pair: lane L returns the result for head L >> 1 (16 shuffles).
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce16(const float (&v)[16]) {
+    const int lane = threadIdx.x & 31;
+    auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
+    float a[8], b[4], c[2];
     {
-        int rr;
-        const int idx = load_idx(0, tid, rr);
-        int slot = -1;
-        if (rr >= 0 && idx >= 0) {
-            const AttRow r = att_row(P, rr);
-            if (r.T < 0 || idx > r.pos) {               // past the query (causal) or a bad length
-                flag_status(kStatusBounds);
-            } else {
-                const int64_t ph = P.page_table[static_cast<int64_t>(r.b) * P.max_pages + (idx >> 6)];
-                if (ph < 0 || ph >= P.num_pages) flag_status(kStatusBounds);
-                else slot = static_cast<int>(ph * kPage + (idx & 63));
-            }
-        }
-        if (tid < kAttChunkKeys) sm.slot[0][tid] = slot;
-    }
-    __syncthreads();
-    // the issue pointer (row, step) runs kAttStages steps ahead of the compute pointer
-    int irow = row, is = s;
-    for (int i = 0; i < kAttStages; ++i) {
-        issue(i, irow, is);
-        if (++is == n_st) { is = 0; ++irow; }
-    }
-    cp_async_wait<kAttStages - 1>();                    // step 0 has landed (this thread's copies)
-    __syncthreads();                                    // ... everyone's
-
-    AttRow cur = att_row(P, row);
-    if (cur.T < 0 && tid == 0) flag_status(kStatusBounds);
-    int seg_first = s;                                   // first step of the current segment
-    int seg_no = 0;                                      // segments finished so far
-    int nrow = -1, nidx = -1;                            // slot resolution of the next chunk in flight
-    int64_t npage = -1;
-    const int sh = warp < kHeads / 2 ? 2 * warp + (lane >> 4) : 0;     // softmax head of this lane
-    const int sk = lane & 15;                                          // softmax key of this lane
-
-    for (int i = 0; i < n_my; ++i) {
-        // ---- next chunk's slots: index load, page load, store (two steps apart)
-        const int ch = i / kAttChunkSteps, ph = i % kAttChunkSteps;
-        if (ph == 0) nidx = load_idx(ch + 1, tid, nrow);
-        if (ph == 2) {
-            npage = -1;
-            if (nrow >= 0 && nidx >= 0) {
-                const AttRow r = att_row(P, nrow);
-                if (r.T >= 0 && nidx <= r.pos) npage = P.page_table[static_cast<int64_t>(r.b) * P.max_pages + (nidx >> 6)];
-            }
-        }
-        if (ph == 4 && tid < kAttChunkKeys) {
-            int slot = -1;
-            if (nrow >= 0 && nidx >= 0) {
-                const AttRow r = att_row(P, nrow);
-                if (r.T < 0 || nidx > r.pos || npage < 0 || npage >= P.num_pages) flag_status(kStatusBounds);
-                else slot = static_cast<int>(npage * kPage + (nidx & 63));
-            }
-            sm.slot[(ch + 1) & 1][tid] = slot;
-        }
-        // step i's stage is complete and visible (barrier at the end of the previous step)
-        const int st = i % kAttStages;
-        const uint8_t *stg = sm.stage[st];
-        const uint32_t vm = sm.vmask[st];
-        const bool win = s < P.n_win;
-
-        // ---- key fragments of keys g and g + 8 (n-tiles 0, 1)
-        uint32_t kb[2][4][2];
-        int k_exp = 0;
-        if (!win) {
+        const bool up = lane & 16;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int e = nt * 8 + g;
-                const uint2 rv = *reinterpret_cast<const uint2 *>(stg + e * kFp4Bytes + cbase / 2 + 8 * tig);
-                const uint8_t sc = stg[kAttRecBytes + e * kAttScaleWin + sm.soff[st][e] + 4 * warp + tig];
-                const uint32_t s2 = e4m3x2_to_f16x2(static_cast<uint32_t>(sc) * 0x0101u);
+        for (int i = 0; i < 8; ++i) {
+            const float send = up ? v[i] : v[i + 8], keep = up ? v[i + 8] : v[i];
+            a[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+        }
+    }
+    {
+        const bool up = lane & 8;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t wv = q < 2 ? rv.x : rv.y;
-                    kb[nt][q][0] = hmul2_u32(e2m1x2_to_f16x2((wv >> (16 * (q & 1))) & 0xffu), s2);
-                    kb[nt][q][1] = hmul2_u32(e2m1x2_to_f16x2((wv >> (16 * (q & 1) + 8)) & 0xffu), s2);
-                }
-            }
+        for (int i = 0; i < 4; ++i) {
+            const float send = up ? a[i] : a[i + 4], keep = up ? a[i + 4] : a[i];
+            b[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+        }
+    }
+    {
+        const bool up = lane & 4;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const float send = up ? b[i] : b[i + 2], keep = up ? b[i + 2] : b[i];
+            c[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+        }
+    }
+    const bool up = lane & 2;
+    float d = op(up ? c[1] : c[0], __shfl_xor_sync(0xffffffffu, up ? c[0] : c[1], 2));
+    return op(d, __shfl_xor_sync(0xffffffffu, d, 1));
+}
+
+__device__ __forceinline__ uint32_t slab_off(int key, int cgroup) {
+    return static_cast<uint32_t>(cgroup * kAttSlab + (key >> 3) * 128 + (key & 7) * 16);
+}
+
+// ------------------------------------------------------------------ producers
+// Physical slot of key r of fp4 block i (top-k index idx, its page entry
+// pg), or -1; flags out-of-range data.
+__device__ __forceinline__ int att_slot(const AttParams &P, const AttBlk &k, const AttRow &rw, int r, int idx,
+                                        int64_t pg) {
+    if (r >= k.n || idx < 0) return -1;                  // padding
+    if (rw.T < 0 || idx > rw.pos || pg < 0 || pg >= P.num_pages) {
+        flag_status(kStatusBounds);
+        return -1;
+    }
+    return static_cast<int>(pg * kPage + (idx & 63));
+}
+
+__device__ __forceinline__ bool att_producers(const AttParams &P, AttSmem &sm, int64_t b0, int nblk) {
+    const int r = threadIdx.x - kAttSoftWarps * 32;       // key of the block
+    const int pw = r >> 5, lane = r & 31;
+    const int n_rows_swa = kWindow + P.Sq - 1;
+    const uint32_t mykey = static_cast<uint32_t>((r >> 3) * 128 + (r & 7) * 16);
+    auto next_fp4 = [&](int i) {
+        while (i < nblk && att_blk(P, b0, nblk, i).win) ++i;
+        return i;
+    };
+    auto load_idx = [&](int i) -> int {
+        if (i >= nblk) return -1;
+        const AttBlk k = att_blk(P, b0, nblk, i);
+        return r < k.n ? __ldg(P.topk_idx + static_cast<int64_t>(k.row) * P.k + k.e0 + r) : -1;
+    };
+    auto load_page = [&](int i, int idx) -> int64_t {
+        if (i >= nblk || idx < 0) return -1;
+        const AttBlk k = att_blk(P, b0, nblk, i);
+        const AttRow rw = att_row(P, k.row);
+        if (rw.T < 0 || idx > rw.pos) return -1;
+        return __ldg(P.page_table + static_cast<int64_t>(rw.b) * P.max_pages + (idx >> 6));
+    };
+    auto resolve = [&](int i, int idx, int64_t pg) -> int {
+        if (i >= nblk) return -1;
+        const AttBlk k = att_blk(P, b0, nblk, i);
+        return att_slot(P, k, att_row(P, k.row), r, idx, pg);
+    };
+    uint32_t sc_next[9];
+    auto issue = [&](int slot) {                          // copy + scales of this key's next record
+        if (slot >= 0) {
+            mbar_arrive_expect_tx(&sm.raw_full, kFp4Bytes);
+            bulk_g2s_plain(sm.raw + r * kAttRawStride, P.kv_fp4 + static_cast<int64_t>(slot) * kFp4Bytes, kFp4Bytes,
+                           &sm.raw_full);
+            const uint32_t *sp = reinterpret_cast<const uint32_t *>(P.kv_scale + static_cast<int64_t>(slot) * kScaleBytes);
+#pragma unroll
+            for (int u = 0; u < 9; ++u) sc_next[u] = __ldg(sp + u);
         } else {
-            // bf16 window rows: read, take this warp's maximum, convert under
-            // the exponent that keeps them in f16 range.
-            uint4 w4[2][2];
+            mbar_arrive(&sm.raw_full);
+#pragma unroll
+            for (int u = 0; u < 9; ++u) sc_next[u] = 0u;  // zero scale: the key's tile row is zero
+        }
+    };
+    // pipeline: the next fp4 block's copy is in flight; the one after has its top-k index loaded
+    int f1 = next_fp4(0);
+    int slot1 = -1;
+    if (f1 < nblk) {
+        const int idx = load_idx(f1);
+        slot1 = resolve(f1, idx, load_page(f1, idx));
+        issue(slot1);
+    }
+    int f2 = next_fp4(f1 + 1);
+    int idx2 = load_idx(f2);
+    uint32_t raw_par = 0u;
+    int eq = 0, qrow_par = 0;
+
+    for (int i = 0; i < nblk; ++i) {
+        const AttBlk k = att_blk(P, b0, nblk, i);
+        const AttRow rw = att_row(P, k.row);
+        const uint32_t pp = static_cast<uint32_t>((i - 1) & 1);
+        if (k.first) {
+            // ---- the row's query: bf16 copy and f16 copy under exponent eq
+            if (rw.T < 0 && r == 0) flag_status(kStatusBounds);
+            const __nv_bfloat16 *qr = P.q + static_cast<int64_t>(k.row) * kHeads * kDim;
+            uint4 qv[9];
             float mx = 0.0f;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const int e = nt * 8 + g;
-                const uint8_t *rowp = stg + e * (kDim * 2);
-                const int c0 = (cbase + 16 * tig) / 8;                     // 16-byte chunk of the lane's channels
-                w4[nt][0] = *reinterpret_cast<const uint4 *>(rowp + ((c0 ^ (e & 7)) << 4));
-                w4[nt][1] = *reinterpret_cast<const uint4 *>(rowp + (((c0 + 1) ^ (e & 7)) << 4));
+            for (int u = 0; u < 9; ++u) {
+                const int c = u * 128 + r, h = c & 15, jg = c >> 4;
+                qv[u] = __ldg(reinterpret_cast<const uint4 *>(qr + h * kDim + 8 * jg));
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const float2 f = bf16x2_f32((&w4[nt][0].x)[q]);
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = bf16x2_f32((&qv[u].x)[e]);
                     mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
                 }
             }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            k_exp = f16_exponent(mx);
-            const float sdown = exp2f(static_cast<float>(-k_exp));
+            if (lane == 0) sm.qmax[qrow_par][pw] = mx;
+            named_bar(2, kAttProdWarps * 32);
+            mx = fmaxf(fmaxf(sm.qmax[qrow_par][0], sm.qmax[qrow_par][1]), fmaxf(sm.qmax[qrow_par][2], sm.qmax[qrow_par][3]));
+            qrow_par ^= 1;
+            eq = f16_exponent(mx);
+            const float sdown = exp2f(static_cast<float>(-eq));
+            // the previous block's QK has read the old query once its PV tile 0 is done
+            if (i > 0 && !mbar_wait_bounded(&sm.pv_done[0], pp)) return false;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int u = 0; u < 9; ++u) {
+                const int c = u * 128 + r, h = c & 15, jg = c >> 4;
+                const uint32_t off = static_cast<uint32_t>(jg * 256 + (h >> 3) * 128 + (h & 7) * 16);
+                *reinterpret_cast<uint4 *>(sm.qb + off) = qv[u];
+                uint32_t hv[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 a = bf16x2_f32((&w4[nt][0].x)[2 * q]), c = bf16x2_f32((&w4[nt][0].x)[2 * q + 1]);
-                    kb[nt][q][0] = f32x2_f16x2(a.x * sdown, a.y * sdown);
-                    kb[nt][q][1] = f32x2_f16x2(c.x * sdown, c.y * sdown);
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = bf16x2_f32((&qv[u].x)[e]);
+                    hv[e] = f32x2_f16x2(f.x * sdown, f.y * sdown);
                 }
-        }
-
-        // ---- partial scores over this warp's unit
-        {
-            float acc[2][4];
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-                    mma_f16_16816(acc[nt], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], kb[nt][ks][0], kb[nt][ks][1]);
-            const float smul = q_mul * exp2f(static_cast<float>(k_exp)) * P.scale_log2;   // undo the exponents
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-                sm.spart[i & 1][warp][nt][lane] =
-                    make_float4(acc[nt][0] * smul, acc[nt][1] * smul, acc[nt][2] * smul, acc[nt][3] * smul);
-        }
-        // value fragments: the key fragments transposed (keys = values)
-        uint32_t vb[4][2][2];
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                vb[ks][h][0] = movmatrix_t(kb[0][ks][h]);
-                vb[ks][h][1] = movmatrix_t(kb[1][ks][h]);
+                *reinterpret_cast<uint4 *>(sm.qf + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
             }
-        __syncthreads();                                // all partial scores are in; step i's stage is free
-        // stage the copies of step i + 4 into the stage step i no longer reads
-        issue(i + kAttStages, irow, is);
-        if (++is == n_st) { is = 0; ++irow; }
-
-        // ---- softmax of heads 2 warp, 2 warp + 1 (warps 0..7), one key per lane
-        if (warp < kHeads / 2) {
-            // partial of (head sh, key sk) sits in lane (sh % 8) * 4 + (sk % 8) / 2 of n-tile sk / 8,
-            // component (sh / 8) * 2 + sk % 2
-            const int L = (sh & 7) * 4 + ((sk & 7) >> 1), nt = sk >> 3, comp = (sh >> 3) * 2 + (sk & 1);
-            float x = 0.0f;
-#pragma unroll
-            for (int w = 0; w < kAttWarps; ++w) x += (&sm.spart[i & 1][w][nt][L].x)[comp];
-            x = ((vm >> sk) & 1u) ? x : -INFINITY;
-            float mx = x;
-#pragma unroll
-            for (int off = 8; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            const float m_new = fmaxf(m_run, mx);
-            const float alpha = (m_run == -INFINITY) ? 1.0f : exp2f(m_run - m_new);   // O and l still zero when -inf
-            const float p = (m_new == -INFINITY || x == -INFINITY) ? 0.0f : exp2f(x - m_new);
-            const __half ph16 = __float2half_rn(p);
-            float ps = __half2float(ph16);
-#pragma unroll
-            for (int off = 8; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-            l_run = l_run * alpha + ps;
-            m_run = m_new;
-            // P[head][key]: 32-byte rows, the two 16-byte chunks swizzled by the head
-            *reinterpret_cast<__half *>(sm.p16 + sh * 32 + ((((sk >> 3) ^ ((sh >> 2) & 1))) << 4) + (sk & 7) * 2) = ph16;
-            if (sk == 0) sm.alpha[sh] = alpha;
         }
-        cp_async_wait<kAttStages - 1>();                // step i + 1 has landed (this thread's copies)
-        __syncthreads();                                // probabilities, rescale factors, step i + 1's stage are in
-
-        // ---- O = alpha O + P V, keeping O in units of 2^k_exp for this step
-        {
-            const float ex = exp2f(static_cast<float>(o_exp - k_exp));
-            const float a0 = sm.alpha[g] * ex, a1 = sm.alpha[g + 8] * ex;
-            if (__any_sync(0xffffffffu, a0 != 1.0f || a1 != 1.0f)) {
+        if (!k.win) {
+            // ---- FP4 block: its records are (being) staged; resolve the one after next
+            const int64_t pg2 = load_page(f2, idx2);
+            uint32_t sc[9];
 #pragma unroll
-                for (int n = 0; n < 8; ++n) {
-                    o[n][0] *= a0;
-                    o[n][1] *= a0;
-                    o[n][2] *= a1;
-                    o[n][3] *= a1;
+            for (int u = 0; u < 9; ++u) sc[u] = sc_next[u];
+            const bool valid = slot1 >= 0;
+            if (!mbar_wait_bounded(&sm.raw_full, raw_par)) return false;
+            raw_par ^= 1u;
+            const uint8_t *rr = sm.raw + r * kAttRawStride;
+#pragma unroll
+            for (int t = 0; t < kAttGroups; ++t) {
+                if (i > 0 && !mbar_wait_bounded(&sm.pv_done[t], pp)) return false;
+#pragma unroll
+                for (int m = 4 * t; m < (t < 4 ? 4 * t + 4 : 18); ++m) {     // channels 32m .. 32m + 31
+                    const uint4 v = *reinterpret_cast<const uint4 *>(rr + 16 * m);
+                    const uint32_t s2 = e4m3x2_to_f16x2((sc[m >> 1] >> (16 * (m & 1))) & 0xffffu);
+                    const uint32_t sa = (s2 & 0xffffu) | (s2 << 16), sb = (s2 >> 16) | (s2 & 0xffff0000u);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t w = (&v.x)[u], s = u < 2 ? sa : sb;
+                        const uint4 o = make_uint4(hmul2_u32(e2m1x2_to_f16x2(w & 0xffu), s),
+                                                   hmul2_u32(e2m1x2_to_f16x2((w >> 8) & 0xffu), s),
+                                                   hmul2_u32(e2m1x2_to_f16x2((w >> 16) & 0xffu), s),
+                                                   hmul2_u32(e2m1x2_to_f16x2(w >> 24), s));
+                        *reinterpret_cast<uint4 *>(sm.tile + (4 * m + u) * kAttSlab + mykey) = o;
+                    }
                 }
+                if (t == kAttGroups - 1) {
+                    const uint32_t mk = __ballot_sync(0xffffffffu, valid);
+                    if (lane == 0) sm.mask[i & 1][pw] = mk;
+                    if (r == 0) sm.eq[i & 1] = eq;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.deq_done[t]);
             }
-            o_exp = k_exp;
-            uint32_t pa0, pa1, pa2, pa3;
-            const int prow = lane & 15, pch = lane >> 4;
-            ldsm_x4(pa0, pa1, pa2, pa3, sm.p16 + prow * 32 + ((pch ^ ((prow >> 2) & 1)) << 4));
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) mma_f16_16816(o[2 * ks + h], pa0, pa1, pa2, pa3, vb[ks][h][0], vb[ks][h][1]);
-        }
-
-        // ---- segment end: the row ends here or the range does
-        const bool last_of_row = s == n_st - 1;
-        if (last_of_row || i == n_my - 1) {
-            // partial slot: the first segment of the range uses 2c, a later one 2c + 1
-            finish_row(cur, seg_first, s, 2 * static_cast<int>(blockIdx.x) + (seg_no > 0 ? 1 : 0));
-            ++seg_no;
-            if (i + 1 < n_my) {
-                ++row;
-                s = 0;
-                seg_first = 0;
-                cur = att_row(P, row);
-                if (cur.T < 0 && tid == 0) flag_status(kStatusBounds);
-                load_query(row);
-                reset_row();
-            }
+            // this thread's staging row is consumed: start the next fp4 block's copy
+            f1 = f2;
+            slot1 = resolve(f1, idx2, pg2);
+            if (f1 < nblk) issue(slot1);
+            f2 = next_fp4(f1 + 1);
+            idx2 = load_idx(f2);
         } else {
-            ++s;
+            // ---- window block: bf16 rows j .. j + 127 of the band, by 16-byte cp.async
+            const bool valid = rw.T >= 0 && rw.pos - (kWindow - 1) + r >= 0;
+            const __nv_bfloat16 *src = P.swa + (static_cast<int64_t>(rw.b) * n_rows_swa + rw.j + r) * kDim;
+#pragma unroll
+            for (int t = 0; t < kAttGroups; ++t) {
+                if (i > 0 && !mbar_wait_bounded(&sm.pv_done[t], pp)) return false;
+                const int g1 = t < 4 ? 16 * t + 16 : 72;
+                for (int jg = 16 * t; jg < g1; ++jg)
+                    cp_async16(sm.tile + jg * kAttSlab + mykey, valid ? src + 8 * jg : P.swa, valid ? 16u : 0u);
+                cp_async_commit();
+                if (t > 0) {
+                    cp_async_wait<1>();                   // group t - 1 has landed
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.deq_done[t - 1]);
+                }
+            }
+            const uint32_t mk = __ballot_sync(0xffffffffu, valid);
+            if (lane == 0) sm.mask[i & 1][pw] = mk;
+            if (r == 0) sm.eq[i & 1] = 0;
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.deq_done[kAttGroups - 1]);
+        }
+    }
+    return true;
+}
+
+// ------------------------------------------------------------------ MMA issue
+__device__ __forceinline__ bool att_mma(const AttParams &P, AttSmem &sm, uint32_t tmem, int64_t b0, int nblk) {
+    // descriptors at offset 0; an operand k-step / tile adds its byte offset / 16 (start-address field)
+    const uint64_t d_kt = umma_desc(smem_u32(sm.tile), kTileLboK, kTileSboK, 0);
+    const uint64_t d_vt = umma_desc(smem_u32(sm.tile), kTileLboMN, kTileSboMN, 0);
+    const uint64_t d_qf = umma_desc(smem_u32(sm.qf), kQLbo, kQSbo, 0);
+    const uint64_t d_qb = umma_desc(smem_u32(sm.qb), kQLbo, kQSbo, 0);
+    const uint64_t d_ph = umma_desc(smem_u32(sm.p_hi), kPLbo, kPSbo, 0);
+    const uint64_t d_pl = umma_desc(smem_u32(sm.p_lo), kPLbo, kPSbo, 0);
+    constexpr uint32_t id_qk = umma_idesc(kAttBlk, kHeads, false, false);
+    constexpr uint32_t id_pv = umma_idesc(kAttBlk, kHeads, true, true);
+    for (int i = 0; i < nblk; ++i) {
+        const AttBlk k = att_blk(P, b0, nblk, i);
+        const uint32_t par = static_cast<uint32_t>(i & 1);
+        const uint32_t fmt = k.win ? kIdescBf16 : 0u;
+        const uint64_t d_q = k.win ? d_qb : d_qf;
+#pragma unroll
+        for (int t = 0; t < kAttGroups; ++t) {
+            if (!mbar_wait_bounded(&sm.deq_done[t], par)) return false;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 8 * t; ks < (t < 4 ? 8 * t + 8 : kDim / 16); ++ks)
+                umma_f16(tmem + kAttSCol, d_kt + static_cast<uint64_t>((ks * 2 * kAttSlab) >> 4),
+                         d_q + static_cast<uint64_t>((ks * 512) >> 4), id_qk | fmt, ks > 0 ? 1u : 0u);
+        }
+        umma_commit(&sm.s_full);
+        if (!mbar_wait_bounded(&sm.p_ready, par)) return false;
+        tc_fence_after();
+        const uint32_t acc0 = k.first ? 0u : 1u;
+#pragma unroll
+        for (int t = 0; t < kAttGroups; ++t) {
+            const uint32_t d = tmem + kAttOCol + 16 * t;
+#pragma unroll
+            for (int ks = 0; ks < kAttBlk / 16; ++ks) {
+                const uint64_t a = d_vt + static_cast<uint64_t>((t * 16 * kAttSlab + ks * 256) >> 4);
+                umma_f16(d, a, d_ph + static_cast<uint64_t>((ks * 512) >> 4), id_pv | fmt, ks == 0 ? acc0 : 1u);
+                if (k.win) umma_f16(d, a, d_pl + static_cast<uint64_t>((ks * 512) >> 4), id_pv | fmt, 1u);
+            }
+            umma_commit(&sm.pv_done[t]);
+        }
+    }
+    return true;
+}
+
+// ------------------------------------------------------------------ softmax, epilogue
+__device__ __forceinline__ bool att_softmax(const AttParams &P, AttSmem &sm, uint32_t tmem, int64_t b0, int nblk) {
+    const int q = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int r = threadIdx.x;                                  // key of the block (TMEM lane)
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    float m_run[kHeads], l_acc[kHeads];
+    int seg_j0 = 0, seg_no = 0;
+    for (int i = 0; i < nblk; ++i) {
+        const AttBlk k = att_blk(P, b0, nblk, i);
+        const uint32_t par = static_cast<uint32_t>(i & 1);
+        if (k.first) {
+#pragma unroll
+            for (int h = 0; h < kHeads; ++h) {
+                m_run[h] = -INFINITY;
+                l_acc[h] = 0.0f;
+            }
+            seg_j0 = k.j;
+        }
+        if (!mbar_wait_bounded(&sm.deq_done[kAttGroups - 1], par)) return false;   // mask, exponent
+        if (!mbar_wait_bounded(&sm.s_full, par)) return false;
+        tc_fence_after();
+        float s[kHeads];
+        tmem_ld16(trow + kAttSCol, s);
+        const bool valid = (sm.mask[i & 1][q] >> lane) & 1u;
+        const float sc = P.scale_log2 * (k.win ? 1.0f : exp2f(static_cast<float>(sm.eq[i & 1])));
+#pragma unroll
+        for (int h = 0; h < kHeads; ++h) s[h] = valid ? s[h] * sc : -INFINITY;
+        {
+            const float mh = warp_reduce16<true>(s);
+            if ((lane & 1) == 0) sm.red_m[q][lane >> 1] = mh;
+        }
+        named_bar(1, kAttSoftWarps * 32);
+        float alpha[kHeads];
+        bool rescale = false;
+#pragma unroll
+        for (int h = 0; h < kHeads; ++h) {
+            const float mb = fmaxf(fmaxf(sm.red_m[0][h], sm.red_m[1][h]), fmaxf(sm.red_m[2][h], sm.red_m[3][h]));
+            const float mn = fmaxf(m_run[h], mb);
+            alpha[h] = m_run[h] == -INFINITY ? 1.0f : exp2f(m_run[h] - mn);
+            rescale |= alpha[h] != 1.0f;
+            m_run[h] = mn;
+        }
+        // probabilities of this key: f16 (FP4 block) or bf16 hi + lo (window block)
+        {
+            uint32_t hi[8], lo[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                float p0 = s[2 * u] == -INFINITY ? 0.0f : exp2f(s[2 * u] - m_run[2 * u]);
+                float p1 = s[2 * u + 1] == -INFINITY ? 0.0f : exp2f(s[2 * u + 1] - m_run[2 * u + 1]);
+                if (!k.win) {
+                    const __half2 h2 = __floats2half2_rn(p0, p1);
+                    hi[u] = *reinterpret_cast<const uint32_t *>(&h2);
+                    const float2 used = __half22float2(h2);
+                    p0 = used.x;
+                    p1 = used.y;
+                } else {
+                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+                    const float2 bh = __bfloat1622float2(b2);
+                    const __nv_bfloat162 c2 = __floats2bfloat162_rn(p0 - bh.x, p1 - bh.y);
+                    const float2 bl = __bfloat1622float2(c2);
+                    hi[u] = *reinterpret_cast<const uint32_t *>(&b2);
+                    lo[u] = *reinterpret_cast<const uint32_t *>(&c2);
+                    p0 = bh.x + bl.x;
+                    p1 = bh.y + bl.y;
+                }
+                l_acc[2 * u] = l_acc[2 * u] * alpha[2 * u] + p0;
+                l_acc[2 * u + 1] = l_acc[2 * u + 1] * alpha[2 * u + 1] + p1;
+            }
+            const uint32_t po = static_cast<uint32_t>((r >> 3) * 256 + (r & 7) * 16);
+            *reinterpret_cast<uint4 *>(sm.p_hi + po) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4 *>(sm.p_hi + po + 128) = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+            if (k.win) {
+                *reinterpret_cast<uint4 *>(sm.p_lo + po) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                *reinterpret_cast<uint4 *>(sm.p_lo + po + 128) = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+            }
+        }
+        if (!k.first && rescale) {
+            // the running maximum rose: O *= alpha once the previous block's PV is done
+            if (!mbar_wait_bounded(&sm.pv_done[kAttGroups - 1], par ^ 1u)) return false;
+            tc_fence_after();
+#pragma unroll 1
+            for (int t = 0; t < kAttGroups; ++t) {
+                float o[kHeads];
+                tmem_ld16(trow + kAttOCol + 16 * t, o);
+#pragma unroll
+                for (int h = 0; h < kHeads; ++h) o[h] *= alpha[h];
+                tmem_st16(trow + kAttOCol + 16 * t, o);
+            }
+            tmem_st_wait();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_ready);
+        if (!k.last) continue;
+
+        // ---- end of a row segment: read O, write the result or the partial
+        if (!mbar_wait_bounded(&sm.pv_done[kAttGroups - 1], par)) return false;
+        tc_fence_after();
+        {
+            const float lh = warp_reduce16<false>(l_acc);
+            if ((lane & 1) == 0) sm.red_l[q][lane >> 1] = lh;
+        }
+        named_bar(1, kAttSoftWarps * 32);
+        float l[kHeads], mul[kHeads];
+        const bool whole = seg_j0 == 0 && k.j == P.n_st - 1;
+#pragma unroll
+        for (int h = 0; h < kHeads; ++h) {
+            l[h] = (sm.red_l[0][h] + sm.red_l[1][h]) + (sm.red_l[2][h] + sm.red_l[3][h]);
+            mul[h] = whole ? (l[h] > 0.0f ? 1.0f / l[h] : 0.0f) : 1.0f;
+        }
+        const int slot = 2 * static_cast<int>(blockIdx.x) + (seg_no > 0 ? 1 : 0);
+        float *dst = whole ? P.out + static_cast<int64_t>(k.row) * kHeads * kDim
+                           : P.part_o + static_cast<int64_t>(slot) * kHeads * kDim;
+#pragma unroll 1
+        for (int t = 0; t < kAttGroups; ++t) {
+            float o[kHeads];
+            tmem_ld16(trow + kAttOCol + 16 * t, o);
+            const int c = 128 * t + r;
+            if (c < kDim) {
+#pragma unroll
+                for (int h = 0; h < kHeads; ++h) dst[h * kDim + c] = o[h] * mul[h];
+            }
+        }
+        if (r < kHeads) {
+            float lr = 0.0f, mr = 0.0f;
+#pragma unroll
+            for (int h = 0; h < kHeads; ++h)
+                if (h == r) {
+                    lr = l[h];
+                    mr = m_run[h];
+                }
+            if (whole)
+                P.lse[static_cast<int64_t>(k.row) * kHeads + r] = lr > 0.0f ? (mr + log2f(lr)) * 0.69314718055994530942f
+                                                                            : -INFINITY;
+            else
+                P.part_ml[static_cast<int64_t>(slot) * kHeads + r] = make_float2(mr, lr);
+        }
+        tc_fence_before();
+        ++seg_no;
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(kAttThreads, 1)
+sparse_attn_kernel(const AttParams P) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    AttSmem &sm = *reinterpret_cast<AttSmem *>(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int grid = static_cast<int>(gridDim.x);
+    const int64_t b0 = att_range_start(P.total_steps, blockIdx.x, grid);
+    const int nblk = static_cast<int>(att_range_start(P.total_steps, blockIdx.x + 1, grid) - b0);
+    if (nblk <= 0) return;                                      // uniform
+    if (tid == 0) {
+        for (int t = 0; t < kAttGroups; ++t) {
+            mbar_init(&sm.deq_done[t], kAttProdWarps);
+            mbar_init(&sm.pv_done[t], 1);
+        }
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.p_ready, kAttSoftWarps);
+        mbar_init(&sm.raw_full, kAttProdWarps * 32);
+        mbar_init(&sm.drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == kAttMmaWarp) {
+        tmem_alloc(&sm.tmem_base, kAttTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    pdl_wait();                                                 // the top-k indices are ready
+    pdl_trigger();
+    if (warp < kAttSoftWarps) {
+        att_softmax(P, sm, tmem, b0, nblk);
+    } else if (warp < kAttSoftWarps + kAttProdWarps) {
+        att_producers(P, sm, b0, nblk);
+    } else if ((tid & 31) == 0) {
+        const bool ok = att_mma(P, sm, tmem, b0, nblk);
+        if (!ok) {                                              // let every MMA issued finish before the release
+            umma_commit(&sm.drain);
+            mbar_wait_bounded(&sm.drain, 0);
         }
     }
     cp_async_wait<0>();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kAttMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kAttTmemCols);
+    }
 }
 
 // K5: merge the partials of the rows whose steps were split over CTAs:

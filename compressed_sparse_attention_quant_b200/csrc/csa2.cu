@@ -147,19 +147,19 @@ IdxLayout idx_layout(int B, int Sq, int max_pages, int k) {
 
 // ---------------------------------------------------------------- attention work plan
 struct AttPlan {
-    int n_win;           // window steps per query row (8, or 0 without a window)
-    int n_st;            // steps of 16 keys per query row
-    int64_t total;       // steps over all rows
-    int grid;            // CTAs (each a contiguous range of steps)
+    int n_win;           // window blocks per query row (1, or 0 without a window)
+    int n_st;            // blocks of 128 keys per query row
+    int64_t total;       // blocks over all rows
+    int grid;            // CTAs (each a contiguous range of blocks)
 };
 
-// At most one wave of CTAs, each with at least 4 steps of work.
+// One persistent CTA per SM (at most one wave), each with at least one block.
 AttPlan att_plan(int R, int k, int slots, bool window = true) {
     AttPlan pl;
-    pl.n_win = window ? kAttWinSteps : 0;
-    pl.n_st = pl.n_win + (k + kAttStepKeys - 1) / kAttStepKeys;
+    pl.n_win = window ? 1 : 0;
+    pl.n_st = pl.n_win + (k + kAttBlk - 1) / kAttBlk;
     pl.total = static_cast<int64_t>(R) * pl.n_st;
-    pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(std::min(slots, kMergeMaxParts), pl.total / 4)));
+    pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(std::min(slots, kMergeMaxParts), pl.total)));
     return pl;
 }
 
