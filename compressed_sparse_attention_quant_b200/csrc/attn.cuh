@@ -36,8 +36,10 @@
 //            commit; after the probabilities, PV tile by tile, one commit per
 //            tile (each releases that channel group to the producers).
 //   softmax  (warps 0..3, one key per thread, the block's S row from tensor
-//            memory): exp2 domain, exact running maximum per head (a block
-//            whose maximum rises rescales O in tensor memory first),
+//            memory): exp2 domain, a reference maximum per head that rises
+//            only when a block exceeds it by more than 8 (then O is rescaled
+//            in tensor memory first; otherwise probabilities up to 2^8 stay
+//            as they are, at the same relative precision),
 //            probabilities rounded to f16 (FP4 blocks) or split into two bf16
 //            terms hi + lo (the window block, bf16 operands), and the sum of
 //            exactly the values the MMA uses. At the end of a row segment
@@ -64,6 +66,7 @@ constexpr int kAttRawBytes = kAttBlk * kAttRawStride;          // 38,912
 constexpr int kAttTmemCols = 128;
 constexpr int kAttSCol = 0;                                    // S^T: 16 columns
 constexpr int kAttOCol = 16;                                   // O^T: 5 tiles x 16 columns
+constexpr float kAttSlack = 8.0f;                              // log2 units a block may exceed the reference max
 constexpr uint32_t kIdescBf16 = (1u << 7) | (1u << 10);        // A and B format BF16 (kind::f16)
 // Operand strides (bytes between adjacent 8 x 16-byte core matrices).
 // K-major: LBO = along K, SBO = along M/N.
@@ -90,7 +93,7 @@ struct AttSmem {
     uint32_t mask[2][4];                                       // valid keys of a block, by block parity
     int eq[2];                                                 // query exponent of a block
     float qmax[2][kAttProdWarps];
-    float red_m[kAttSoftWarps][kHeads];
+    alignas(16) float red_m[kAttSoftWarps][kHeads];
     float red_l[kAttSoftWarps][kHeads];
 };
 constexpr size_t kAttSmemBytes = sizeof(AttSmem);
@@ -520,15 +523,35 @@ __device__ __forceinline__ bool att_softmax(const AttParams &P, AttSmem &sm, uin
             if ((lane & 1) == 0) sm.red_m[q][lane >> 1] = mh;
         }
         named_bar(1, kAttSoftWarps * 32);
+        // Reference maximum per head: the first finite block maximum, raised
+        // only when a block exceeds it by more than kAttSlack (then O and l
+        // are rescaled); otherwise probabilities up to 2^kAttSlack are kept,
+        // which f16 and the bf16 pair represent with the same relative error.
         float alpha[kHeads];
         bool rescale = false;
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) {
-            const float mb = fmaxf(fmaxf(sm.red_m[0][h], sm.red_m[1][h]), fmaxf(sm.red_m[2][h], sm.red_m[3][h]));
-            const float mn = fmaxf(m_run[h], mb);
-            alpha[h] = m_run[h] == -INFINITY ? 1.0f : exp2f(m_run[h] - mn);
-            rescale |= alpha[h] != 1.0f;
-            m_run[h] = mn;
+        for (int h4 = 0; h4 < kHeads / 4; ++h4) {
+            const float4 a = reinterpret_cast<const float4 *>(sm.red_m[0])[h4];
+            const float4 b = reinterpret_cast<const float4 *>(sm.red_m[1])[h4];
+            const float4 c = reinterpret_cast<const float4 *>(sm.red_m[2])[h4];
+            const float4 d = reinterpret_cast<const float4 *>(sm.red_m[3])[h4];
+            const float mbv[4] = {fmaxf(fmaxf(a.x, b.x), fmaxf(c.x, d.x)), fmaxf(fmaxf(a.y, b.y), fmaxf(c.y, d.y)),
+                                  fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, d.z)), fmaxf(fmaxf(a.w, b.w), fmaxf(c.w, d.w))};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int h = 4 * h4 + e;
+                const float mb = mbv[e];
+                if (m_run[h] == -INFINITY) {
+                    alpha[h] = 1.0f;                     // O and l of this head are still zero
+                    m_run[h] = mb;
+                } else if (mb > m_run[h] + kAttSlack) {
+                    alpha[h] = exp2f(m_run[h] - mb);
+                    m_run[h] = mb;
+                    rescale = true;
+                } else {
+                    alpha[h] = 1.0f;
+                }
+            }
         }
         // probabilities of this key: f16 (FP4 block) or bf16 hi + lo (window block)
         {
@@ -565,7 +588,7 @@ __device__ __forceinline__ bool att_softmax(const AttParams &P, AttSmem &sm, uin
             }
         }
         if (!k.first && rescale) {
-            // the running maximum rose: O *= alpha once the previous block's PV is done
+            // the reference maximum rose: O *= alpha once the previous block's PV is done
             if (!mbar_wait_bounded(&sm.pv_done[kAttGroups - 1], par ^ 1u)) return false;
             tc_fence_after();
 #pragma unroll 1

@@ -5,17 +5,19 @@
 // The pool is the Full layer's top-C (ascending token indices, -1 padded, as
 // K3 emits it); the layer scores only those tokens with its own query.
 //
-// One thread-block cluster of S CTAs (512 threads each) per query row; CTA q
-// owns the q-th contiguous slice of the pool, so the slices are in pool order.
-//   score   warps take 16 pool entries at a time. The entries' page-table
-//           entries, scales and 64-byte indexer keys are gathered in phases
-//           (indices, then pages, then keys) so the loads of many entries are
-//           in flight together; the keys are the A operand (16 entries x 32
-//           channels per k-step) of FP8 mma.sync m16n8k32 against the row's
-//           query (4 heads as B columns), fp32 accumulation. ReLU, sigma and
-//           the head weights follow; the score's order-preserving 32-bit key
-//           goes to shared memory (0 marks an empty or invalid entry: no
-//           finite score maps there).
+// One thread-block cluster of S CTAs (S = 1 or 2, 512 threads each) per
+// query row; CTA q owns the q-th contiguous slice of the pool, so the slices
+// are in pool order.
+//   slots   each thread resolves 8 of its slice's entries at a time (pool
+//           index, then page-table entry, loads of all 8 in flight) to
+//           physical cache slots, kept in shared memory.
+//   score   warps take 4 groups of 16 entries at a time: their indexer keys
+//           (64 bytes each) and scales are loaded together, the keys are the
+//           A operand (16 entries x 32 channels per k-step) of FP8 mma.sync
+//           m16n8k32 against the row's query (4 heads as B columns), fp32
+//           accumulation. ReLU, sigma and the head weights follow; the
+//           score's order-preserving 32-bit key replaces the slot (0 marks an
+//           empty or invalid entry: no finite score maps there).
 //   select  radix select on the keys, 11 + 11 + 10 bits: each level a shared
 //           histogram per CTA, summed over the cluster through distributed
 //           shared memory, and a warp-level pick; it gives the k-th largest
@@ -50,8 +52,9 @@ constexpr int kPoolWarps = kPoolThreads / 32;
 constexpr int kPoolBins = 2048;
 static_assert(kPoolBins == kTopkBins, "the pool shares warp_pick and its padded histogram with K3");
 constexpr int kPoolMax = 32768;                  // largest pool per row
-constexpr int kPoolMaxCluster = 8;
-constexpr int kPoolMaxIt = 8;                    // 16-entry groups per warp held in flight
+constexpr int kPoolMaxCluster = 2;
+constexpr int kPoolBatch = 8;                    // entries per thread resolved together (pass 1)
+constexpr int kPoolGroups = 4;                   // 16-entry groups per warp scored together (pass 2)
 
 struct PoolSmemFixed {
     uint32_t qb[kIdxHeads * kIdxDim / 4];        // the row's query, E4M3 bytes (4 per word)
@@ -60,6 +63,7 @@ struct PoolSmemFixed {
     uint32_t hsum[kTopkBinsPadded];              // cluster-wide sum, padded (hpad) as warp_pick reads it
     uint32_t wcnt[2][kPoolWarps];
     uint32_t xchg[3];                            // (valid entries, selected, ties) of this CTA, read by peers
+    uint32_t s_pick[2];                          // (bin, count above) of the current level
 };
 
 constexpr size_t pool_smem_bytes(int slice) {
@@ -138,6 +142,7 @@ pool_topk_kernel(const PoolArgs A) {
     };
 
     // ---------------- keys of this CTA's entries
+    const int n_mine = max(e1 - e0, 0);
     uint32_t n_valid = 0u;
     if (A.given) {
         for (int i = e0 + tid; i < e1; i += kPoolThreads) {
@@ -151,6 +156,42 @@ pool_topk_kernel(const PoolArgs A) {
             keys[i - e0] = key;
         }
     } else {
+        // ---- pass 1: the slice's physical slots (pool index -> page -> slot,
+        // -1 for an empty or invalid entry), written in place into keys[];
+        // kPoolBatch entries per thread have their loads in flight together
+        for (int base = 0; base < n_mine; base += kPoolThreads * kPoolBatch) {
+            int tk[kPoolBatch], tprev[kPoolBatch];
+            int64_t pg[kPoolBatch];
+#pragma unroll
+            for (int u = 0; u < kPoolBatch; ++u) {
+                const int il = base + u * kPoolThreads + tid, i = e0 + il;
+                tk[u] = il < n_mine ? A.pool[entry(i)] : -1;
+                tprev[u] = il < n_mine && i > 0 ? A.pool[entry(i - 1)] : -1;
+            }
+#pragma unroll
+            for (int u = 0; u < kPoolBatch; ++u)
+                pg[u] = tk[u] >= 0 && tk[u] < lim ? A.page_table[static_cast<int64_t>(b) * A.max_pages + (tk[u] >> 6)] : -1;
+#pragma unroll
+            for (int u = 0; u < kPoolBatch; ++u) {
+                const int il = base + u * kPoolThreads + tid;
+                if (il >= n_mine) continue;
+                int slot = -1;
+                const int t = tk[u];
+                if (t >= 0) {
+                    if (tprev[u] >= t) flag_status(kStatusBounds);                // the pool must ascend
+                    if (t >= lim || pg[u] < 0 || pg[u] >= A.num_pages) {
+                        flag_status(kStatusBounds);
+                    } else {
+                        slot = static_cast<int>(pg[u] * kPage + (t & 63));
+                        ++n_valid;
+                    }
+                }
+                keys[il] = static_cast<uint32_t>(slot);
+            }
+        }
+        __syncthreads();
+        // ---- pass 2: scores. A warp takes kPoolGroups groups of 16 entries at
+        // a time (all their key and sigma loads in flight), one MMA per group.
         // query B fragments: head g (< 4) channels 4 tig .. +3 and 16 + 4 tig .. +3 of each k-step
         uint32_t qf[2][2];
 #pragma unroll
@@ -159,67 +200,44 @@ pool_topk_kernel(const PoolArgs A) {
             qf[ks][1] = g < kIdxHeads ? fs.qb[(g * kIdxDim + ks * 32 + 16 + 4 * tig) / 4] : 0u;
         }
         const float wlo = fs.w[2 * (tig & 1)], whi = fs.w[2 * (tig & 1) + 1];
-        // groups of 16 entries: warp w takes groups w, w + 16, ... of the slice
-        const int n_groups = (e1 - e0 + 15) / 16;
-        for (int gb = warp; gb < n_groups; gb += kPoolWarps * kPoolMaxIt) {
-            int tok[kPoolMaxIt][2];
-            int64_t pg[kPoolMaxIt][2];
+        const int n_groups = (n_mine + 15) / 16;
+        for (int g0 = warp * kPoolGroups; g0 < n_groups; g0 += kPoolWarps * kPoolGroups) {
+            int sl[kPoolGroups][2];
+            uint32_t a[kPoolGroups][2][4];
+            float sg[kPoolGroups][2];
 #pragma unroll
-            for (int it = 0; it < kPoolMaxIt; ++it)              // phase 1: pool indices
+            for (int q = 0; q < kPoolGroups; ++q)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const int grp = gb + it * kPoolWarps;
-                    const int i = e0 + grp * 16 + g + 8 * h;
-                    tok[it][h] = (grp < n_groups && i < e1) ? A.pool[entry(i)] : -1;
+                    const int il = (g0 + q) * 16 + g + 8 * h;
+                    sl[q][h] = g0 + q < n_groups && il < n_mine ? static_cast<int>(keys[il]) : -1;
                 }
 #pragma unroll
-            for (int it = 0; it < kPoolMaxIt; ++it)              // phase 2: pages
+            for (int q = 0; q < kPoolGroups; ++q)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const int t = tok[it][h];
-                    pg[it][h] = (t >= 0 && t < lim) ? A.page_table[static_cast<int64_t>(b) * A.max_pages + (t >> 6)] : -1;
-                }
-#pragma unroll
-            for (int it = 0; it < kPoolMaxIt; ++it) {           // phase 3: keys, MMA, scores
-                const int grp = gb + it * kPoolWarps;
-                if (grp >= n_groups) break;                      // warp-uniform
-                uint32_t a[2][4];
-                float sg[2];
-                bool ok[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int t = tok[it][h];
-                    const int64_t p = pg[it][h];
-                    ok[h] = t >= 0 && t < lim && p >= 0 && p < A.num_pages;
-                    const int r = t & 63;
-                    const uint8_t *kb = A.kidx + (ok[h] ? p * kKidxPageBytes + (r >> 3) * 512 + (r & 7) * 16 + 4 * tig : 0);
+                    const int sv = sl[q][h];
+                    const uint8_t *kb = A.kidx + (sv >= 0 ? static_cast<int64_t>(sv >> 6) * kKidxPageBytes +
+                                                                ((sv & 63) >> 3) * 512 + (sv & 7) * 16 + 4 * tig
+                                                          : 0);
 #pragma unroll
                     for (int c = 0; c < 4; ++c)                 // 16-byte chunk c = channels 16c .. 16c + 15
-                        a[c >> 1][(c & 1) * 2 + h] = ok[h] ? __ldg(reinterpret_cast<const uint32_t *>(kb + c * 128)) : 0u;
-                    sg[h] = ok[h] ? __ldg(A.kidx_scale + p * kPage + r) : 0.0f;
+                        a[q][c >> 1][(c & 1) * 2 + h] = sv >= 0 ? __ldg(reinterpret_cast<const uint32_t *>(kb + c * 128)) : 0u;
+                    sg[q][h] = sv >= 0 ? __ldg(A.kidx_scale + sv) : 0.0f;
                 }
+#pragma unroll
+            for (int q = 0; q < kPoolGroups; ++q) {
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks)
-                    mma_e4m3_16832(acc, a[ks][0], a[ks][1], a[ks][2], a[ks][3], qf[ks][0], qf[ks][1]);
+                    mma_e4m3_16832(acc, a[q][ks][0], a[q][ks][1], a[q][ks][2], a[q][ks][3], qf[ks][0], qf[ks][1]);
                 // lanes with tig 0 / 1 hold heads 0, 1 / 2, 3 of entries g and g + 8
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    float part = wlo * fmaxf(0.0f, sg[h] * acc[2 * h]) + whi * fmaxf(0.0f, sg[h] * acc[2 * h + 1]);
+                    float part = wlo * fmaxf(0.0f, sg[q][h] * acc[2 * h]) + whi * fmaxf(0.0f, sg[q][h] * acc[2 * h + 1]);
                     part += __shfl_xor_sync(0xffffffffu, part, 1);   // heads 0..3
-                    const int i = e0 + grp * 16 + g + 8 * h;
-                    const int t = tok[it][h];
-                    if (tig == 0 && i < e1) {
-                        uint32_t key = 0u;
-                        if (ok[h]) {
-                            if (i > 0 && A.pool[entry(i - 1)] >= t) flag_status(kStatusBounds);   // pool must ascend
-                            key = float_key(part);
-                            ++n_valid;
-                        } else if (t >= 0) {
-                            flag_status(kStatusBounds);
-                        }
-                        keys[i - e0] = key;
-                    }
+                    const int il = (g0 + q) * 16 + g + 8 * h;
+                    if (tig == 0 && g0 + q < n_groups && il < n_mine) keys[il] = sl[q][h] >= 0 ? float_key(part) : 0u;
                 }
             }
         }
@@ -239,7 +257,6 @@ pool_topk_kernel(const PoolArgs A) {
     uint32_t row_valid = 0u;
     for (int q = 0; q < S; ++q) row_valid += *cluster.map_shared_rank(&fs.xchg[0], q);
     const uint32_t need = min(static_cast<uint32_t>(A.k), row_valid);
-    const int n_mine = max(e1 - e0, 0);
 
     // ---------------- threshold key T: the need-th largest key over the cluster
     uint32_t thr = 0u, n_gt = 0u;                // select keys > thr, then (need - n_gt) ties == thr
@@ -268,10 +285,17 @@ pool_topk_kernel(const PoolArgs A) {
                 fs.hsum[hpad(i)] = v;
             }
             __syncthreads();
-            uint32_t bin, ab;
-            warp_pick<false>(fs.hsum, 1 << wdt, need - above, bin, ab);
-            above += ab;
-            prefix = (prefix << wdt) | bin;
+            if (warp == 0) {
+                uint32_t bin, ab;
+                warp_pick<false>(fs.hsum, 1 << wdt, need - above, bin, ab);
+                if (lane == 0) {
+                    fs.s_pick[0] = bin;
+                    fs.s_pick[1] = ab;
+                }
+            }
+            __syncthreads();
+            above += fs.s_pick[1];
+            prefix = (prefix << wdt) | fs.s_pick[0];
         }
         thr = prefix;
         n_gt = above;
@@ -341,8 +365,8 @@ pool_topk_kernel(const PoolArgs A) {
     cluster.sync();                                             // no CTA leaves while a peer may read its counts
 }
 
-// Cluster size: the largest power of two (<= 8) with every CTA holding at
-// least 1024 entries and all clusters within one wave of two CTAs per SM.
+// Cluster size: 2 when every CTA still holds at least 1024 entries and all
+// clusters fit in one wave of two CTAs per SM, else 1.
 inline cudaError_t launch_pool_topk(PoolArgs A, int rows, int sm_count, cudaStream_t stream) {
     int S = 1;
     while (S * 2 <= kPoolMaxCluster && static_cast<int64_t>(rows) * S * 2 <= 2 * sm_count && A.C / (S * 2) >= 1024)
