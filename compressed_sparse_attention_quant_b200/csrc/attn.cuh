@@ -213,6 +213,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+__device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
+// Barrier over n threads that also ORs a predicate across them.
+__device__ __forceinline__ bool bar_red_or(int id, int n, bool v) {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(res) : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(n) : "memory");
+    return res != 0u;
+}
+
 __device__ __forceinline__ void named_bar(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -317,6 +329,78 @@ __device__ __forceinline__ bool att_producers(const AttParams &P, AttSmem &sm, i
             for (int u = 0; u < 9; ++u) sc_next[u] = 0u;  // zero scale: the key's tile row is zero
         }
     };
+    // The row's query: a bf16 copy and an f16 copy under exponent eq. Before
+    // overwriting, the previous block's QK must be done (its PV tile 0 is).
+    int eq = 0, qrow_par = 0;
+    auto stage_q = [&](const AttBlk &k, const AttRow &rw, int i) -> bool {
+        const uint32_t pp = static_cast<uint32_t>((i - 1) & 1);
+        // ---- the row's query: bf16 copy and f16 copy under exponent eq
+        if (rw.T < 0 && r == 0) flag_status(kStatusBounds);
+        const __nv_bfloat16 *qr = P.q + static_cast<int64_t>(k.row) * kHeads * kDim;
+        uint4 qv[9];
+        float mx = 0.0f;
+#pragma unroll
+        for (int u = 0; u < 9; ++u) {
+            const int c = u * 128 + r, h = c & 15, jg = c >> 4;
+            qv[u] = __ldg(reinterpret_cast<const uint4 *>(qr + h * kDim + 8 * jg));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = bf16x2_f32((&qv[u].x)[e]);
+                mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        if (lane == 0) sm.qmax[qrow_par][pw] = mx;
+        named_bar(2, kAttProdWarps * 32);
+        mx = fmaxf(fmaxf(sm.qmax[qrow_par][0], sm.qmax[qrow_par][1]), fmaxf(sm.qmax[qrow_par][2], sm.qmax[qrow_par][3]));
+        qrow_par ^= 1;
+        eq = f16_exponent(mx);
+        const float sdown = exp2f(static_cast<float>(-eq));
+        // the previous block's QK has read the old query once its PV tile 0 is done
+        if (i > 0 && !mbar_wait_bounded(&sm.pv_done[0], pp)) return false;
+#pragma unroll
+        for (int u = 0; u < 9; ++u) {
+            const int c = u * 128 + r, h = c & 15, jg = c >> 4;
+            const uint32_t off = static_cast<uint32_t>(jg * 256 + (h >> 3) * 128 + (h & 7) * 16);
+            *reinterpret_cast<uint4 *>(sm.qb + off) = qv[u];
+            uint32_t hv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = bf16x2_f32((&qv[u].x)[e]);
+                hv[e] = f32x2_f16x2(f.x * sdown, f.y * sdown);
+            }
+            *reinterpret_cast<uint4 *>(sm.qf + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        }
+        return true;
+    };
+    // Window rows j .. j + 127 of the band into the tile, one cp.async group
+    // per channel group, each issued once the previous block's PV has
+    // released it.
+    auto win_issue = [&](const AttRow &rw, int i) -> bool {
+        const uint32_t pp = static_cast<uint32_t>((i - 1) & 1);
+        const bool valid = rw.T >= 0 && rw.pos - (kWindow - 1) + r >= 0;
+        const __nv_bfloat16 *src = P.swa + (static_cast<int64_t>(rw.b) * n_rows_swa + rw.j + r) * kDim;
+#pragma unroll 1
+        for (int t = 0; t < kAttGroups; ++t) {
+            if (i > 0 && !mbar_wait_bounded(&sm.pv_done[t], pp)) return false;
+            const int g1 = t < 4 ? 16 * t + 16 : 72;
+            for (int jg = 16 * t; jg < g1; ++jg)
+                cp_async16(sm.tile + jg * kAttSlab + mykey, valid ? src + 8 * jg : P.swa, valid ? 16u : 0u);
+            cp_async_commit();
+        }
+        return true;
+    };
+    // The first block's query (and window rows) are inputs that no kernel
+    // of this path writes: they are staged before waiting for the selection
+    // of the previous kernel, while it finishes.
+    {
+        const AttBlk k0 = att_blk(P, b0, nblk, 0);
+        const AttRow rw0 = att_row(P, k0.row);
+        stage_q(k0, rw0, 0);
+        if (k0.win) win_issue(rw0, 0);
+    }
+    pdl_wait();                                           // the top-k indices are ready
     // pipeline: the next fp4 block's copy is in flight; the one after has its top-k index loaded
     int f1 = next_fp4(0);
     int slot1 = -1;
@@ -328,58 +412,15 @@ __device__ __forceinline__ bool att_producers(const AttParams &P, AttSmem &sm, i
     int f2 = next_fp4(f1 + 1);
     int idx2 = load_idx(f2);
     uint32_t raw_par = 0u;
-    int eq = 0, qrow_par = 0;
 
     for (int i = 0; i < nblk; ++i) {
         const AttBlk k = att_blk(P, b0, nblk, i);
         const AttRow rw = att_row(P, k.row);
         const uint32_t pp = static_cast<uint32_t>((i - 1) & 1);
-        if (k.first) {
-            // ---- the row's query: bf16 copy and f16 copy under exponent eq
-            if (rw.T < 0 && r == 0) flag_status(kStatusBounds);
-            const __nv_bfloat16 *qr = P.q + static_cast<int64_t>(k.row) * kHeads * kDim;
-            uint4 qv[9];
-            float mx = 0.0f;
-#pragma unroll
-            for (int u = 0; u < 9; ++u) {
-                const int c = u * 128 + r, h = c & 15, jg = c >> 4;
-                qv[u] = __ldg(reinterpret_cast<const uint4 *>(qr + h * kDim + 8 * jg));
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = bf16x2_f32((&qv[u].x)[e]);
-                    mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-                }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-            if (lane == 0) sm.qmax[qrow_par][pw] = mx;
-            named_bar(2, kAttProdWarps * 32);
-            mx = fmaxf(fmaxf(sm.qmax[qrow_par][0], sm.qmax[qrow_par][1]), fmaxf(sm.qmax[qrow_par][2], sm.qmax[qrow_par][3]));
-            qrow_par ^= 1;
-            eq = f16_exponent(mx);
-            const float sdown = exp2f(static_cast<float>(-eq));
-            // the previous block's QK has read the old query once its PV tile 0 is done
-            if (i > 0 && !mbar_wait_bounded(&sm.pv_done[0], pp)) return false;
-#pragma unroll
-            for (int u = 0; u < 9; ++u) {
-                const int c = u * 128 + r, h = c & 15, jg = c >> 4;
-                const uint32_t off = static_cast<uint32_t>(jg * 256 + (h >> 3) * 128 + (h & 7) * 16);
-                *reinterpret_cast<uint4 *>(sm.qb + off) = qv[u];
-                uint32_t hv[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = bf16x2_f32((&qv[u].x)[e]);
-                    hv[e] = f32x2_f16x2(f.x * sdown, f.y * sdown);
-                }
-                *reinterpret_cast<uint4 *>(sm.qf + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-            }
-        }
+        if (k.first && i > 0 && !stage_q(k, rw, i)) return false;
         if (!k.win) {
             // ---- FP4 block: its records are (being) staged; resolve the one after next
             const int64_t pg2 = load_page(f2, idx2);
-            uint32_t sc[9];
-#pragma unroll
-            for (int u = 0; u < 9; ++u) sc[u] = sc_next[u];
             const bool valid = slot1 >= 0;
             if (!mbar_wait_bounded(&sm.raw_full, raw_par)) return false;
             raw_par ^= 1u;
@@ -387,19 +428,31 @@ __device__ __forceinline__ bool att_producers(const AttParams &P, AttSmem &sm, i
 #pragma unroll
             for (int t = 0; t < kAttGroups; ++t) {
                 if (i > 0 && !mbar_wait_bounded(&sm.pv_done[t], pp)) return false;
+                // scale bytes 8t .. 8t + 7 (pieces 4t .. 4t + 3): two words, selected without indexing
+                uint32_t sw0 = 0u, sw1 = 0u;
 #pragma unroll
-                for (int m = 4 * t; m < (t < 4 ? 4 * t + 4 : 18); ++m) {     // channels 32m .. 32m + 31
-                    const uint4 v = *reinterpret_cast<const uint4 *>(rr + 16 * m);
-                    const uint32_t s2 = e4m3x2_to_f16x2((sc[m >> 1] >> (16 * (m & 1))) & 0xffffu);
-                    const uint32_t sa = (s2 & 0xffffu) | (s2 << 16), sb = (s2 >> 16) | (s2 & 0xffff0000u);
+                for (int u = 0; u < 9; ++u) {
+                    sw0 = u == 2 * t ? sc_next[u] : sw0;
+                    sw1 = u == 2 * t + 1 ? sc_next[u] : sw1;
+                }
+                const int npc = t < kAttGroups - 1 ? 4 : 2;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint32_t w = (&v.x)[u], s = u < 2 ? sa : sb;
-                        const uint4 o = make_uint4(hmul2_u32(e2m1x2_to_f16x2(w & 0xffu), s),
-                                                   hmul2_u32(e2m1x2_to_f16x2((w >> 8) & 0xffu), s),
-                                                   hmul2_u32(e2m1x2_to_f16x2((w >> 16) & 0xffu), s),
-                                                   hmul2_u32(e2m1x2_to_f16x2(w >> 24), s));
-                        *reinterpret_cast<uint4 *>(sm.tile + (4 * m + u) * kAttSlab + mykey) = o;
+                for (int mm = 0; mm < 4; ++mm) {                 // channels 32m .. 32m + 31, m = 4t + mm
+                    if (mm < npc) {
+                        const int m = 4 * t + mm;
+                        const uint4 v = *reinterpret_cast<const uint4 *>(rr + 16 * m);
+                        const uint32_t sw = mm < 2 ? sw0 : sw1;
+                        const uint32_t s2 = e4m3x2_to_f16x2((sw >> (16 * (mm & 1))) & 0xffffu);
+                        const uint32_t sa = (s2 & 0xffffu) | (s2 << 16), sb = (s2 >> 16) | (s2 & 0xffff0000u);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint32_t w = (&v.x)[u], s = u < 2 ? sa : sb;
+                            const uint4 o = make_uint4(hmul2_u32(e2m1x2_to_f16x2(w & 0xffu), s),
+                                                       hmul2_u32(e2m1x2_to_f16x2((w >> 8) & 0xffu), s),
+                                                       hmul2_u32(e2m1x2_to_f16x2((w >> 16) & 0xffu), s),
+                                                       hmul2_u32(e2m1x2_to_f16x2(w >> 24), s));
+                            *reinterpret_cast<uint4 *>(sm.tile + (4 * m + u) * kAttSlab + mykey) = o;
+                        }
                     }
                 }
                 if (t == kAttGroups - 1) {
@@ -418,74 +471,100 @@ __device__ __forceinline__ bool att_producers(const AttParams &P, AttSmem &sm, i
             f2 = next_fp4(f1 + 1);
             idx2 = load_idx(f2);
         } else {
-            // ---- window block: bf16 rows j .. j + 127 of the band, by 16-byte cp.async
+            // ---- window block: its copies (issued here, or for block 0 before the
+            // wait for the selection) are published in order as they land
             const bool valid = rw.T >= 0 && rw.pos - (kWindow - 1) + r >= 0;
-            const __nv_bfloat16 *src = P.swa + (static_cast<int64_t>(rw.b) * n_rows_swa + rw.j + r) * kDim;
-#pragma unroll
-            for (int t = 0; t < kAttGroups; ++t) {
-                if (i > 0 && !mbar_wait_bounded(&sm.pv_done[t], pp)) return false;
-                const int g1 = t < 4 ? 16 * t + 16 : 72;
-                for (int jg = 16 * t; jg < g1; ++jg)
-                    cp_async16(sm.tile + jg * kAttSlab + mykey, valid ? src + 8 * jg : P.swa, valid ? 16u : 0u);
-                cp_async_commit();
-                if (t > 0) {
-                    cp_async_wait<1>();                   // group t - 1 has landed
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.deq_done[t - 1]);
-                }
-            }
+            if (i > 0 && !win_issue(rw, i)) return false;
             const uint32_t mk = __ballot_sync(0xffffffffu, valid);
             if (lane == 0) sm.mask[i & 1][pw] = mk;
             if (r == 0) sm.eq[i & 1] = 0;
-            cp_async_wait<0>();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.deq_done[kAttGroups - 1]);
+#define ATT_WIN_DONE(T)                                                                  \
+            cp_async_wait<kAttGroups - 1 - (T)>();                                       \
+            fence_proxy_async_smem();                                                    \
+            __syncwarp();                                                                \
+            if (lane == 0) mbar_arrive(&sm.deq_done[T]);
+            ATT_WIN_DONE(0)
+            ATT_WIN_DONE(1)
+            ATT_WIN_DONE(2)
+            ATT_WIN_DONE(3)
+            ATT_WIN_DONE(4)
+#undef ATT_WIN_DONE
+        }
+        // ---- the next block starts a row: pull its query and window band into L2
+        if (i + 1 < nblk) {
+            const AttBlk kn = att_blk(P, b0, nblk, i + 1);
+            if (kn.j == 0) {
+                const uint8_t *qn = reinterpret_cast<const uint8_t *>(P.q + static_cast<int64_t>(kn.row) * kHeads * kDim);
+                for (int l = r; l < kAttQBytes / 128; l += kAttBlk) prefetch_l2(qn + l * 128);
+                const AttRow rn = att_row(P, kn.row);
+                if (kn.win && rn.T >= 0 && rn.pos - (kWindow - 1) + r >= 0) {
+                    const uint8_t *wr = reinterpret_cast<const uint8_t *>(
+                        P.swa + (static_cast<int64_t>(rn.b) * n_rows_swa + rn.j + r) * kDim);
+#pragma unroll
+                    for (int l = 0; l < kDim * 2 / 128; ++l) prefetch_l2(wr + l * 128);
+                }
+            }
         }
     }
     return true;
 }
 
 // ------------------------------------------------------------------ MMA issue
+// Every MMA operand is a base descriptor plus a compile-time offset, and the
+// instruction descriptor and accumulate flag are compile-time constants (one
+// instantiation per block kind): with descriptors or flags computed at run
+// time, the issue of each MMA was measured to take about twice as long.
+template <bool kWin>
+__device__ __forceinline__ bool att_qk(AttSmem &sm, uint32_t tmem, uint64_t d_kt, uint64_t d_q, uint32_t par) {
+    constexpr uint32_t id = umma_idesc(kAttBlk, kHeads, false, false) | (kWin ? kIdescBf16 : 0u);
+#pragma unroll
+    for (int t = 0; t < kAttGroups; ++t) {
+        if (!mbar_wait_bounded(&sm.deq_done[t], par)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 8 * t; ks < (t < kAttGroups - 1 ? 8 * t + 8 : kDim / 16); ++ks)
+            umma_f16(tmem + kAttSCol, d_kt + static_cast<uint64_t>((ks * 2 * kAttSlab) >> 4),
+                     d_q + static_cast<uint64_t>((ks * 512) >> 4), id, ks > 0 ? 1u : 0u);
+    }
+    umma_commit(&sm.s_full);
+    return true;
+}
+
+template <bool kWin, bool kFirst>
+__device__ __forceinline__ void att_pv(AttSmem &sm, uint32_t tmem, uint64_t d_vt, uint64_t d_ph, uint64_t d_pl) {
+    constexpr uint32_t id = umma_idesc(kAttBlk, kHeads, true, true) | (kWin ? kIdescBf16 : 0u);
+#pragma unroll
+    for (int t = 0; t < kAttGroups; ++t) {
+#pragma unroll
+        for (int ks = 0; ks < kAttBlk / 16; ++ks) {
+            const uint64_t a = d_vt + static_cast<uint64_t>((t * 16 * kAttSlab + ks * 256) >> 4);
+            umma_f16(tmem + kAttOCol + 16 * t, a, d_ph + static_cast<uint64_t>((ks * 512) >> 4), id,
+                     (kFirst && ks == 0) ? 0u : 1u);
+            if (kWin) umma_f16(tmem + kAttOCol + 16 * t, a, d_pl + static_cast<uint64_t>((ks * 512) >> 4), id, 1u);
+        }
+        umma_commit(&sm.pv_done[t]);
+    }
+}
+
 __device__ __forceinline__ bool att_mma(const AttParams &P, AttSmem &sm, uint32_t tmem, int64_t b0, int nblk) {
-    // descriptors at offset 0; an operand k-step / tile adds its byte offset / 16 (start-address field)
     const uint64_t d_kt = umma_desc(smem_u32(sm.tile), kTileLboK, kTileSboK, 0);
     const uint64_t d_vt = umma_desc(smem_u32(sm.tile), kTileLboMN, kTileSboMN, 0);
     const uint64_t d_qf = umma_desc(smem_u32(sm.qf), kQLbo, kQSbo, 0);
     const uint64_t d_qb = umma_desc(smem_u32(sm.qb), kQLbo, kQSbo, 0);
     const uint64_t d_ph = umma_desc(smem_u32(sm.p_hi), kPLbo, kPSbo, 0);
     const uint64_t d_pl = umma_desc(smem_u32(sm.p_lo), kPLbo, kPSbo, 0);
-    constexpr uint32_t id_qk = umma_idesc(kAttBlk, kHeads, false, false);
-    constexpr uint32_t id_pv = umma_idesc(kAttBlk, kHeads, true, true);
     for (int i = 0; i < nblk; ++i) {
         const AttBlk k = att_blk(P, b0, nblk, i);
         const uint32_t par = static_cast<uint32_t>(i & 1);
-        const uint32_t fmt = k.win ? kIdescBf16 : 0u;
-        const uint64_t d_q = k.win ? d_qb : d_qf;
-#pragma unroll
-        for (int t = 0; t < kAttGroups; ++t) {
-            if (!mbar_wait_bounded(&sm.deq_done[t], par)) return false;
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 8 * t; ks < (t < 4 ? 8 * t + 8 : kDim / 16); ++ks)
-                umma_f16(tmem + kAttSCol, d_kt + static_cast<uint64_t>((ks * 2 * kAttSlab) >> 4),
-                         d_q + static_cast<uint64_t>((ks * 512) >> 4), id_qk | fmt, ks > 0 ? 1u : 0u);
-        }
-        umma_commit(&sm.s_full);
-        if (!mbar_wait_bounded(&sm.p_ready, par)) return false;
+        const bool ok = k.win ? att_qk<true>(sm, tmem, d_kt, d_qb, par) : att_qk<false>(sm, tmem, d_kt, d_qf, par);
+        if (!ok || !mbar_wait_bounded(&sm.p_ready, par)) return false;
         tc_fence_after();
-        const uint32_t acc0 = k.first ? 0u : 1u;
-#pragma unroll
-        for (int t = 0; t < kAttGroups; ++t) {
-            const uint32_t d = tmem + kAttOCol + 16 * t;
-#pragma unroll
-            for (int ks = 0; ks < kAttBlk / 16; ++ks) {
-                const uint64_t a = d_vt + static_cast<uint64_t>((t * 16 * kAttSlab + ks * 256) >> 4);
-                umma_f16(d, a, d_ph + static_cast<uint64_t>((ks * 512) >> 4), id_pv | fmt, ks == 0 ? acc0 : 1u);
-                if (k.win) umma_f16(d, a, d_pl + static_cast<uint64_t>((ks * 512) >> 4), id_pv | fmt, 1u);
-            }
-            umma_commit(&sm.pv_done[t]);
+        if (k.win) {
+            if (k.first) att_pv<true, true>(sm, tmem, d_vt, d_ph, d_pl);
+            else att_pv<true, false>(sm, tmem, d_vt, d_ph, d_pl);
+        } else {
+            if (k.first) att_pv<false, true>(sm, tmem, d_vt, d_ph, d_pl);
+            else att_pv<false, false>(sm, tmem, d_vt, d_ph, d_pl);
         }
     }
     return true;
@@ -518,38 +597,45 @@ __device__ __forceinline__ bool att_softmax(const AttParams &P, AttSmem &sm, uin
         const float sc = P.scale_log2 * (k.win ? 1.0f : exp2f(static_cast<float>(sm.eq[i & 1])));
 #pragma unroll
         for (int h = 0; h < kHeads; ++h) s[h] = valid ? s[h] * sc : -INFINITY;
-        {
-            const float mh = warp_reduce16<true>(s);
-            if ((lane & 1) == 0) sm.red_m[q][lane >> 1] = mh;
-        }
-        named_bar(1, kAttSoftWarps * 32);
         // Reference maximum per head: the first finite block maximum, raised
         // only when a block exceeds it by more than kAttSlack (then O and l
         // are rescaled); otherwise probabilities up to 2^kAttSlack are kept,
         // which f16 and the bf16 pair represent with the same relative error.
+        // In the common case no key exceeds it and the block's maximum is not
+        // needed: one barrier-reduction over the 128 keys decides (a segment's
+        // first block always exceeds the empty reference).
+        bool exceed = false;
+#pragma unroll
+        for (int h = 0; h < kHeads; ++h) exceed |= s[h] > m_run[h] + kAttSlack;
         float alpha[kHeads];
+#pragma unroll
+        for (int h = 0; h < kHeads; ++h) alpha[h] = 1.0f;
         bool rescale = false;
+        if (bar_red_or(1, kAttSoftWarps * 32, exceed)) {
+            {
+                const float mh = warp_reduce16<true>(s);
+                if ((lane & 1) == 0) sm.red_m[q][lane >> 1] = mh;
+            }
+            named_bar(1, kAttSoftWarps * 32);
 #pragma unroll
-        for (int h4 = 0; h4 < kHeads / 4; ++h4) {
-            const float4 a = reinterpret_cast<const float4 *>(sm.red_m[0])[h4];
-            const float4 b = reinterpret_cast<const float4 *>(sm.red_m[1])[h4];
-            const float4 c = reinterpret_cast<const float4 *>(sm.red_m[2])[h4];
-            const float4 d = reinterpret_cast<const float4 *>(sm.red_m[3])[h4];
-            const float mbv[4] = {fmaxf(fmaxf(a.x, b.x), fmaxf(c.x, d.x)), fmaxf(fmaxf(a.y, b.y), fmaxf(c.y, d.y)),
-                                  fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, d.z)), fmaxf(fmaxf(a.w, b.w), fmaxf(c.w, d.w))};
+            for (int h4 = 0; h4 < kHeads / 4; ++h4) {
+                const float4 a = reinterpret_cast<const float4 *>(sm.red_m[0])[h4];
+                const float4 b = reinterpret_cast<const float4 *>(sm.red_m[1])[h4];
+                const float4 c = reinterpret_cast<const float4 *>(sm.red_m[2])[h4];
+                const float4 d = reinterpret_cast<const float4 *>(sm.red_m[3])[h4];
+                const float mbv[4] = {fmaxf(fmaxf(a.x, b.x), fmaxf(c.x, d.x)), fmaxf(fmaxf(a.y, b.y), fmaxf(c.y, d.y)),
+                                      fmaxf(fmaxf(a.z, b.z), fmaxf(c.z, d.z)), fmaxf(fmaxf(a.w, b.w), fmaxf(c.w, d.w))};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int h = 4 * h4 + e;
-                const float mb = mbv[e];
-                if (m_run[h] == -INFINITY) {
-                    alpha[h] = 1.0f;                     // O and l of this head are still zero
-                    m_run[h] = mb;
-                } else if (mb > m_run[h] + kAttSlack) {
-                    alpha[h] = exp2f(m_run[h] - mb);
-                    m_run[h] = mb;
-                    rescale = true;
-                } else {
-                    alpha[h] = 1.0f;
+                for (int e = 0; e < 4; ++e) {
+                    const int h = 4 * h4 + e;
+                    const float mb = mbv[e];
+                    if (m_run[h] == -INFINITY) {
+                        m_run[h] = mb;                   // O and l of this head are still zero
+                    } else if (mb > m_run[h] + kAttSlack) {
+                        alpha[h] = exp2f(m_run[h] - mb);
+                        m_run[h] = mb;
+                        rescale = true;
+                    }
                 }
             }
         }
@@ -683,8 +769,7 @@ sparse_attn_kernel(const AttParams P) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    pdl_wait();                                                 // the top-k indices are ready
-    pdl_trigger();
+    pdl_trigger();                                              // producers wait for the selection themselves
     if (warp < kAttSoftWarps) {
         att_softmax(P, sm, tmem, b0, nblk);
     } else if (warp < kAttSoftWarps + kAttProdWarps) {
