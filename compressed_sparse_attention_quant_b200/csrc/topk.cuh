@@ -17,20 +17,22 @@
 //   pass A   one read of the CTA's scores (L2-resident): keys in bins above
 //            b1 are certainly selected and set bits of a shared-memory
 //            bitmap over the window; keys in bin b1 are candidates, counted
-//            into a histogram of their next 11 bits and kept (key, position)
-//            in shared memory while they fit.
+//            into a histogram of their next 11 bits and marked in a second
+//            bitmap (both bitmaps assembled from 4-bit pieces by shuffles).
 //   level 2/3 the CTAs sum their histograms through distributed shared
 //            memory (every CTA reads every peer's), so each CTA picks the same
 //            digit; level 3 is skipped when the level-2 bin is taken whole.
 //   emit     candidates above the threshold key join the bitmap, candidates
-//            equal to it go to a tie bitmap; one exchange of (selected, ties)
+//            equal to it go to a tie bitmap (level 3 and the emission re-read
+//            only the candidates' scores, each thread over its own bitmap
+//            words); one exchange of (selected, ties)
 //            counts across the cluster gives each CTA its first tie rank and
 //            output offset, ties are taken lowest position first, and each
 //            thread writes the positions of its contiguous bitmap words.
-// If some CTA's candidates overflow its shared list, or the row needs more
-// than one round, the levels and the emission re-read the scores instead of
-// the list (same result, more L2 reads). Cluster barriers are the only
-// waits, and every CTA of a cluster takes the same branches.
+// If the row needs more than one round of windows, the levels and the
+// emission re-read all the scores instead of the candidate bitmap (same
+// result, more L2 reads). Cluster barriers are the only waits, and every
+// CTA of a cluster takes the same branches.
 #pragma once
 
 #include "common.cuh"
@@ -43,7 +45,6 @@ namespace csa2 {
 constexpr int kTkThreads = 1024;
 constexpr int kTkWin = 1 << 17;                  // positions per CTA window
 constexpr int kTkWinWords = kTkWin / 32;
-constexpr int kTkCandCap = 12288;                // candidates kept in shared memory per CTA
 constexpr int kTkMaxCluster = 16;
 
 // Zeroes the per-row level-1 histograms before the indexer accumulates them.
@@ -193,16 +194,13 @@ __device__ __forceinline__ void warp_pick(const uint32_t *h, int nbins, uint32_t
 struct TkSmem {
     uint32_t sel[kTkWinWords];          // 16 KB: selected positions of the window
     uint32_t tie[kTkWinWords];          // 16 KB: positions whose key equals the threshold
-    uint32_t ckey[kTkCandCap];          // 48 KB: candidate keys (bin b1)
-    int32_t cpos[kTkCandCap];           // 48 KB: candidate positions
+    uint32_t cand[kTkWinWords];         // 16 KB: positions whose key is in the level-1 bin b1
     uint32_t hloc[2][kTopkBins];        // this CTA's level-2 / level-3 histograms (read by peers)
     uint32_t hsum[kTopkBinsPadded];     // cluster-wide sum of the current level (padded, hpad)
     uint32_t wsel[kTkThreads / 32];     // per-warp counts of the emission
     uint32_t wtie[kTkThreads / 32];
     uint32_t xchg[2][2];                // per round parity: (selected before ties, ties), read by peers
-    uint32_t n_cand;
     uint32_t s_pick[2];                 // (bin / digit, count above) of the current level
-    uint32_t s_flag;
 };
 
 // Guarded float4 of scores at positions p .. p+3 (< w1 only).
@@ -258,7 +256,6 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     };
 
     for (int i = tid; i < 2 * kTopkBins; i += kTkThreads) (&sm.hloc[0][0])[i] = 0u;
-    if (tid == 0) sm.n_cand = 0u;
     // ---- level 1: one warp scans the indexer's histogram of the row
     if (warp == 0) {
         uint32_t b1w, a1w;
@@ -331,23 +328,12 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
                     sw |= __shfl_xor_sync(0xffffffffu, sw, 4);
                     if ((lane & 7) == 0) sm.sel[(p - w0) >> 5] = sw;
                 }
-                // candidates of this piece -> the shared list (warp-aggregated slots)
-                const uint32_t cnt = __popc(cn);
-                if (fast && __any_sync(0xffffffffu, cnt != 0u)) {
-                    const uint32_t incl = warp_incl_scan(cnt);
-                    uint32_t base = 0u;
-                    if (lane == 31) base = atomicAdd(&sm.n_cand, incl);
-                    base = __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        if ((cn >> e) & 1u) {
-                            if (base < static_cast<uint32_t>(kTkCandCap)) {
-                                sm.ckey[base] = float_key(fv[e]);
-                                sm.cpos[base] = static_cast<int32_t>(p + e);
-                            }
-                            ++base;
-                        }
-                    }
+                if (fast) {                                  // candidate word (bin b1), same assembly
+                    uint32_t cw = cn << (4 * (lane & 7));
+                    cw |= __shfl_xor_sync(0xffffffffu, cw, 1);
+                    cw |= __shfl_xor_sync(0xffffffffu, cw, 2);
+                    cw |= __shfl_xor_sync(0xffffffffu, cw, 4);
+                    if ((lane & 7) == 0) sm.cand[(p - w0) >> 5] = cw;
                 }
             }
         }
@@ -360,13 +346,8 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
         for (int q = 0; q < C; ++q) v += cluster.map_shared_rank(&sm.hloc[0][0], q)[i];
         sm.hsum[hpad(i)] = v;
     }
-    if (tid == 0) {
-        uint32_t of = 0u;
-        for (int q = 0; q < C; ++q) of |= *cluster.map_shared_rank(&sm.n_cand, q) > static_cast<uint32_t>(kTkCandCap);
-        sm.s_flag = of;
-    }
     __syncthreads();
-    const bool use_list = fast && sm.s_flag == 0u;
+    const bool use_list = fast;                         // the candidate words of a single-round window
     if (warp == 0) {
         uint32_t d, a;
         warp_pick<false>(sm.hsum, kTopkBins, need, d, a);
@@ -384,10 +365,26 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     if (cnt2 != need) {
         // ---- level 3: the low 10 bits of the keys with this 22-bit prefix
         if (use_list) {
-            const uint32_t nc = sm.n_cand;
-            for (uint32_t i = tid; i < nc; i += kTkThreads) {
-                const uint32_t key = sm.ckey[i];
-                if ((key >> 10) == prefix) atomicAdd(&sm.hloc[1][key & 1023u], 1u);
+            int64_t w0, w1;
+            win(0, w0, w1);
+            const int64_t t0 = w0 + static_cast<int64_t>(tid) * P;
+            for (int wi = 0; wi < NW; ++wi) {
+                uint32_t m = sm.cand[tid * NW + wi];
+                while (m) {                                  // four candidates' loads in flight at a time
+                    int bit[4];
+                    float f[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        bit[u] = m ? __ffs(m) - 1 : -1;
+                        m &= m - 1u;
+                        f[u] = bit[u] >= 0 ? __ldcg(srow + t0 + 32 * wi + bit[u]) : 0.0f;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t key = float_key(f[u]);
+                        if (bit[u] >= 0 && (key >> 10) == prefix) atomicAdd(&sm.hloc[1][key & 1023u], 1u);
+                    }
+                }
             }
         } else {
             for (int r = 0; r < rounds; ++r) {
@@ -436,15 +433,29 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
         win(r, w0, w1);
         const int64_t t0 = w0 + static_cast<int64_t>(tid) * P;
         if (use_list) {
-            for (int wi = 0; wi < NW; ++wi) sm.tie[tid * NW + wi] = 0u;
-            __syncthreads();                            // tie words zero before any candidate lands
-            const uint32_t nc = sm.n_cand;
-            for (uint32_t i = tid; i < nc; i += kTkThreads) {
-                const uint32_t key = sm.ckey[i];
-                const uint32_t top = bits == 32 ? key : key >> 10;
-                const int64_t rel = sm.cpos[i] - w0;
-                if (top > prefix) atomicOr(&sm.sel[rel >> 5], 1u << (rel & 31));
-                else if (top == prefix) atomicOr(&sm.tie[rel >> 5], 1u << (rel & 31));
+            // this thread's candidate words: above the threshold -> selected, equal -> tie
+            for (int wi = 0; wi < NW; ++wi) {
+                uint32_t m = sm.cand[tid * NW + wi], s4 = 0u, t4 = 0u;
+                while (m) {                                  // four candidates' loads in flight at a time
+                    int bit[4];
+                    float f[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        bit[u] = m ? __ffs(m) - 1 : -1;
+                        m &= m - 1u;
+                        f[u] = bit[u] >= 0 ? __ldcg(srow + t0 + 32 * wi + bit[u]) : 0.0f;
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if (bit[u] < 0) continue;
+                        const uint32_t key = float_key(f[u]);
+                        const uint32_t top = bits == 32 ? key : key >> 10;
+                        if (top > prefix) s4 |= 1u << bit[u];
+                        else if (top == prefix) t4 |= 1u << bit[u];
+                    }
+                }
+                sm.sel[tid * NW + wi] |= s4;
+                sm.tie[tid * NW + wi] = t4;
             }
         } else {
             for (int wi = 0; wi < NW; ++wi) {
