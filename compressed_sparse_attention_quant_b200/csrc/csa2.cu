@@ -147,28 +147,44 @@ IdxLayout idx_layout(int B, int Sq, int max_pages, int k) {
 
 // ---------------------------------------------------------------- attention work plan
 struct AttPlan {
-    int n_win;           // window blocks per query row (1, or 0 without a window)
-    int n_st;            // blocks of 128 keys per query row
-    int64_t total;       // blocks over all rows
-    int grid;            // CTAs (each a contiguous range of blocks)
+    int n_win;           // window tiles per query row (2, or 0 without a window)
+    int n_st;            // tiles of 64 keys per query row
+    int n_splits;        // S: runs per row, one CTA each
+    int tps;             // tiles per run
+    int R;
 };
 
-// One persistent CTA per SM (at most one wave), each with at least one block.
+// Split each row's tiles into S runs so that the R * S CTAs fill the machine:
+// minimise waves x tiles per CTA, with a small charge per run for writing and
+// merging its partial.
 AttPlan att_plan(int R, int k, int slots, bool window = true) {
     AttPlan pl;
-    pl.n_win = window ? 1 : 0;
-    pl.n_st = pl.n_win + (k + kAttBlk - 1) / kAttBlk;
-    pl.total = static_cast<int64_t>(R) * pl.n_st;
-    pl.grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(std::min(slots, kMergeMaxParts), pl.total)));
+    pl.R = R;
+    pl.n_win = window ? kWindow / kAttTile : 0;
+    pl.n_st = pl.n_win + (k + kAttTile - 1) / kAttTile;
+    pl.n_splits = 1;
+    pl.tps = pl.n_st;
+    double best = 1e30;
+    for (int s = 1; s <= pl.n_st && s <= kMergeMaxParts; ++s) {
+        const int tps = (pl.n_st + s - 1) / s;
+        const int s_eff = (pl.n_st + tps - 1) / tps;
+        if (s_eff > 1 && static_cast<int64_t>(R) * s_eff > slots) break;   // split only within one wave
+        const int64_t waves = (static_cast<int64_t>(R) * s_eff + slots - 1) / slots;
+        const double cost = static_cast<double>(waves) * tps + (s_eff > 1 ? 0.25 * s_eff : 0.0);
+        if (cost < best - 1e-9) {
+            best = cost;
+            pl.n_splits = s_eff;
+            pl.tps = tps;
+        }
+    }
     return pl;
 }
 
-// Partials: two per CTA (the first and the last row segment of its range).
+// Partials: one per (row, run) when a row is split.
 size_t att_ws_bytes(const AttPlan &pl) {
-    if (pl.grid <= 1) return 0;
-    const size_t po = round_up(static_cast<size_t>(2) * pl.grid * kHeads * kDim * 4, 256);
-    const size_t pm = round_up(static_cast<size_t>(2) * pl.grid * kHeads * 8, 256);
-    return po + pm;
+    if (pl.n_splits <= 1) return 0;
+    const size_t n = static_cast<size_t>(pl.R) * pl.n_splits;
+    return round_up(n * kHeads * kDim * 4, 256) + round_up(n * kHeads * 8, 256);
 }
 
 csa2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
@@ -427,7 +443,8 @@ size_t csa2_sparse_attn_workspace_bytes(int B, int Sq, int k) {
     if (B <= 0 || Sq <= 0 || k < 0 || k > 65536 || static_cast<int64_t>(B) * Sq > 65535) return 0;
     DeviceInfo *dev = nullptr;
     if (device_info(&dev) != cudaSuccess) return 0;
-    return att_ws_bytes(att_plan(B * Sq, k, dev->sm_count * dev->att_ctas_per_sm));
+    const int slots = dev->sm_count * dev->att_ctas_per_sm;
+    return std::max(att_ws_bytes(att_plan(B * Sq, k, slots, true)), att_ws_bytes(att_plan(B * Sq, k, slots, false)));
 }
 
 csa2_status csa2_sparse_attn_decode(const void *q_bf16, int B, int Sq, int H, int D,
@@ -472,21 +489,21 @@ csa2_status csa2_sparse_attn_decode(const void *q_bf16, int B, int Sq, int H, in
     P.part_o = nullptr;
     P.part_ml = nullptr;
     P.n_win = pl.n_win;
-    P.n_st = pl.n_st;
-    P.total_steps = pl.total;
+    P.n_splits = pl.n_splits;
+    P.tiles_per_split = pl.tps;
     if (need > 0) {
         uint8_t *base = static_cast<uint8_t *>(ws);
         P.part_o = reinterpret_cast<float *>(base);
         P.part_ml = reinterpret_cast<float2 *>(
-            base + round_up(static_cast<size_t>(2) * pl.grid * kHeads * kDim * 4, 256));
+            base + round_up(static_cast<size_t>(R) * pl.n_splits * kHeads * kDim * 4, 256));
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_pdl(sparse_attn_kernel, dim3(pl.grid), dim3(kAttThreads), kAttSmemBytes, st, P);
+    cudaError_t e = launch_pdl(sparse_attn_kernel, dim3(pl.n_splits, R), dim3(kAttThreads), kAttSmemBytes, st, P);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
-    if (pl.grid > 1) {
+    if (pl.n_splits > 1) {
         e = launch_pdl(attn_merge_kernel, dim3(R, kHeads / kMergeHeads), dim3(kMergeThreads), 0, st,
-                       static_cast<const float *>(P.part_o), static_cast<const float2 *>(P.part_ml), pl.total,
-                       pl.n_st, pl.grid, out, lse);
+                       static_cast<const float *>(P.part_o), static_cast<const float2 *>(P.part_ml), pl.n_splits,
+                       out, lse);
     }
     return cuda_status(e);
 }

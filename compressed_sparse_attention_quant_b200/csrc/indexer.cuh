@@ -414,14 +414,11 @@ indexer_score_kernel(const IdxArgs A) {
                         st_policy(srow + qq * A.t_cap, score, pol_keep);
                         // Scores crowd into few bins: lanes with the same bin add
                         // their count with one atomic (the lowest such lane).
-                        const bool live = t <= cur_T - Sq + qq;
-                        const uint32_t bin = live ? float_key(score) >> kTopkDigitShift : 0xFFFFFFFFu;
-                        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-                        if (live && __ffs(peers) - 1 == lane) {
+                        if (t <= cur_T - Sq + qq) {
+                            const uint32_t bin = float_key(score) >> kTopkDigitShift;
                             const int hr = hrow0 + qq;
-                            const uint32_t n = __popc(peers);
-                            if (hr < kRows) atomicAdd(&sm.hist[hr * kTopkBins + bin], n);
-                            else atomicAdd(&A.hist[(static_cast<int64_t>(cur_b) * Sq + qq) * kTopkBins + bin], n);
+                            if (hr < kRows) atomicAdd(&sm.hist[hr * kTopkBins + bin], 1u);
+                            else atomicAdd(&A.hist[(static_cast<int64_t>(cur_b) * Sq + qq) * kTopkBins + bin], 1u);
                         }
                     }
                 }

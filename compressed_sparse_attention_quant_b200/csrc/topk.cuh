@@ -10,29 +10,26 @@
 // 11 + 11 + 10 bits, run by one thread-block cluster of C CTAs per query row
 // (C = 1..16). CTA r of the cluster owns the position windows
 // [(i*C + r)*W, +W) for rounds i = 0, 1, ... (a single round unless the row
-// exceeds C * 2^17 positions); inside a window each thread owns a contiguous
-// run of positions and the bitmap words over them.
+// exceeds C * 2^17 positions).
 //   level 1  the indexer already built the row's histogram of the top 11 key
 //            bits: every CTA finds the bin b1 holding the k-th largest key.
 //   pass A   one read of the CTA's scores (L2-resident): keys in bins above
 //            b1 are certainly selected and set bits of a shared-memory
 //            bitmap over the window; keys in bin b1 are candidates, counted
-//            into a histogram of their next 11 bits and marked in a second
-//            bitmap (both bitmaps assembled from 4-bit pieces by shuffles).
+//            into a histogram of their next 11 bits and kept (key, position)
+//            in shared memory while they fit.
 //   level 2/3 the CTAs sum their histograms through distributed shared
 //            memory (every CTA reads every peer's), so each CTA picks the same
 //            digit; level 3 is skipped when the level-2 bin is taken whole.
 //   emit     candidates above the threshold key join the bitmap, candidates
-//            equal to it go to a tie bitmap (level 3 and the emission re-read
-//            only the candidates' scores, each thread over its own bitmap
-//            words); one exchange of (selected, ties)
+//            equal to it go to a tie bitmap; one exchange of (selected, ties)
 //            counts across the cluster gives each CTA its first tie rank and
 //            output offset, ties are taken lowest position first, and each
 //            thread writes the positions of its contiguous bitmap words.
-// If the row needs more than one round of windows, the levels and the
-// emission re-read all the scores instead of the candidate bitmap (same
-// result, more L2 reads). Cluster barriers are the only waits, and every
-// CTA of a cluster takes the same branches.
+// If some CTA's candidates overflow its shared list, or the row needs more
+// than one round, the levels and the emission re-read the scores instead of
+// the list (same result, more L2 reads). Cluster barriers are the only
+// waits, and every CTA of a cluster takes the same branches.
 #pragma once
 
 #include "common.cuh"
@@ -45,7 +42,9 @@ namespace csa2 {
 constexpr int kTkThreads = 1024;
 constexpr int kTkWin = 1 << 17;                  // positions per CTA window
 constexpr int kTkWinWords = kTkWin / 32;
+constexpr int kTkCandCap = 12288;                // candidates kept in shared memory per CTA
 constexpr int kTkMaxCluster = 16;
+constexpr int kTkUnroll = 4;                     // float4 loads in flight per thread
 
 // Zeroes the per-row level-1 histograms before the indexer accumulates them.
 __global__ void __launch_bounds__(256) topk_zero_kernel(uint4 *__restrict__ p, int64_t n16) {
@@ -128,6 +127,41 @@ __device__ __forceinline__ uint64_t block_excl_scan64(uint64_t v, uint64_t *wbuf
     return res;
 }
 
+// From the row's 2048-bin histogram (global), the bin holding the need-th
+// largest key, and how many keys lie in higher bins. Every thread of the
+// block gets the answer.
+template <int NT>
+__device__ __forceinline__ void find_threshold_bin(const uint32_t *__restrict__ gh, uint32_t need,
+                                                   uint32_t *wbuf, int *s_bin, uint32_t *s_above,
+                                                   int *bin_out, uint32_t *above_out) {
+    constexpr int PER = kTopkBins / NT;
+    const int top = kTopkBins - 1 - threadIdx.x * PER;   // this thread's bins: top, top-1, ...
+    uint32_t c[PER];
+    uint32_t local = 0u;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        c[i] = __ldcg(&gh[top - i]);
+        local += c[i];
+    }
+    if (threadIdx.x == 0) {                 // stays if the counts fall short of need (corrupt input)
+        *s_bin = 0;
+        *s_above = 0u;
+    }
+    uint32_t tot;
+    uint32_t run = block_excl_scan<NT>(local, wbuf, &tot);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        if (run < need && run + c[i] >= need) {
+            *s_bin = top - i;
+            *s_above = run;
+        }
+        run += c[i];
+    }
+    __syncthreads();
+    *bin_out = *s_bin;
+    *above_out = *s_above;
+}
+
 // Warp-level pick over a histogram of nbins (<= 2048, a multiple of 64) bins
 // in shared or global memory: the bin holding the need-th largest element
 // (bins scanned from the top) and the count in higher bins. Lane l owns the 64
@@ -194,31 +228,68 @@ __device__ __forceinline__ void warp_pick(const uint32_t *h, int nbins, uint32_t
 struct TkSmem {
     uint32_t sel[kTkWinWords];          // 16 KB: selected positions of the window
     uint32_t tie[kTkWinWords];          // 16 KB: positions whose key equals the threshold
-    uint32_t cand[kTkWinWords];         // 16 KB: positions whose key is in the level-1 bin b1
+    uint32_t ckey[kTkCandCap];          // 48 KB: candidate keys (bin b1)
+    int32_t cpos[kTkCandCap];           // 48 KB: candidate positions
     uint32_t hloc[2][kTopkBins];        // this CTA's level-2 / level-3 histograms (read by peers)
-    uint32_t hsum[kTopkBinsPadded];     // cluster-wide sum of the current level (padded, hpad)
-    uint32_t wsel[kTkThreads / 32];     // per-warp counts of the emission
-    uint32_t wtie[kTkThreads / 32];
+    uint32_t hsum[kTopkBins];           // cluster-wide sum of the current level
+    uint32_t wbuf[kTkThreads / 32 + 1];
+    uint64_t wbuf64[kTkThreads / 32 + 1];
     uint32_t xchg[2][2];                // per round parity: (selected before ties, ties), read by peers
-    uint32_t s_pick[2];                 // (bin / digit, count above) of the current level
+    uint32_t n_cand;
+    int s_bin;
+    uint32_t s_above;
+    uint32_t s_digit;
+    uint32_t s_cum;
+    uint32_t s_flag;
+    uint32_t s_base[4];
 };
 
+// Digit of the need-th largest element of a histogram of nbins (<= 2048)
+// bins, and the count of elements in higher bins.
+__device__ __forceinline__ void tk_pick(TkSmem &sm, const uint32_t *h, int nbins, uint32_t need, uint32_t &digit,
+                                        uint32_t &above) {
+    const int top = kTopkBins - 1 - static_cast<int>(threadIdx.x) * 2;
+    if (threadIdx.x == 0) {                 // stays if the counts fall short of need (corrupt input)
+        sm.s_digit = 0u;
+        sm.s_cum = 0u;
+    }
+    const uint32_t c0 = top < nbins ? h[top] : 0u;
+    const uint32_t c1 = top - 1 < nbins ? h[top - 1] : 0u;
+    uint32_t tot;
+    const uint32_t run = block_excl_scan<kTkThreads>(c0 + c1, sm.wbuf, &tot);
+    if (run < need && run + c0 >= need) {
+        sm.s_digit = static_cast<uint32_t>(top);
+        sm.s_cum = run;
+    } else if (run + c0 < need && run + c0 + c1 >= need) {
+        sm.s_digit = static_cast<uint32_t>(top - 1);
+        sm.s_cum = run + c0;
+    }
+    __syncthreads();
+    digit = sm.s_digit;
+    above = sm.s_cum;
+    __syncthreads();
+}
+
 // Guarded float4 of scores at positions p .. p+3 (< w1 only).
-__device__ __forceinline__ float4 tk_load(const float *srow, int64_t p, int64_t w1) {
-    if (p + 4 <= w1) return __ldcg(reinterpret_cast<const float4 *>(srow + p));
+__device__ __forceinline__ float4 tk_load(const float *srow, int64_t p, int64_t w1, bool live) {
+    if (live && p + 4 <= w1) return __ldcg(reinterpret_cast<const float4 *>(srow + p));
     float t[4] = {0.f, 0.f, 0.f, 0.f};
+    if (live)
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-        if (p + u < w1) t[u] = __ldcg(srow + p + u);
+        for (int u = 0; u < 4; ++u)
+            if (p + u < w1) t[u] = __ldcg(srow + p + u);
     return make_float4(t[0], t[1], t[2], t[3]);
 }
 
-// Work layout: in each round the CTA's window of Wn positions is split into
-// contiguous runs of P = Wn / 1024 positions (a multiple of 32), one per
-// thread, so a thread's bitmap words hold only its own positions and need no
-// exchange between lanes. Warp-level scans replace block-wide ones: every
-// level and the emission take one CTA barrier plus, for the cluster-wide
-// counts, one cluster barrier.
+// OR of a 4-bit group over the 8 lanes sharing one 32-position bitmap word.
+__device__ __forceinline__ uint32_t tk_word(uint32_t nib) {
+    uint32_t w = nib << ((threadIdx.x & 7) * 4);
+    w |= __shfl_xor_sync(0xffffffffu, w, 1);
+    w |= __shfl_xor_sync(0xffffffffu, w, 2);
+    w |= __shfl_xor_sync(0xffffffffu, w, 4);
+    return w;
+}
+
 __global__ void __launch_bounds__(kTkThreads, 1)
 topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint32_t *__restrict__ hist,
                     const int32_t *__restrict__ seq_lens, int Sq, int max_pages, int k, int32_t *__restrict__ out,
@@ -230,7 +301,7 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     const int C = static_cast<int>(cluster.num_blocks());
     const int rank = static_cast<int>(cluster.block_rank());
     const int row = blockIdx.x / C;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     pdl_wait();                                         // scores and histograms are complete
     pdl_trigger();
     const int n_valid = topk_n_valid(seq_lens, row, Sq, max_pages);
@@ -246,94 +317,115 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     }
     const int64_t per = (static_cast<int64_t>(n_valid) + C - 1) / C;
     const int64_t Wn = min(static_cast<int64_t>(kTkWin), (per + 31) / 32 * 32);
-    const int NW = static_cast<int>((Wn / 32 + kTkThreads - 1) / kTkThreads);   // bitmap words per thread: 1 .. 4
-    const int P = 32 * NW;                              // positions per thread (threads past Wn have none)
     const int rounds = static_cast<int>((n_valid + C * Wn - 1) / (C * Wn));
     const bool fast = rounds == 1;
-    auto win = [&](int r, int64_t &w0, int64_t &w1) {
+    auto win = [&](int r, int64_t &w0, int64_t &w1, int &n_it) {
         w0 = (static_cast<int64_t>(r) * C + rank) * Wn;
         w1 = min(w0 + Wn, static_cast<int64_t>(n_valid));
+        n_it = w1 > w0 ? static_cast<int>((w1 - w0 + 4 * kTkThreads - 1) / (4 * kTkThreads)) : 0;
     };
 
     for (int i = tid; i < 2 * kTopkBins; i += kTkThreads) (&sm.hloc[0][0])[i] = 0u;
-    // ---- level 1: one warp scans the indexer's histogram of the row
-    if (warp == 0) {
-        uint32_t b1w, a1w;
-        warp_pick<true>(hist + static_cast<int64_t>(row) * kTopkBins, kTopkBins, static_cast<uint32_t>(k), b1w, a1w);
-        if (lane == 0) {
-            sm.s_pick[0] = b1w;
-            sm.s_pick[1] = a1w;
-        }
-    }
-    __syncthreads();
-    const int b1 = static_cast<int>(sm.s_pick[0]);
-    uint32_t need = static_cast<uint32_t>(k) - sm.s_pick[1];
+    if (tid == 0) sm.n_cand = 0u;
+    // ---- level 1: from the indexer's histogram
+    int b1;
+    uint32_t above1;
+    find_threshold_bin<kTkThreads>(hist + static_cast<int64_t>(row) * kTopkBins, static_cast<uint32_t>(k), sm.wbuf,
+                                   &sm.s_bin, &sm.s_above, &b1, &above1);
+    uint32_t need = static_cast<uint32_t>(k) - above1;
 
     // ---- pass A: sure bits, level-2 histogram, candidate list
     // With a positive threshold bin (1024 < b1 < 2047) a score is above b1,
     // or in b1, exactly when its IEEE bits as a signed integer are at least
     // hi_bits, or in [lo_bits, hi_bits): negative scores and -0 fall below
-    // both. Otherwise the order-preserving key decides.
+    // both. That skips the key transform for all but the candidates.
     const bool pos = b1 > 1024 && b1 < kTopkBins - 1;
     const int32_t lo_bits = (b1 - 1024) << kTopkDigitShift;
     const int32_t hi_bits = (b1 - 1023) << kTopkDigitShift;
-    auto classify = [&](float f, int64_t p, int64_t w1, bool &sure, bool &cand, uint32_t &key) {
-        key = float_key(f);
-        if (p >= w1) {
-            sure = cand = false;
-        } else if (pos) {
-            const int32_t bits = __float_as_int(f);
-            sure = bits >= hi_bits;
-            cand = !sure && bits >= lo_bits;
-        } else {
-            const int bin = static_cast<int>(key >> kTopkDigitShift);
-            sure = bin > b1;
-            cand = bin == b1;
-        }
-    };
-    // Loads are coalesced: lane L of warp w reads positions wb + 128 j + 4 L
-    // .. + 3 (wb = the warp's first position); the eight lanes 8q .. 8q + 7
-    // of iteration j cover one 32-position bitmap word, which three
-    // shuffles assemble from their 4-bit pieces. The words are the same ones
-    // the owning threads read later.
     for (int r = 0; r < rounds; ++r) {
         int64_t w0, w1;
-        win(r, w0, w1);
-        const int64_t wb = w0 + static_cast<int64_t>(warp) * 32 * P;
-        const int n_it = P / 4;                          // 8 * NW iterations of 128 positions
-        for (int j0 = 0; j0 < n_it; j0 += 4) {
-            float4 f[4];
+        int n_it;
+        win(r, w0, w1, n_it);
+        for (int i0 = 0; i0 < n_it; i0 += kTkUnroll) {
+            float4 f[kTkUnroll];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) f[u] = tk_load(srow, wb + 128 * (j0 + u) + 4 * lane, w1);
+            for (int u = 0; u < kTkUnroll; ++u)
+                f[u] = tk_load(srow, w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) + tid * 4, w1,
+                               i0 + u < n_it);
+            uint32_t cmask = 0u;                         // 4 bits per unrolled load
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int64_t p = wb + 128 * (j0 + u) + 4 * lane;
+            for (int u = 0; u < kTkUnroll; ++u) {
+                const int64_t p = w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) + tid * 4;
                 const float fv[4] = {f[u].x, f[u].y, f[u].z, f[u].w};
-                uint32_t sn = 0u, cn = 0u;
+                uint32_t s4 = 0u;
+                // one bounds check per float4; per element only on the ragged tail
+                const bool full4 = i0 + u < n_it && p + 4 <= w1;
+                if (pos && full4) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    bool su, ca;
-                    uint32_t key;
-                    classify(fv[e], p + e, w1, su, ca, key);
-                    sn |= (su ? 1u : 0u) << e;
-                    if (ca) {
-                        cn |= 1u << e;
-                        atomicAdd(&sm.hloc[0][(key >> 10) & (kTopkBins - 1)], 1u);
+                    for (int e = 0; e < 4; ++e) {
+                        const int32_t bits = __float_as_int(fv[e]);
+                        if (bits >= lo_bits) {
+                            if (bits >= hi_bits) {
+                                s4 |= 1u << e;
+                            } else {
+                                cmask |= 1u << (4 * u + e);
+                                atomicAdd(&sm.hloc[0][(static_cast<uint32_t>(bits) >> 10) & (kTopkBins - 1)], 1u);
+                            }
+                        }
+                    }
+                } else if (pos) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int32_t bits = __float_as_int(fv[e]);
+                        if (i0 + u < n_it && p + e < w1 && bits >= lo_bits) {
+                            if (bits >= hi_bits) {
+                                s4 |= 1u << e;
+                            } else {
+                                cmask |= 1u << (4 * u + e);
+                                atomicAdd(&sm.hloc[0][(static_cast<uint32_t>(bits) >> 10) & (kTopkBins - 1)], 1u);
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t key = float_key(fv[e]);
+                        const int bin = static_cast<int>(key >> kTopkDigitShift);
+                        if (i0 + u < n_it && p + e < w1) {
+                            if (bin > b1) s4 |= 1u << e;
+                            if (bin == b1) {
+                                cmask |= 1u << (4 * u + e);
+                                atomicAdd(&sm.hloc[0][(key >> 10) & (kTopkBins - 1)], 1u);
+                            }
+                        }
                     }
                 }
                 if (fast) {
-                    uint32_t sw = sn << (4 * (lane & 7));
-                    sw |= __shfl_xor_sync(0xffffffffu, sw, 1);
-                    sw |= __shfl_xor_sync(0xffffffffu, sw, 2);
-                    sw |= __shfl_xor_sync(0xffffffffu, sw, 4);
-                    if ((lane & 7) == 0) sm.sel[(p - w0) >> 5] = sw;
+                    const uint32_t w = tk_word(s4);
+                    if ((tid & 7) == 0 && i0 + u < n_it) sm.sel[(i0 + u) * (kTkThreads / 8) + (tid >> 3)] = w;
                 }
-                if (fast) {                                  // candidate word (bin b1), same assembly
-                    uint32_t cw = cn << (4 * (lane & 7));
-                    cw |= __shfl_xor_sync(0xffffffffu, cw, 1);
-                    cw |= __shfl_xor_sync(0xffffffffu, cw, 2);
-                    cw |= __shfl_xor_sync(0xffffffffu, cw, 4);
-                    if ((lane & 7) == 0) sm.cand[(p - w0) >> 5] = cw;
+            }
+            if (fast && __any_sync(0xffffffffu, cmask != 0u)) {
+                const uint32_t cnt = __popc(cmask);
+                const uint32_t incl = warp_incl_scan(cnt);
+                uint32_t base = 0u;
+                if ((tid & 31) == 31) base = atomicAdd(&sm.n_cand, incl);
+                base = __shfl_sync(0xffffffffu, base, 31) + incl - cnt;
+                while (cmask) {
+                    const int bit = __ffs(cmask) - 1;
+                    cmask &= cmask - 1u;
+                    const int u = bit >> 2, e = bit & 3;
+                    float4 fu = f[0];
+#pragma unroll
+                    for (int uu = 1; uu < kTkUnroll; ++uu)
+                        if (u == uu) fu = f[uu];                 // register select, no local array
+                    const float v = e == 0 ? fu.x : e == 1 ? fu.y : e == 2 ? fu.z : fu.w;
+                    if (base < static_cast<uint32_t>(kTkCandCap)) {
+                        sm.ckey[base] = float_key(v);
+                        sm.cpos[base] = static_cast<int32_t>(w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) +
+                                                             tid * 4 + e);
+                    }
+                    ++base;
                 }
             }
         }
@@ -344,60 +436,42 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     for (int i = tid; i < kTopkBins; i += kTkThreads) {
         uint32_t v = 0u;
         for (int q = 0; q < C; ++q) v += cluster.map_shared_rank(&sm.hloc[0][0], q)[i];
-        sm.hsum[hpad(i)] = v;
+        sm.hsum[i] = v;
+    }
+    if (tid == 0) {
+        uint32_t of = 0u;
+        for (int q = 0; q < C; ++q) of |= *cluster.map_shared_rank(&sm.n_cand, q) > static_cast<uint32_t>(kTkCandCap);
+        sm.s_flag = of;
     }
     __syncthreads();
-    const bool use_list = fast;                         // the candidate words of a single-round window
-    if (warp == 0) {
-        uint32_t d, a;
-        warp_pick<false>(sm.hsum, kTopkBins, need, d, a);
-        if (lane == 0) {
-            sm.s_pick[0] = d;
-            sm.s_pick[1] = a;
-        }
-    }
-    __syncthreads();
-    const uint32_t d2 = sm.s_pick[0], above2 = sm.s_pick[1];
-    const uint32_t cnt2 = sm.hsum[hpad(static_cast<int>(d2))];
+    const bool use_list = fast && sm.s_flag == 0u;
+    uint32_t d2, above2;
+    tk_pick(sm, sm.hsum, kTopkBins, need, d2, above2);
+    const uint32_t cnt2 = sm.hsum[d2];
     need -= above2;
     uint32_t prefix = (static_cast<uint32_t>(b1) << 11) | d2;
     int bits = 22;
     if (cnt2 != need) {
         // ---- level 3: the low 10 bits of the keys with this 22-bit prefix
         if (use_list) {
-            int64_t w0, w1;
-            win(0, w0, w1);
-            const int64_t t0 = w0 + static_cast<int64_t>(tid) * P;
-            for (int wi = 0; wi < NW; ++wi) {
-                uint32_t m = sm.cand[tid * NW + wi];
-                while (m) {                                  // four candidates' loads in flight at a time
-                    int bit[4];
-                    float f[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        bit[u] = m ? __ffs(m) - 1 : -1;
-                        m &= m - 1u;
-                        f[u] = bit[u] >= 0 ? __ldcg(srow + t0 + 32 * wi + bit[u]) : 0.0f;
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint32_t key = float_key(f[u]);
-                        if (bit[u] >= 0 && (key >> 10) == prefix) atomicAdd(&sm.hloc[1][key & 1023u], 1u);
-                    }
-                }
+            const uint32_t nc = sm.n_cand;
+            for (uint32_t i = tid; i < nc; i += kTkThreads) {
+                const uint32_t key = sm.ckey[i];
+                if ((key >> 10) == prefix) atomicAdd(&sm.hloc[1][key & 1023u], 1u);
             }
         } else {
             for (int r = 0; r < rounds; ++r) {
                 int64_t w0, w1;
-                win(r, w0, w1);
-                const int64_t t0 = w0 + static_cast<int64_t>(tid) * P;
-                for (int i = 0; i < P; i += 4) {
-                    const float4 f = tk_load(srow, t0 + i, w1);
+                int n_it;
+                win(r, w0, w1, n_it);
+                for (int i = 0; i < n_it; ++i) {
+                    const int64_t p = w0 + static_cast<int64_t>(i) * (4 * kTkThreads) + tid * 4;
+                    const float4 f = tk_load(srow, p, w1, true);
                     const float fv[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const uint32_t key = float_key(fv[e]);
-                        if (t0 + i + e < w1 && (key >> 10) == prefix) atomicAdd(&sm.hloc[1][key & 1023u], 1u);
+                        if (p + e < w1 && (key >> 10) == prefix) atomicAdd(&sm.hloc[1][key & 1023u], 1u);
                     }
                 }
             }
@@ -406,19 +480,11 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
         for (int i = tid; i < 1024; i += kTkThreads) {
             uint32_t v = 0u;
             for (int q = 0; q < C; ++q) v += cluster.map_shared_rank(&sm.hloc[1][0], q)[i];
-            sm.hsum[hpad(i)] = v;
+            sm.hsum[i] = v;
         }
         __syncthreads();
-        if (warp == 0) {
-            uint32_t d, a;
-            warp_pick<false>(sm.hsum, 1024, need, d, a);
-            if (lane == 0) {
-                sm.s_pick[0] = d;
-                sm.s_pick[1] = a;
-            }
-        }
-        __syncthreads();
-        const uint32_t d3 = sm.s_pick[0], above3 = sm.s_pick[1];
+        uint32_t d3, above3;
+        tk_pick(sm, sm.hsum, 1024, need, d3, above3);
         need -= above3;
         prefix = (prefix << 10) | d3;
         bits = 32;
@@ -430,151 +496,120 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     uint32_t out_base = 0u, tie_base = 0u;
     for (int r = 0; r < rounds; ++r) {
         int64_t w0, w1;
-        win(r, w0, w1);
-        const int64_t t0 = w0 + static_cast<int64_t>(tid) * P;
+        int n_it;
+        win(r, w0, w1, n_it);
+        const int nw = w1 > w0 ? static_cast<int>((w1 - w0 + 31) / 32) : 0;
+        __syncthreads();                                // the previous round's bitmaps are consumed
         if (use_list) {
-            // this thread's candidate words: above the threshold -> selected, equal -> tie
-            for (int wi = 0; wi < NW; ++wi) {
-                uint32_t m = sm.cand[tid * NW + wi], s4 = 0u, t4 = 0u;
-                while (m) {                                  // four candidates' loads in flight at a time
-                    int bit[4];
-                    float f[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        bit[u] = m ? __ffs(m) - 1 : -1;
-                        m &= m - 1u;
-                        f[u] = bit[u] >= 0 ? __ldcg(srow + t0 + 32 * wi + bit[u]) : 0.0f;
-                    }
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        if (bit[u] < 0) continue;
-                        const uint32_t key = float_key(f[u]);
-                        const uint32_t top = bits == 32 ? key : key >> 10;
-                        if (top > prefix) s4 |= 1u << bit[u];
-                        else if (top == prefix) t4 |= 1u << bit[u];
-                    }
-                }
-                sm.sel[tid * NW + wi] |= s4;
-                sm.tie[tid * NW + wi] = t4;
+            for (int i = tid; i < nw; i += kTkThreads) sm.tie[i] = 0u;
+            __syncthreads();
+            const uint32_t nc = sm.n_cand;
+            for (uint32_t i = tid; i < nc; i += kTkThreads) {
+                const uint32_t key = sm.ckey[i];
+                const uint32_t top = bits == 32 ? key : key >> 10;
+                const int64_t rel = sm.cpos[i] - w0;
+                if (top > prefix) atomicOr(&sm.sel[rel >> 5], 1u << (rel & 31));
+                else if (top == prefix) atomicOr(&sm.tie[rel >> 5], 1u << (rel & 31));
             }
         } else {
-            for (int wi = 0; wi < NW; ++wi) {
+            for (int i = 0; i < n_it; ++i) {
+                const int64_t p = w0 + static_cast<int64_t>(i) * (4 * kTkThreads) + tid * 4;
+                const float4 f = tk_load(srow, p, w1, true);
+                const float fv[4] = {f.x, f.y, f.z, f.w};
                 uint32_t s4 = 0u, t4 = 0u;
-                for (int i = 0; i < 32; i += 4) {
-                    const int64_t p = t0 + 32 * wi + i;
-                    const float4 f = tk_load(srow, p, w1);
-                    const float fv[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint32_t key = float_key(fv[e]);
-                        const uint32_t top = bits == 32 ? key : key >> 10;
-                        if (p + e < w1) {
-                            if (top > prefix) s4 |= 1u << (i + e);
-                            else if (top == prefix) t4 |= 1u << (i + e);
-                        }
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t key = float_key(fv[e]);
+                    const uint32_t top = bits == 32 ? key : key >> 10;
+                    if (p + e < w1) {
+                        if (top > prefix) s4 |= 1u << e;
+                        else if (top == prefix) t4 |= 1u << e;
                     }
                 }
-                sm.sel[tid * NW + wi] = s4;
-                sm.tie[tid * NW + wi] = t4;
+                const uint32_t ws = tk_word(s4), wt = tk_word(t4);
+                if ((tid & 7) == 0) {
+                    sm.sel[i * (kTkThreads / 8) + (tid >> 3)] = ws;
+                    sm.tie[i * (kTkThreads / 8) + (tid >> 3)] = wt;
+                }
             }
         }
         __syncthreads();
-        // counts of this thread's words, then of its warp (warp-level scans)
-        uint32_t n_sel = 0u, n_tie = 0u;
-        for (int wi = 0; wi < NW; ++wi) {
-            n_sel += __popc(sm.sel[tid * NW + wi]);
-            n_tie += __popc(sm.tie[tid * NW + wi]);
+        // thread t owns the contiguous words [wb, we)
+        const int wper = (nw + kTkThreads - 1) / kTkThreads;
+        const int wb = min(tid * wper, nw), we = min(wb + wper, nw);
+        uint32_t n_tie = 0u, n_sel = 0u;
+        for (int i = wb; i < we; ++i) {
+            n_tie += __popc(sm.tie[i]);
+            n_sel += __popc(sm.sel[i]);
         }
-        const uint32_t is_ = warp_incl_scan(n_sel), it_ = warp_incl_scan(n_tie);
-        if (lane == 31) {
-            sm.wsel[warp] = is_;
-            sm.wtie[warp] = it_;
-        }
-        __syncthreads();
-        uint32_t cta_sel = 0u, cta_tie = 0u, wsel_before = 0u, wtie_before = 0u;
-        for (int w = 0; w < kTkThreads / 32; ++w) {
-            const uint32_t a = sm.wsel[w], t = sm.wtie[w];
-            if (w < warp) {
-                wsel_before += a;
-                wtie_before += t;
-            }
-            cta_sel += a;
-            cta_tie += t;
-        }
+        uint64_t tot2;                                   // (ties, selected) in one scan
+        const uint32_t tie_off = static_cast<uint32_t>(
+            block_excl_scan64<kTkThreads>((static_cast<uint64_t>(n_tie) << 32) | n_sel, sm.wbuf64, &tot2) >> 32);
+        const uint32_t cta_ties = static_cast<uint32_t>(tot2 >> 32), cta_sel = static_cast<uint32_t>(tot2);
         if (tid == 0) {
             sm.xchg[r & 1][0] = cta_sel;
-            sm.xchg[r & 1][1] = cta_tie;
+            sm.xchg[r & 1][1] = cta_ties;
         }
         cluster.sync();
-        // Walk the cluster in position order: ranks, each with its ties
-        // taken while the global tie rank is below `need` (every thread
-        // computes the same bases).
-        uint32_t op = out_base, tp = tie_base, my_op = 0u, my_tp = 0u;
-        for (int q = 0; q < C; ++q) {
-            const uint32_t *x = cluster.map_shared_rank(&sm.xchg[r & 1][0], q);
-            const uint32_t sq = x[0], tq = x[1];
-            if (q == rank) {
-                my_op = op;
-                my_tp = tp;
+        if (tid == 0) {
+            // Walk the cluster in position order: ranks, each with its ties
+            // taken while the global tie rank is below `need`.
+            uint32_t op = out_base, tp = tie_base;
+            for (int q = 0; q < C; ++q) {
+                const uint32_t *x = cluster.map_shared_rank(&sm.xchg[r & 1][0], q);
+                const uint32_t s = x[0], t = x[1];
+                if (q == rank) {
+                    sm.s_base[0] = op;
+                    sm.s_base[1] = tp;
+                }
+                const uint32_t taken = need > tp ? min(t, need - tp) : 0u;
+                op += s + taken;
+                tp += t;
             }
-            const uint32_t taken = need > tp ? min(tq, need - tp) : 0u;
-            op += sq + taken;
-            tp += tq;
+            sm.s_base[2] = op;
+            sm.s_base[3] = tp;
         }
-        uint32_t tie_rank = my_tp + wtie_before + it_ - n_tie;
-        // this thread's outputs: its selected positions plus its kept ties
-        uint32_t kept = 0u;
-        {
-            uint32_t tr = tie_rank;
-            for (int wi = 0; wi < NW; ++wi) {
-                uint32_t tm = sm.tie[tid * NW + wi];
+        __syncthreads();
+        uint32_t tie_rank = sm.s_base[1] + tie_off;
+        uint32_t n_out = 0u;
+        for (int i = wb; i < we; ++i) {
+            uint32_t m = sm.sel[i];
+            uint32_t tm = sm.tie[i];
+            if (tm) {
                 const uint32_t c = __popc(tm);
-                if (tr + c <= need) {
-                    kept += c;
+                if (tie_rank + c <= need) {
+                    m |= tm;
                 } else {
+                    uint32_t tr = tie_rank;
                     while (tm) {
                         const uint32_t bit = tm & (0u - tm);
                         tm ^= bit;
-                        if (tr < need) ++kept;
+                        if (tr < need) m |= bit;
                         ++tr;
                     }
-                    tr -= c;
                 }
-                tr += c;
+                tie_rank += c;
+                sm.sel[i] = m;
             }
+            n_out += __popc(m);
         }
-        // output offset: selected and kept ties before this thread, in position order
-        const uint32_t mine = n_sel + kept;
-        const uint32_t incl = warp_incl_scan(mine);
-        __syncthreads();                                // the warp totals of the counts above are read
-        if (lane == 31) sm.wsel[warp] = incl;
-        __syncthreads();
-        uint32_t wout_before = 0u;
-        for (int w = 0; w < warp; ++w) wout_before += sm.wsel[w];
-        uint32_t pos_out = my_op + wout_before + incl - mine;
-        for (int wi = 0; wi < NW; ++wi) {
-            uint32_t m = sm.sel[tid * NW + wi];
-            uint32_t tm = sm.tie[tid * NW + wi];
-            while (tm) {                                // keep ties while the global tie rank allows
-                const uint32_t bit = tm & (0u - tm);
-                tm ^= bit;
-                if (tie_rank < need) m |= bit;
-                ++tie_rank;
-            }
+        uint32_t cta_out;
+        uint32_t pos = sm.s_base[0] + block_excl_scan<kTkThreads>(n_out, sm.wbuf, &cta_out);
+        for (int i = wb; i < we; ++i) {
+            uint32_t m = sm.sel[i];
             while (m) {
                 const int bit = __ffs(m) - 1;
                 m &= m - 1u;
-                if (pos_out < static_cast<uint32_t>(k)) {
-                    const int64_t t = t0 + 32 * wi + bit;
-                    orow[pos_out] = static_cast<int32_t>(t);
-                    if (srow_out) srow_out[pos_out] = __ldcg(srow + t);
+                if (pos < static_cast<uint32_t>(k)) {
+                    const int64_t t = w0 + i * 32 + bit;
+                    orow[pos] = static_cast<int32_t>(t);
+                    if (srow_out) srow_out[pos] = __ldcg(srow + t);
                 }
-                ++pos_out;
+                ++pos;
             }
         }
-        out_base = op;
-        tie_base = tp;
-        __syncthreads();                                // the next round rewrites the bitmaps
+        out_base = sm.s_base[2];
+        tie_base = sm.s_base[3];
     }
     cluster.sync();                                     // no CTA leaves while a peer may read its counts
 }

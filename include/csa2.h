@@ -303,10 +303,12 @@ csa2_status csa2_indexer_pool_topk(const void *q_idx, const float *w, int B, int
  *     out[b][j][h] = sum_i softmax_i(scale * <q, key_i>) * key_i
  *     lse[b][j][h] = log sum_i exp(scale * <q, key_i>)
  * With no key at all out = 0 and lse = -inf. Dequantized FP4 entries are
- * exact in f16. q and the window rows are carried in f16 under a power-of-two
- * exponent per 144-channel quarter (chosen from the values), so magnitudes
- * from about 2^-100 to 2^110 keep f16 precision; probabilities are rounded to
- * f16; all sums accumulate in fp32. Logits must stay within fp32 range.
+ * exact in f16. q is carried in f16 under a power-of-two exponent per query
+ * row, and the window rows under one per 64-row tile (each chosen from the
+ * values: none when the largest magnitude lies in [2^-4, 2^15)), so rows
+ * whose largest magnitude lies between about 2^-50 and 2^70 keep f16
+ * precision; probabilities are rounded to f16; all sums accumulate in fp32.
+ * Logits must stay within fp32 range.
  *
  *   q_bf16      device bf16 [B][Sq][16][576]
  *   cache       host pointer; reads kv_fp4 and kv_scale of the owner's cache
@@ -320,9 +322,11 @@ csa2_status csa2_indexer_pool_topk(const void *q_idx, const float *w, int B, int
  *               W = 0 with k = 0 is CSA2_ERR_INVALID_ARG.
  *   out         device float [B][Sq][16][576];  lse device float [B][Sq][16]
  *   ws          device workspace of csa2_sparse_attn_workspace_bytes() bytes,
- *               256-byte aligned (partials of rows split over CTAs; at most
- *               2 x CTAs x 37 KB); clobbered. The size returned for (B, Sq, k)
- *               also covers W = 0.
+ *               256-byte aligned (partials of rows split into runs, one per
+ *               CTA, 37 KB each; rows are split only while all the runs fit
+ *               one wave of CTAs, so at most 2 x SMs partials); clobbered.
+ *               The size returned for (B, Sq, k) also covers W = 0; it is 0
+ *               when no row is split.
  */
 size_t csa2_sparse_attn_workspace_bytes(int B, int Sq, int k);
 csa2_status csa2_sparse_attn_decode(const void *q_bf16, int B, int Sq, int H,

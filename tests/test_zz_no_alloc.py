@@ -53,13 +53,16 @@ def test_noalloc_attention_matches_workspace_entry_point_twice():
 
 def test_noalloc_scratch_bound_and_argument_checks():
     """The partials of any shape fit the library-owned array on this GPU
-    (at most two per CTA of one wave), and argument errors are reported as
-    themselves, before the scratch size is considered; nothing is launched."""
+    (rows are split into runs only while the runs fit one wave, one partial
+    each), and argument errors are reported as themselves, before the scratch
+    size is considered; nothing is launched."""
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
     import ctypes
     from compressed_sparse_attention_quant_b200 import lib
-    assert 0 < lib.sparse_attn_workspace_bytes(65535, 1, 65536) <= lib.NOALLOC_SCRATCH_BYTES
+    sizes = [lib.sparse_attn_workspace_bytes(B, Sq, k) for B in (1, 2, 7, 64, 148, 300, 65535)
+             for Sq in (1, 4) for k in (1, 64, 2048, 65536) if B * Sq <= 65535]
+    assert 0 < max(sizes) <= lib.NOALLOC_SCRATCH_BYTES
     assert lib.sparse_attn_workspace_bytes(65536, 1, 1) == 0            # B * Sq > 65535: unsupported shape
     assert lib.sparse_attn_workspace_bytes(1, 1, 65537) == 0            # k > 65536
     L = lib._L
