@@ -42,9 +42,10 @@ namespace csa2 {
 constexpr int kTkThreads = 1024;
 constexpr int kTkWin = 1 << 17;                  // positions per CTA window
 constexpr int kTkWinWords = kTkWin / 32;
-constexpr int kTkCandCap = 12288;                // candidates kept in shared memory per CTA
+constexpr int kTkCandCap = 4096;                 // candidates kept in shared memory per CTA
 constexpr int kTkMaxCluster = 16;
 constexpr int kTkUnroll = 4;                     // float4 loads in flight per thread
+constexpr int kTkGrp = 4 * kTkThreads * kTkUnroll; // positions of one pass-A group (64 KB of scores)
 
 // Zeroes the per-row level-1 histograms before the indexer accumulates them.
 __global__ void __launch_bounds__(256) topk_zero_kernel(uint4 *__restrict__ p, int64_t n16) {
@@ -226,10 +227,12 @@ __device__ __forceinline__ void warp_pick(const uint32_t *h, int nbins, uint32_t
 }
 
 struct TkSmem {
+    alignas(128) float ring[2][kTkGrp]; // 128 KB: scores of pass-A groups, filled by bulk copies ahead
+    uint64_t ring_full[2];
     uint32_t sel[kTkWinWords];          // 16 KB: selected positions of the window
     uint32_t tie[kTkWinWords];          // 16 KB: positions whose key equals the threshold
-    uint32_t ckey[kTkCandCap];          // 48 KB: candidate keys (bin b1)
-    int32_t cpos[kTkCandCap];           // 48 KB: candidate positions
+    uint32_t ckey[kTkCandCap];          // 16 KB: candidate keys (bin b1)
+    int32_t cpos[kTkCandCap];           // 16 KB: candidate positions
     uint32_t hloc[2][kTopkBins];        // this CTA's level-2 / level-3 histograms (read by peers)
     uint32_t hsum[kTopkBins];           // cluster-wide sum of the current level
     uint32_t wbuf[kTkThreads / 32 + 1];
@@ -302,6 +305,12 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
     const int rank = static_cast<int>(cluster.block_rank());
     const int row = blockIdx.x / C;
     const int tid = threadIdx.x;
+    if (tid == 0) {
+        mbar_init(&sm.ring_full[0], 1);
+        mbar_init(&sm.ring_full[1], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
     pdl_wait();                                         // scores and histograms are complete
     pdl_trigger();
     const int n_valid = topk_n_valid(seq_lens, row, Sq, max_pages);
@@ -324,6 +333,23 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
         w1 = min(w0 + Wn, static_cast<int64_t>(n_valid));
         n_it = w1 > w0 ? static_cast<int>((w1 - w0 + 4 * kTkThreads - 1) / (4 * kTkThreads)) : 0;
     };
+
+    // Single-round rows stream their window's scores through two 64 KB slots
+    // of shared memory (one pass-A group each), filled by bulk copies (no
+    // multicast) issued ahead of the reads: the first two before level 1.
+    int64_t fw0 = 0, fw1 = 0;
+    int fn_it = 0;
+    if (fast) win(0, fw0, fw1, fn_it);
+    const int n_grp = (fn_it + kTkUnroll - 1) / kTkUnroll;
+    auto issue_grp = [&](int gi) {
+        const int64_t p0 = fw0 + static_cast<int64_t>(gi) * kTkGrp;
+        const int64_t cnt = min(static_cast<int64_t>(kTkGrp), fw1 - p0);
+        const uint32_t bytes = static_cast<uint32_t>((cnt * 4 + 15) & ~static_cast<int64_t>(15));
+        mbar_arrive_expect_tx(&sm.ring_full[gi & 1], bytes);
+        bulk_g2s(sm.ring[gi & 1], srow + p0, bytes, &sm.ring_full[gi & 1], l2_policy_evict_first());
+    };
+    if (tid == 0)
+        for (int gi = 0; gi < min(2, n_grp); ++gi) issue_grp(gi);
 
     for (int i = tid; i < 2 * kTopkBins; i += kTkThreads) (&sm.hloc[0][0])[i] = 0u;
     if (tid == 0) sm.n_cand = 0u;
@@ -348,10 +374,20 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
         win(r, w0, w1, n_it);
         for (int i0 = 0; i0 < n_it; i0 += kTkUnroll) {
             float4 f[kTkUnroll];
+            const int gi = i0 / kTkUnroll;
+            if (fast) {
+                // positions past w1 in the slot are stale and masked below
+                mbar_wait_bounded(&sm.ring_full[gi & 1], static_cast<uint32_t>((gi >> 1) & 1));
+                const float4 *slot = reinterpret_cast<const float4 *>(sm.ring[gi & 1]);
 #pragma unroll
-            for (int u = 0; u < kTkUnroll; ++u)
-                f[u] = tk_load(srow, w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) + tid * 4, w1,
-                               i0 + u < n_it);
+                for (int u = 0; u < kTkUnroll; ++u)
+                    f[u] = i0 + u < n_it ? slot[u * kTkThreads + tid] : make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+#pragma unroll
+                for (int u = 0; u < kTkUnroll; ++u)
+                    f[u] = tk_load(srow, w0 + static_cast<int64_t>(i0 + u) * (4 * kTkThreads) + tid * 4, w1,
+                                   i0 + u < n_it);
+            }
             uint32_t cmask = 0u;                         // 4 bits per unrolled load
 #pragma unroll
             for (int u = 0; u < kTkUnroll; ++u) {
@@ -427,6 +463,10 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
                     }
                     ++base;
                 }
+            }
+            if (fast) {
+                __syncthreads();                         // every thread has read slot gi & 1
+                if (tid == 0 && gi + 2 < n_grp) issue_grp(gi + 2);
             }
         }
     }
