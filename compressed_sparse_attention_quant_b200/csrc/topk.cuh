@@ -13,11 +13,13 @@
 // exceeds C * 2^17 positions).
 //   level 1  the indexer already built the row's histogram of the top 11 key
 //            bits: every CTA finds the bin b1 holding the k-th largest key.
-//   pass A   one read of the CTA's scores (L2-resident): keys in bins above
-//            b1 are certainly selected and set bits of a shared-memory
-//            bitmap over the window; keys in bin b1 are candidates, counted
-//            into a histogram of their next 11 bits and kept (key, position)
-//            in shared memory while they fit.
+//   pass A   one read of the CTA's scores (L2-resident; a single-round
+//            window streams through two 64 KB shared-memory slots filled by
+//            bulk copies issued ahead, the first two before level 1): keys in
+//            bins above b1 are certainly selected and set bits of a
+//            shared-memory bitmap over the window; keys in bin b1 are
+//            candidates, counted into a histogram of their next 11 bits and
+//            kept (key, position) in shared memory while they fit.
 //   level 2/3 the CTAs sum their histograms through distributed shared
 //            memory (every CTA reads every peer's), so each CTA picks the same
 //            digit; level 3 is skipped when the level-2 bin is taken whole.
@@ -25,7 +27,8 @@
 //            equal to it go to a tie bitmap; one exchange of (selected, ties)
 //            counts across the cluster gives each CTA its first tie rank and
 //            output offset, ties are taken lowest position first, and each
-//            thread writes the positions of its contiguous bitmap words.
+//            thread writes the positions of its contiguous bitmap words (and,
+//            when asked, their scores: the context-parallel candidates).
 // If some CTA's candidates overflow its shared list, or the row needs more
 // than one round, the levels and the emission re-read the scores instead of
 // the list (same result, more L2 reads). Cluster barriers are the only
