@@ -107,25 +107,33 @@ inline cudaError_t launch_quant_kv_fp4(const void *x, int64_t n_tok, const int32
 // value nearest to the exact quotient x / sigma (one rounding, ties to even,
 // saturating, canonical +0), all codes 0 (and sigma 0) for an all-zero row.
 //
-// Exact rounding without a division per channel: p = RN(|x| * RN(1 / sigma))
-// is within 2 binary32 ulps of the exact quotient, so the hardware RNE
-// conversion of p can differ from the exact decision only when an E4M3
-// midpoint lies within those ulps of p. Such channels (the low 20 bits of p
-// within 3 of a midpoint's pattern, or p in the E4M3 subnormal range) take a
-// fix-up that decides the side by the sign of fma(midpoint, sigma, -|x|): the
-// product is exact in the fma and a single rounding keeps the sign. Rows with
+// Exact rounding without a division per channel: p = RN(|x| * r), r an
+// approximation of 1 / sigma to ~1 ulp, lies within 2^-22 (relative) of the
+// exact quotient q. The codes of lo = RN(p (1 - 2^-21)) < q and
+// hi = RN(p (1 + 2^-21)) > q are taken by the hardware RNE satfinite E4M3
+// conversion; rounding is monotone, so when they agree that code is the
+// exact decision for q. When they differ (an E4M3 midpoint lies between them:
+// a fraction of a percent of the channels) a fix-up decides the side by the
+// sign of fma(midpoint, sigma, -|x|), which is exact. Rows with
 // sigma < 2^-100 are first scaled by 2^64 (exact), so no product of the
 // fix-up underflows.
 //
-// Eight threads per row, each with 8 channels; a thread runs kIdxQuantRows
-// rows per pass with all their 16-byte loads issued first, so more bytes are
-// in flight per warp. HBM-bound: 128 B read + 68 B written per row.
+// Four threads per row; thread t of a row takes channels 8t .. 8t + 7 and
+// 32 + 8t .. 32 + 8t + 7 (two 16-byte loads, each warp load covering whole
+// 64-byte runs of its 8 rows); each thread keeps kIdxQuantStages rows in
+// flight (cp.async into its own shared-memory slots). The
+// codes are packed four at a time: magnitudes from the paired conversions,
+// signs from the high bytes of the bf16 inputs, and a sign only on a nonzero
+// magnitude (canonical +0). 128 B read + 68 B written per row; as built the
+// per-row chain (maximum, shuffles, scale, reciprocal, conversions) bounds
+// it at about half of the copy bandwidth, not the HBM.
 constexpr int kIdxQuantThreads = 256;
-constexpr int kIdxQuantRows = 4;                                   // rows per thread per pass
-constexpr int kIdxQuantRowsPerBlock = kIdxQuantThreads / 8 * kIdxQuantRows;
+constexpr int kIdxQuantStages = 4;                                 // rows per thread in flight
+constexpr int kIdxQuantTpr = 4;                                    // threads per row
+constexpr int kIdxQuantRowsPerBlock = kIdxQuantThreads / kIdxQuantTpr;
 
 // E4M3FN magnitude code of the exact quotient a / s (a >= 0, s > 0 binary32,
-// s >= 2^-100), given p = a * RN(1 / s) rounded once.
+// s >= 2^-100), given p = a * r rounded once with r within a few ulps of 1 / s.
 __device__ __forceinline__ uint32_t e4m3_quotient_fixup(float a, float s, float p) {
     if (p >= 448.0f) return 0x7Eu;
     if (p < 0.015625f) {                                           // E4M3 subnormal range: steps of 2^-9
@@ -141,80 +149,113 @@ __device__ __forceinline__ uint32_t e4m3_quotient_fixup(float a, float s, float 
     return d > 0.0f ? clo : d < 0.0f ? chi : ((clo & 1u) ? chi : clo);
 }
 
-// Whether RNE(p) may differ from the exact decision (see above).
-__device__ __forceinline__ bool e4m3_quotient_near(float p) {
-    const uint32_t b = __float_as_uint(p);
-    const bool mid = ((b - 0x7FFFDu) & 0xFFFFFu) <= 6u;            // within 3 ulps of an E4M3 midpoint
-    const bool sub = b - 0x3A000000u < 0x3C800000u - 0x3A000000u;  // p in [2^-11, 2^-6)
-    return mid || sub;
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
 
-__global__ void __launch_bounds__(kIdxQuantThreads, 4)
+// Two E4M3FN codes (RNE, satfinite) of a pair of non-negative floats, low
+// byte first, in the low 16 bits.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+    return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
+__global__ void __launch_bounds__(kIdxQuantThreads, 3)
 quant_index_fp8_kernel(const uint4 *__restrict__ x, int64_t n_rows, uint2 *__restrict__ codes,
                        float *__restrict__ sigma) {
     pdl_wait();
     pdl_trigger();
-    const int lane = threadIdx.x & 31, part = threadIdx.x & 7;
-    const unsigned gmask = 0xffu << (lane & 24);        // the 8 lanes of this row
-    const int64_t stride = static_cast<int64_t>(gridDim.x) * kIdxQuantRowsPerBlock;
-    for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * kIdxQuantRowsPerBlock + (threadIdx.x >> 3);
-         row0 < n_rows; row0 += stride) {
-        uint4 v[kIdxQuantRows];
+    const int lane = threadIdx.x & 31, part = threadIdx.x & (kIdxQuantTpr - 1);
+    const unsigned gmask = 0xfu << (lane & 28);         // the 4 lanes of this row
+    // Each thread keeps its next kIdxQuantStages rows in flight with cp.async
+    // into its own shared-memory slots (no registers held, no barrier: a
+    // thread reads only what it copied).
+    __shared__ __align__(16) uint4 stage[kIdxQuantStages][kIdxQuantThreads][2];
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * (kIdxQuantThreads / kIdxQuantTpr);
+    const int64_t row0 = static_cast<int64_t>(blockIdx.x) * (kIdxQuantThreads / kIdxQuantTpr) + threadIdx.x / kIdxQuantTpr;
+    auto fetch = [&](int64_t k) {                       // row row0 + k * stride into stage k % kIdxQuantStages
+        const int64_t row = row0 + k * stride;
+        const bool ok = row < n_rows;
+        const uint4 *src = ok ? x + row * 8 + part : x;
 #pragma unroll
-        for (int r = 0; r < kIdxQuantRows; ++r) {
-            const int64_t row = row0 + r * (kIdxQuantThreads / 8);
-            v[r] = row < n_rows ? x[row * 8 + part] : make_uint4(0u, 0u, 0u, 0u);
-        }
+        for (int h = 0; h < 2; ++h)
+            cp_async16(&stage[k % kIdxQuantStages][threadIdx.x][h], src + 4 * h, ok ? 16u : 0u);
+    };
 #pragma unroll
-        for (int r = 0; r < kIdxQuantRows; ++r) {
-            const int64_t row = row0 + r * (kIdxQuantThreads / 8);
-            const uint32_t w[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
-            float f[8];
+    for (int k = 0; k < kIdxQuantStages - 1; ++k) {
+        fetch(k);
+        cp_async_commit();
+    }
+    for (int64_t k = 0; row0 + k * stride < n_rows; ++k) {
+        fetch(k + kIdxQuantStages - 1);
+        cp_async_commit();
+        cp_async_wait<kIdxQuantStages - 1>();           // row k has landed
+        {
+            const int64_t row = row0 + k * stride;
+            const uint4 va = stage[k % kIdxQuantStages][threadIdx.x][0];
+            const uint4 vb = stage[k % kIdxQuantStages][threadIdx.x][1];
+            const uint32_t w[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+            float f[16];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 8; ++i) {
                 f[2 * i] = __uint_as_float(w[i] << 16);
                 f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
             }
             float amax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
-#pragma unroll
-            for (int off = 1; off < 8; off <<= 1) amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, off));
-            const float sg = __fdiv_rn(amax, 448.0f);
-            // Scaled domain for tiny sigma (exact power-of-two scaling).
+            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+            amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(gmask, amax, 2));
+            // sigma = RN(amax / 448): one rounded product and one fma
+            // correction (equal to the IEEE quotient for every finite bf16
+            // amax, checked exhaustively on the host).
+            const float q0 = __fmul_rn(amax, 1.0f / 448.0f);
+            const float sg = __fmaf_rn(__fmaf_rn(-q0, 448.0f, amax), 1.0f / 448.0f, q0);
+            // Scaled domain for tiny sigma (exact power-of-two scaling): a =
+            // |x| scl, s2 = sigma scl, p = a / s2 through inv = scl / s2;
+            // below 2^-120 the inputs themselves are scaled (inv would overflow).
             const float scl = sg < 0x1p-100f ? 0x1p64f : 1.0f;
             const float s2 = sg * scl;
-            const float inv = __frcp_rn(s2);
-            float a[8], p[8];
+            float inv = rcp_approx(s2) * scl, ascl = scl;
+            if (sg < 0x1p-120f) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) f[i] *= scl;
+                inv = rcp_approx(s2);
+                ascl = 1.0f;
+            }
+            uint32_t mag[8];                                    // code pairs (2i, 2i + 1)
             uint32_t near = 0u;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                a[i] = fabsf(f[i]) * scl;
-                p[i] = a[i] * inv;
-                near |= e4m3_quotient_near(p[i]) ? (1u << i) : 0u;
+                const float p0 = fabsf(f[2 * i]) * inv, p1 = fabsf(f[2 * i + 1]) * inv;
+                const uint32_t lo = e4m3x2(p0 * 0.99999952316284180f, p1 * 0.99999952316284180f);   // 1 - 2^-21
+                const uint32_t hi = e4m3x2(p0 * 1.00000047683715820f, p1 * 1.00000047683715820f);   // 1 + 2^-21
+                mag[i] = lo;
+                near |= lo != hi ? (1u << i) : 0u;
             }
-            uint32_t mag[8];
-#pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-                const uint32_t c2 = __nv_cvt_float2_to_fp8x2(make_float2(p[i], p[i + 1]), __NV_SATFINITE, __NV_E4M3);
-                mag[i] = c2 & 0x7Fu;
-                mag[i + 1] = (c2 >> 8) & 0x7Fu;
-            }
-            if (__any_sync(0xffffffffu, near != 0u)) {                 // rare: exact fix-up of close calls
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    if (near & (1u << i)) mag[i] = e4m3_quotient_fixup(a[i], s2, p[i]);
-            }
-            uint32_t packed[2] = {0u, 0u};
-            if (sg != 0.0f) {
+            if (__any_sync(0xffffffffu, near != 0u)) {          // rare: exact fix-up of close calls
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const uint32_t c = mag[i] | ((mag[i] != 0u && f[i] < 0.0f) ? 0x80u : 0u);   // canonical +0
-                    packed[i >> 2] |= c << (8 * (i & 3));
+                    if (near & (1u << i)) {
+                        const float a0 = fabsf(f[2 * i]) * ascl, a1 = fabsf(f[2 * i + 1]) * ascl;
+                        const float p0 = fabsf(f[2 * i]) * inv, p1 = fabsf(f[2 * i + 1]) * inv;
+                        mag[i] = e4m3_quotient_fixup(a0, s2, p0) | (e4m3_quotient_fixup(a1, s2, p1) << 8);
+                    }
+                }
+            }
+            uint32_t o[4] = {0u, 0u, 0u, 0u};
+            if (sg != 0.0f) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t m4 = __byte_perm(mag[2 * j], mag[2 * j + 1], 0x5410);     // 4 magnitudes
+                    const uint32_t sgn = __byte_perm(w[2 * j], w[2 * j + 1], 0x7531) & 0x80808080u;
+                    o[j] = m4 | (sgn & __vcmpne4(m4, 0u));                                  // canonical +0
                 }
             }
             if (row < n_rows) {
-                codes[row * 8 + part] = make_uint2(packed[0], packed[1]);
+                codes[row * 8 + part] = make_uint2(o[0], o[1]);           // channels 8t .. 8t + 7
+                codes[row * 8 + 4 + part] = make_uint2(o[2], o[3]);       // channels 32 + 8t ..
                 if (part == 0) sigma[row] = sg;
             }
         }
