@@ -143,16 +143,14 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
 }
 
 // Bounded wait on an mbarrier phase. Returns false (and flags a timeout) if
-// the phase did not complete within kWaitLimitNs. try_wait itself blocks for
-// a short hardware-defined time before it reports "not yet", so the loop
-// does not spin hot; the clock is read every 64 probes. (A long suspend-time
-// hint was measured to delay the wake-up well past the phase's completion.)
+// the phase did not complete within kWaitLimitNs. After a first probe the
+// thread sleeps between probes, so idle warps leave the issue slots free.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
-    for (uint32_t n = 1;; ++n) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((n & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
             flag_status(kStatusTimeout);
             return false;
         }

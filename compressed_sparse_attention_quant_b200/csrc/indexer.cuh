@@ -36,8 +36,7 @@
 //        weights, stores the scores (128-byte coalesced, L2 evict-last: the
 //        selection re-reads them) and adds each valid score's top 11 key
 //        bits to a shared-memory histogram per query row (rows past the
-//        shared slots go straight to the global histogram); lanes of a warp
-//        with the same bin add their count with one atomic.
+//        shared slots go straight to the global histogram).
 // Every wait is a bounded mbarrier wait that sleeps between probes; a
 // timeout sets the status word, stops the pipeline and the producer waits
 // (bounded) for its copies before the CTA exits.
@@ -412,8 +411,6 @@ indexer_score_kernel(const IdxArgs A) {
 #pragma unroll
                         for (int h = 0; h < 4; ++h) score += wq[qq][h] * fmaxf(0.0f, sig[hf] * acc[qq * 4 + h]);
                         st_policy(srow + qq * A.t_cap, score, pol_keep);
-                        // Scores crowd into few bins: lanes with the same bin add
-                        // their count with one atomic (the lowest such lane).
                         if (t <= cur_T - Sq + qq) {
                             const uint32_t bin = float_key(score) >> kTopkDigitShift;
                             const int hr = hrow0 + qq;
