@@ -6,36 +6,45 @@
 // 架构拆解…" (blog.zulogic.cn), section 4 (a 128-token window kept per layer
 // beside the global compressed state).
 //
-// One CTA (8 warps, two CTAs per SM) per (query token, split of its key
-// list). The key list is the k selected positions followed by the 128 window
-// rows; a split owns a run of at most 12 tiles of 64 keys.
-//   set-up   the query row is read with 16-byte loads, rounded to f16 and
-//            stored in shared memory in the QK operand order (qk_pos), from
-//            where each warp takes its fragments with ldmatrix; the split's
-//            selected positions are resolved once to physical cache slots
-//            (top-k index -> page table) in a shared table;
-//   prefetch cp.async (16-byte and 4-byte LDGSTS, zero-filled for empty
-//            slots) fetches the next tile's packed FP4 records and scales as
-//            soon as the current tile's QK has consumed them, overlapping the
-//            softmax and PV;
+// Work: the key list of a query row is its k selected entries in ceil(k/64)
+// tiles of 64 keys (the last one padded) followed by its 128 window rows in two
+// tiles of their own (none when the caller passes no window). Each row's tiles
+// are split into S runs, one CTA each (8 warps, two CTAs per SM), S chosen by
+// the host so that all CTAs fit one wave. A run writes the row's result when
+// S = 1; else an unnormalised partial (m, l, O) that K5 merges.
+//   set-up   before waiting for the selection of the previous kernel (the
+//            query is an input): the query row is rounded to f16 while its
+//            largest magnitude is taken, and written again under 2^-eq in the
+//            rare case that it asks for a power-of-two exponent eq != 0; it is
+//            stored in the QK operand order (qk_pos) and each warp takes its
+//            fragments with ldmatrix. The run's selected positions are then
+//            resolved to physical cache slots 12 tiles at a time (top-k index
+//            -> page table, all loads of a chunk in flight);
+//   prefetch cp.async (16-byte and 4-byte LDGSTS, zero-filled for padding)
+//            fetches the next tile's packed FP4 records and scales as soon as
+//            the current tile's QK has consumed them, overlapping the softmax
+//            and PV;
 //   QK       warp (32-key group, 144-channel quarter): each lane converts the
 //            FP4 bytes of its key (hardware E2M1x2 -> f16x2, E4M3 -> f16 and
 //            one exact f16 multiply) directly into m16n8k16 B fragments, and
 //            stores the same f16 values into a [64][576] tile whose 16-byte
-//            chunks are XOR-swizzled by key; the query fragments stay in
-//            registers; the quarters are summed through shared memory. Tiles
-//            holding window rows (bf16 loads rounded to f16), padding, or the
-//            end of the selected list are first written to the f16 tile by
-//            all threads, and QK reads its fragments from there;
-//   softmax  two heads per warp, warp-shuffle max / sum in the exp2 domain,
-//            probabilities rounded to f16 (the same values feed the sum) and
-//            written over partial rows that no other warp reads, so three
-//            CTA barriers per tile remain (data in, QK done, P ready);
+//            chunks are XOR-swizzled by key; the quarters are summed through
+//            shared memory. Window tiles are first written to the f16 tile by
+//            all threads (bf16 -> f16 while the tile's largest magnitude is
+//            taken, again under 2^-ew in the rare other case), and QK reads
+//            its fragments from there;
+//   softmax  two heads per warp, warp-shuffle max / sum in the exp2 domain
+//            (logits carry 2^(eq + ew)), probabilities rounded to f16 (the
+//            same values feed the sum) and written over partial rows that no
+//            other warp reads, so three CTA barriers per tile remain (data in,
+//            QK done, P ready);
 //   PV       warp w owns 72 output channels; ldmatrix.trans of the f16 tile
-//            is the value operand.
+//            is the value operand; a window tile's exponent scales O around
+//            its products.
 // Warp-level mma.sync is used deliberately: with 16 heads the MMA N extent is
-// 16, and at that width the warp MMAs issue faster than tcgen05 single-thread
-// MMAs. Splits write unnormalised partials (m, l, O) that K5 merges.
+// 16; measured on the B200, one tcgen05 kind::f16 M128 N16 K16 MMA costs ~45
+// cycles (728 useful MAC/clk/SM) while mma.sync m16n8k16 sustains 1024
+// MAC/clk/SM with its operands in registers.
 #pragma once
 
 #include "common.cuh"
