@@ -310,10 +310,13 @@ def pool_leg(args, wl, dw, lib, flush, stream, hbm) -> dict:
 def time_steps(dw, args, flush, stream):
     """Mean device time (ms) of one whole step of a DeviceWorkload: W untimed
     warm-up steps, then K steps, each preceded by an untimed L2 flush, CUDA
-    events on the launching stream around each step."""
+    events on the launching stream around each step. The step is the
+    workload's CUDA graph (one replay launches every kernel of the step)
+    unless --eager."""
+    run = dw.step if args.eager else dw.capture().replay
     for _ in range(args.warmup):
         flush.zero_()
-        dw.step()
+        run()
     torch.cuda.synchronize()
     evs = []
     for _ in range(args.steps):
@@ -322,7 +325,7 @@ def time_steps(dw, args, flush, stream):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        dw.step()
+        run()
         e1.record(stream)
         evs.append((e0, e1))
     torch.cuda.synchronize()
@@ -454,6 +457,7 @@ def replay_leg(args, wl, stream, hbm) -> dict:
 
 def run_gpu(args, wl):
     from compressed_sparse_attention_quant_b200 import lib, workload
+    from compressed_sparse_attention_quant_b200.group import StepGraph
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -495,6 +499,17 @@ def run_gpu(args, wl):
     for _ in range(args.warmup):
         flush.zero_()
         step_instrumented([])
+    # The timed step: the whole group step as one CUDA graph (the same
+    # kernels, their programmatic overlap kept as graph edges), or the eager
+    # library calls with --eager.
+    if args.eager:
+        run_step, per_step = dw.step, None
+    else:
+        sg = dw.capture()
+        run_step, per_step = sg.replay, sg.launches
+        for _ in range(args.warmup):
+            flush.zero_()
+            run_step()
     torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
@@ -515,10 +530,12 @@ def run_gpu(args, wl):
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            dw.step()
+            run_step()
             e1.record(stream)
             step_events.append((e0, e1))
-        launches = lib.launch_count() - launches0
+        # library kernels launched in the region: counted at each launch call
+        # when eager, and per replay from the capture when graphed
+        launches = lib.launch_count() - launches0 if per_step is None else per_step * args.steps
         torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize(dev)
         for _ in range(args.steps):
@@ -564,6 +581,15 @@ def run_gpu(args, wl):
     down_done = [torch.cuda.Event() for _ in range(2)]
     used = [False, False]
 
+    # One CUDA graph of the step per buffer set (graphs read and write the
+    # tensors they were captured with); eager calls with --eager.
+    if args.eager:
+        e2e_graphs = None
+    else:
+        e2e_graphs = [StepGraph(g, dw.page_table, dw.seq_lens, dev_in[s]["q"], dw.swa, dev_in[s]["q_idx"],
+                                dev_in[s]["w"], dev_in[s]["append"], out=dev_out[s][0], lse=dev_out[s][1])
+                      for s in range(2)]
+
     def e2e_step(i):
         s = i % 2
         with torch.cuda.stream(ustream):
@@ -575,8 +601,11 @@ def run_gpu(args, wl):
         stream.wait_event(up_done[s])
         if used[s]:
             stream.wait_event(down_done[s])             # step i-2's outputs have left this set
-        g.step(dw.page_table, dw.seq_lens, dev_in[s]["q"], dw.swa, dev_in[s]["q_idx"], dev_in[s]["w"],
-               dev_in[s]["append"], out=dev_out[s][0], lse=dev_out[s][1])
+        if e2e_graphs is None:
+            g.step(dw.page_table, dw.seq_lens, dev_in[s]["q"], dw.swa, dev_in[s]["q_idx"], dev_in[s]["w"],
+                   dev_in[s]["append"], out=dev_out[s][0], lse=dev_out[s][1])
+        else:
+            e2e_graphs[s].replay()
         comp_done[s].record(stream)
         with torch.cuda.stream(dstream):
             dstream.wait_event(comp_done[s])
@@ -639,7 +668,9 @@ def run_gpu(args, wl):
                    "l2": "inputs > L2; plus 256 MB L2 flush between steps (untimed)"
                    if not args.no_flush else "inputs > L2, no flush",
                    "e2e": "pinned H2D inputs + D2H outputs every step, double-buffered on upload / "
-                          "download streams overlapping compute; working set > L2, no flush"},
+                          "download streams overlapping compute; working set > L2, no flush",
+                   "launch": "eager library calls" if args.eager else
+                             "the step's library kernels replayed as one CUDA graph"},
         "step_hbm_gbs": acct["total"] / (step_ms * 1e-3) / 1e9,
         "step_frac_of_8tbs": acct["total"] / (step_ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS,
         "step_frac_of_measured_copy": acct["total"] / (step_ms * 1e-3) / 1e9 / hbm,
@@ -729,6 +760,7 @@ def main():
     ap.add_argument("--workload", default="decode_b64_t128k",
                     choices=sorted(inputs.WORKLOADS) + sorted(inputs.PROFILE_WORKLOADS))
     ap.add_argument("--no-flush", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager library calls instead of the step's CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work (cpu_baseline)")
     ap.add_argument("--ref-seqs", type=int, default=2, help="sequences the oracle arm prepares")

@@ -98,3 +98,29 @@ class LayerGroup:
                                  out=self._index[li], ws=self.ws_idx)
             lib.sparse_attn_decode(q[li], cache, page_table, seq_lens, self.index(li), swa[li], self.scale,
                                    out=out[li], lse=lse[li], ws=self.ws_att)
+
+
+class StepGraph:
+    """One decode step of a LayerGroup captured once as a CUDA graph and then
+    replayed with a single launch: the same library kernels in the same order,
+    the programmatic-dependent-launch overlap between consecutive kernels kept
+    as graph edges, and no host work per kernel. The graph reads and writes the
+    tensors given at capture time, so a caller refreshes those in place between
+    replays (new query rows, new tokens to append, new page-table entries).
+
+    The first eager step runs before the capture so that the library's one-time
+    device set-up does not happen while the stream is being captured.
+    """
+
+    def __init__(self, group: LayerGroup, *step_args, **step_kwargs):
+        group.step(*step_args, **step_kwargs)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        n0 = lib.launch_count()
+        with torch.cuda.graph(self.graph):
+            group.step(*step_args, **step_kwargs)
+        self.launches = lib.launch_count() - n0          # library kernels per replay
+
+    def replay(self) -> None:
+        """Enqueue the captured step on the current stream."""
+        self.graph.replay()

@@ -9,7 +9,7 @@ from typing import Dict, List
 import torch
 
 from . import inputs, lib
-from .group import LayerGroup
+from .group import LayerGroup, StepGraph
 
 
 class DeviceWorkload:
@@ -60,6 +60,11 @@ class DeviceWorkload:
 
     def step(self) -> None:
         self.group.step(self.page_table, self.seq_lens, self.q, self.swa, self.q_idx, self.w, self.append)
+
+    def capture(self) -> StepGraph:
+        """The step as a CUDA graph over this workload's resident tensors."""
+        return StepGraph(self.group, self.page_table, self.seq_lens, self.q, self.swa, self.q_idx, self.w,
+                         self.append)
 
     # ------------------------------------------------------------ accounting
     def algorithmic_bytes(self) -> Dict[str, float]:
