@@ -257,9 +257,16 @@ indexer_score_kernel(const IdxArgs A) {
             const uint32_t todo = __ballot_sync(0xffffffffu, live);
             const int rank = __popc(todo & ((1u << lane) - 1u));
             // Issue in chunks of S ring positions: a lane only waits on a slot
-            // filled by an earlier chunk.
-            for (int c0 = 0; c0 < __popc(todo); c0 += S) {
-                if (live && rank >= c0 && rank < c0 + S) {
+            // filled by an earlier chunk. The launch's first chunk goes one
+            // unit at a time (all of rank r's copies before rank r + 1's): the
+            // SM's bulk-copy engine takes copies in issue order, so the first
+            // unit lands after its own copies instead of after the whole first
+            // wave's. Later chunks issue together (lanes whose slots are free
+            // do not wait for one another).
+            const int n_live = __popc(todo);
+            for (int r0 = 0; r0 < n_live;) {
+                const int r1 = (n_issued == 0 && r0 < S) ? r0 + 1 : min(r0 - r0 % S + S, n_live);
+                if (live && rank >= r0 && rank < r1) {
                     const int64_t i = n_issued + rank;
                     const int s = static_cast<int>(i % S);
                     if (slot_wait(i)) {
@@ -282,6 +289,7 @@ indexer_score_kernel(const IdxArgs A) {
                 }
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
+                r0 = r1;
             }
             n_issued += __popc(todo);
             cur = nxt;
@@ -311,7 +319,20 @@ indexer_score_kernel(const IdxArgs A) {
         constexpr uint32_t idesc = umma_idesc(128, kIdxAccCols, false, false);   // E4M3 x E4M3, fp32
         uint8_t *qop = sm.qop[mw];
         const uint32_t q_addr = smem_u32(qop);
-        int cur_b = -1, stops = 0;
+        // column n = query token * 4 + head; 16 B chunk c of its 64 channels
+        auto stage_q = [&](int b) {
+            for (int k = lane; k < 4 * Sq * (kIdxDim / 16); k += 32) {
+                const int n = k >> 2, c = k & 3;
+                const uint4 v = *reinterpret_cast<const uint4 *>(
+                    A.q_idx + (static_cast<int64_t>(b) * Sq * kIdxHeads + n) * kIdxDim + c * 16);
+                *reinterpret_cast<uint4 *>(qop + (n >> 3) * 512 + c * 128 + (n & 7) * 16) = v;
+            }
+            fence_proxy_async_smem();                   // generic writes -> tensor-core reads
+            __syncwarp();
+        };
+        // The CTA's first sequence is staged while the first copies are in flight.
+        int cur_b = b_first, stops = 0;
+        stage_q(cur_b);
         uint32_t q_phase = 0u;
         for (int64_t i = mw; stops < kIdxGroups / kIdxMmaWarps; i += kIdxMmaWarps) {
             const int s = static_cast<int>(i % S);
@@ -324,21 +345,11 @@ indexer_score_kernel(const IdxArgs A) {
             if (m.b >= 0 && m.b != cur_b) {
                 // New sequence: every MMA reading the old query must be done
                 // before the operand is rewritten.
-                if (cur_b >= 0) {
-                    if (lane == 0) umma_commit(&sm.q_free[mw]);
-                    if (!warp_wait(&sm.q_free[mw], q_phase)) break;
-                    q_phase ^= 1u;
-                }
+                if (lane == 0) umma_commit(&sm.q_free[mw]);
+                if (!warp_wait(&sm.q_free[mw], q_phase)) break;
+                q_phase ^= 1u;
                 cur_b = m.b;
-                // column n = query token * 4 + head; 16 B chunk c of its 64 channels
-                for (int k = lane; k < 4 * Sq * (kIdxDim / 16); k += 32) {
-                    const int n = k >> 2, c = k & 3;
-                    const uint4 v = *reinterpret_cast<const uint4 *>(
-                        A.q_idx + (static_cast<int64_t>(cur_b) * Sq * kIdxHeads + n) * kIdxDim + c * 16);
-                    *reinterpret_cast<uint4 *>(qop + (n >> 3) * 512 + c * 128 + (n & 7) * 16) = v;
-                }
-                fence_proxy_async_smem();               // generic writes -> tensor-core reads
-                __syncwarp();
+                stage_q(cur_b);
             }
             if (lane == 0) {
                 sm.acc_meta[buf] = m;
@@ -371,6 +382,17 @@ indexer_score_kernel(const IdxArgs A) {
         const uint64_t pol_keep = l2_policy_evict_last();
         int cur_b = -1, cur_T = 0, hrow0 = 0;
         float wq[4][4];
+        auto load_seq = [&](int b) {
+            cur_b = b;
+            cur_T = A.seq_lens[b];
+            hrow0 = (b - b_first) * Sq;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+                    wq[qq][h] = qq < Sq ? A.w[(static_cast<int64_t>(b) * Sq + qq) * kIdxHeads + h] : 0.0f;
+        };
+        load_seq(b_first);                              // while the first copies are in flight
         for (int64_t i = grp;; i += kIdxGroups) {
             const int buf = static_cast<int>(i % kIdxAccBufs);
             if (!warp_wait(&sm.acc_full[buf], static_cast<uint32_t>((i / kIdxAccBufs) & 1))) break;
@@ -388,16 +410,7 @@ indexer_score_kernel(const IdxArgs A) {
             for (int hf = 0; hf < kIdxBlocks; ++hf) sig[hf] = sgp[(2 * hf + (q >> 1)) * kPage + j];
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[m.slot]);
-            if (m.b != cur_b) {
-                cur_b = m.b;
-                cur_T = A.seq_lens[cur_b];
-                hrow0 = (cur_b - b_first) * Sq;
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq)
-#pragma unroll
-                    for (int h = 0; h < 4; ++h)
-                        wq[qq][h] = qq < Sq ? A.w[(static_cast<int64_t>(cur_b) * Sq + qq) * kIdxHeads + h] : 0.0f;
-            }
+            if (m.b != cur_b) load_seq(m.b);
             // Scores of this thread's token in block hf from its accumulator row.
             auto emit = [&](int hf, const float *acc) {
                 const int pg = 2 * hf + (q >> 1);

@@ -117,7 +117,9 @@ class StepGraph:
         torch.cuda.synchronize()
         self.graph = torch.cuda.CUDAGraph()
         n0 = lib.launch_count()
-        with torch.cuda.graph(self.graph):
+        # thread-local capture: other threads (a process group's watchdog) may
+        # keep querying the device while this one captures
+        with torch.cuda.graph(self.graph, capture_error_mode="thread_local"):
             group.step(*step_args, **step_kwargs)
         self.launches = lib.launch_count() - n0          # library kernels per replay
 
