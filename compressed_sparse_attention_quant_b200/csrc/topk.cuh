@@ -314,9 +314,11 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
         fence_mbar_init();
     }
     __syncthreads();
+    // The sequence lengths are an input no earlier kernel of the step writes:
+    // read before the wait.
+    const int n_valid = topk_n_valid(seq_lens, row, Sq, max_pages);
     pdl_wait();                                         // scores and histograms are complete
     pdl_trigger();
-    const int n_valid = topk_n_valid(seq_lens, row, Sq, max_pages);
     int32_t *orow = out + static_cast<int64_t>(row) * k;
     float *srow_out = out_scores ? out_scores + static_cast<int64_t>(row) * k : nullptr;
     const float *srow = scores + static_cast<int64_t>(row) * t_cap;
@@ -586,8 +588,9 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
             n_sel += __popc(sm.sel[i]);
         }
         uint64_t tot2;                                   // (ties, selected) in one scan
-        const uint32_t tie_off = static_cast<uint32_t>(
-            block_excl_scan64<kTkThreads>((static_cast<uint64_t>(n_tie) << 32) | n_sel, sm.wbuf64, &tot2) >> 32);
+        const uint64_t off2 =
+            block_excl_scan64<kTkThreads>((static_cast<uint64_t>(n_tie) << 32) | n_sel, sm.wbuf64, &tot2);
+        const uint32_t tie_off = static_cast<uint32_t>(off2 >> 32), sel_off = static_cast<uint32_t>(off2);
         const uint32_t cta_ties = static_cast<uint32_t>(tot2 >> 32), cta_sel = static_cast<uint32_t>(tot2);
         if (tid == 0) {
             sm.xchg[r & 1][0] = cta_sel;
@@ -614,7 +617,11 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
         }
         __syncthreads();
         uint32_t tie_rank = sm.s_base[1] + tie_off;
-        uint32_t n_out = 0u;
+        // Output offset: the CTA's base, the selected positions before this
+        // thread's words, and the ties before them that are taken (global tie
+        // ranks below need).
+        const uint32_t ties_open = need > sm.s_base[1] ? need - sm.s_base[1] : 0u;
+        uint32_t pos = sm.s_base[0] + sel_off + min(tie_off, ties_open);
         for (int i = wb; i < we; ++i) {
             uint32_t m = sm.sel[i];
             uint32_t tm = sm.tie[i];
@@ -634,10 +641,7 @@ topk_cluster_kernel(const float *__restrict__ scores, int64_t t_cap, const uint3
                 tie_rank += c;
                 sm.sel[i] = m;
             }
-            n_out += __popc(m);
         }
-        uint32_t cta_out;
-        uint32_t pos = sm.s_base[0] + block_excl_scan<kTkThreads>(n_out, sm.wbuf, &cta_out);
         for (int i = wb; i < we; ++i) {
             uint32_t m = sm.sel[i];
             while (m) {
