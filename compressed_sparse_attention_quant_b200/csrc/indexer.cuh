@@ -17,7 +17,10 @@
 //        and each lane with a unit copies its pages (4 KB key pages + 256 B
 //        scale rows, cp.async.bulk without multicast, L2 evict-first) into
 //        the next of S ring slots once that slot is free; the slot's "full"
-//        mbarrier completes with the bytes.
+//        mbarrier completes with the bytes. The launch's first S units are
+//        issued one after another (the SM's bulk-copy engine serves copies
+//        in issue order, so the first unit lands early); later units are
+//        issued together by the lanes whose slots are free.
 //   MMA (2 warps)       units alternate between two issuing threads (the
 //        per-unit waits and the commit, not the tensor core, bound one
 //        thread); each issues, per unit, eight tcgen05.mma kind::f8f6f4
@@ -29,7 +32,8 @@
 //        (t/8)*512 + (c/16)*128 + (t%8)*16 + c%16), the tensor core's
 //        no-swizzle K-major operand layout, so they are used as copied. The
 //        query (column n = query token * 4 + head) is written once per
-//        sequence into the same layout.
+//        sequence into the same layout (the CTA's first sequence while the
+//        first copies are in flight).
 //   epilogue (16 warps) 4 groups of 4 warps take the units in turn; warp q
 //        of a group reads TMEM lanes 32q .. 32q+31 of every block (one token
 //        per thread and block, all heads), applies sigma, ReLU and the head
