@@ -68,3 +68,53 @@ def test_without_pool_every_indexing_layer_scans(rec):
 def test_pool_must_hold_top_k(rec):
     with pytest.raises(ValueError):
         group.LayerGroup(("F", "R"), 1, 1, 4, 8, top_k=64, device="cpu", pool_size=32)
+
+
+def test_step_graph_runs_one_eager_step_then_captures_one(rec, monkeypatch):
+    """StepGraph (CPU, CUDA graph API replaced by recorders): one eager step
+    first (library set-up outside the capture), then exactly one step inside a
+    thread-local capture; the launches counted during the capture are the
+    kernels per replay, and replay() only replays the graph."""
+    events = []
+    counter = {"n": 0}
+
+    class _Graph:
+        def replay(self):
+            events.append("replay")
+
+    class _Capture:
+        def __init__(self, graph, capture_error_mode="global"):
+            events.append(("capture", capture_error_mode))
+
+        def __enter__(self):
+            events.append("enter")
+
+        def __exit__(self, *exc):
+            events.append("exit")
+            return False
+
+    def counting(kind):
+        def f(*a, **k):
+            counter["n"] += 3 if kind == "topk" else 2
+            rec.append((kind,))
+            events.append(kind)
+        return f
+
+    monkeypatch.setattr(torch.cuda, "CUDAGraph", _Graph)
+    monkeypatch.setattr(torch.cuda, "graph", _Capture)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a: events.append("sync"))
+    monkeypatch.setattr(lib, "launch_count", lambda: counter["n"])
+    monkeypatch.setattr(lib, "indexer_topk", counting("topk"))
+    monkeypatch.setattr(lib, "sparse_attn_decode", counting("attn"))
+
+    modes = ("F", "U")
+    g = group.LayerGroup(modes, 2, 1, 4, 8, top_k=4, device="cpu")
+    q, q_idx, w = _inputs(len(modes))
+    sg = group.StepGraph(g, None, None, q, [None] * len(modes), q_idx, w)
+    # eager step, sync, capture (thread-local) of one step
+    assert events == ["topk", "attn", "attn", "sync", ("capture", "thread_local"), "enter",
+                      "topk", "attn", "attn", "exit"]
+    assert sg.launches == 3 + 2 + 2
+    events.clear()
+    sg.replay()
+    assert events == ["replay"]
